@@ -1,0 +1,99 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that at least
+one pin catches each of them. The mutations are undone after every test."""
+
+import math
+
+import numpy as np
+import pytest
+
+import tests.test_oracle_pins as pins
+from oracle import spark_oracle as so
+
+_orig = {name: getattr(so, name) for name in
+         ("summaries", "whitening_factor", "split_direction", "select", "attention",
+          "split_group", "round_bf16", "block_means")}
+
+
+def _beta_without_anchor_term(k, v, perm, qbar, mode="reweight"):
+    kt, vt, beta = _orig["summaries"](k, v, perm, qbar, mode)
+    d = k.shape[1]
+    return kt, vt, beta + kt @ qbar / math.sqrt(d)
+
+
+def _meanpool_without_count(k, v, perm, qbar, mode="reweight"):
+    kt, vt, beta = _orig["summaries"](k, v, perm, qbar, mode)
+    return kt, vt, beta - math.log(64)
+
+
+def _transposed_factor(M):
+    return _orig["whitening_factor"](M).T
+
+
+def _uncentered_direction(U):
+    n, d = U.shape
+    S = U.T @ U / n
+    v = np.full(d, 1 / math.sqrt(d))
+    for _ in range(so.POWER_ITERS):
+        v = S @ v
+        v /= np.linalg.norm(v)
+    mu = U.mean(axis=0)
+    return v, mu, (U - mu) @ v
+
+
+def _select_lowest(qm, km, ksel):
+    return _orig["select"](-qm, km, ksel)
+
+
+def _attention_unscaled(q, k, v, perm, sel, kt, vt, beta, rows=None):
+    s = math.sqrt(q.shape[1])
+    return _orig["attention"](q * s, k, v, perm, sel, kt, vt, beta, rows)
+
+
+def _truncating_round(x):
+    m, e = np.frexp(np.asarray(x, dtype=np.float64))
+    return np.ldexp(np.trunc(np.ldexp(m, 8)), e - 8)
+
+
+def _block_sum_not_mean(x, perm):
+    return _orig["block_means"](x, perm) * 64
+
+
+def _split_ceil_left(U, ids):
+    left, right, info = _orig["split_group"](U, ids)
+    g = len(ids) // 64
+    if g % 2:
+        both = np.concatenate([left, right])
+        left, right = both[: 64 * (g // 2 + 1)], both[64 * (g // 2 + 1):]
+    return left, right, info
+
+
+MUTANTS = [
+    ("summaries", _beta_without_anchor_term, [pins.test_beta_is_entropy_of_anchor_weights]),
+    ("summaries", _meanpool_without_count, [pins.test_compressed_branch_exact_for_identical_keys]),
+    ("whitening_factor", _transposed_factor, [pins.test_whitening_inner_products_are_mahalanobis]),
+    ("split_direction", _uncentered_direction, [pins.test_split_direction_is_top_eigenvector]),
+    ("select", _select_lowest, [pins.test_select_against_full_sort]),
+    ("attention", _attention_unscaled, [pins.test_density_one_is_dense_attention]),
+    ("round_bf16", _truncating_round, [pins.test_round_bf16_matches_bit_rounding]),
+    ("split_group", _split_ceil_left, [pins.test_split_group_orientation_and_capacity]),
+]
+
+
+@pytest.mark.parametrize("name,mutant,catchers", MUTANTS, ids=[m[1].__name__ for m in MUTANTS])
+def test_pins_catch_planted_mistake(monkeypatch, name, mutant, catchers):
+    monkeypatch.setattr(so, name, mutant)
+    caught = 0
+    for t in catchers:
+        try:
+            t()
+        except AssertionError:
+            caught += 1
+    assert caught > 0, f"no pin caught the mutation of {name}"
+
+
+def test_brute_force_catches_block_sum_mistake(monkeypatch):
+    monkeypatch.setattr(so, "block_means", _block_sum_not_mean)
+    # scaling block means by 64 keeps the ranking, so selection pins alone do
+    # not see it; nothing downstream uses the scale, so this checks the pins
+    # stay green for a harmless change (no false alarm)
+    pins.test_oracle_matches_brute_force(256, 8, 0.25, "reweight")

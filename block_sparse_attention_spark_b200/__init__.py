@@ -1,0 +1,245 @@
+"""Spark-Attn block-sparse attention forward pass on B200 (sm_100a).
+
+Thin ctypes binding of libspark (include/spark.h): every function marshals
+torch tensors into pointers and calls the C ABI on the current CUDA stream.
+All arithmetic runs in the library's CUDA kernels; there is no CPU path.
+Build the library first:  python -m block_sparse_attention_spark_b200.build
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = ["SparkError", "Params", "lib", "params", "num_selected", "workspace_size",
+           "host_workspace_size", "workspace_region", "alloc_workspace", "moments", "reblock",
+           "positional_perm", "select", "attn_fwd", "forward", "forward_host", "get_status",
+           "LAYOUTS", "SUMMARIES", "WS"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libspark.so")
+
+LAYOUTS = {"q_reuse_k": 0, "k_reuse_q": 1}
+SUMMARIES = {"reweight": 0, "meanpool": 1}
+WS = {"MQ": 0, "MK": 1, "QMEAN": 2, "PERM": 3, "SEL": 4, "QM": 5, "KM": 6, "KT": 7, "VT": 8,
+      "BETA": 9, "UHAT": 10}
+STATUS = {0: "SPARK_OK", 1: "SPARK_ERR_INVALID_ARG", 2: "SPARK_ERR_UNSUPPORTED",
+          3: "SPARK_ERR_WORKSPACE", 4: "SPARK_ERR_CUDA", 5: "SPARK_ERR_TIMEOUT"}
+
+
+class SparkError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        msg = lib().spark_strerror(code).decode() if _LIB is not None else ""
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({msg})")
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("topk_ratio", ctypes.c_double),
+                ("topk_blocks", ctypes.c_int32), ("layout", ctypes.c_int32),
+                ("summary", ctypes.c_int32), ("tail", ctypes.c_int32)]
+
+    def __repr__(self):
+        return (f"Params(B={self.B}, H={self.H}, N={self.N}, d={self.d}, "
+                f"topk_ratio={self.topk_ratio}, topk_blocks={self.topk_blocks}, "
+                f"layout={self.layout}, summary={self.summary}, tail={self.tail})")
+
+
+_LIB = None
+_P = ctypes.POINTER(Params)
+_vp = ctypes.c_void_p
+_sz = ctypes.c_size_t
+_i32 = ctypes.c_int32
+
+_SIGS = {
+    "spark_validate": (_i32, [_P]),
+    "spark_num_selected": (_i32, [_P]),
+    "spark_workspace_size": (_sz, [_P]),
+    "spark_host_workspace_size": (_sz, [_P]),
+    "spark_workspace_region": (_sz, [_P, _i32, ctypes.POINTER(_sz)]),
+    "spark_moments": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "spark_reblock": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "spark_positional_perm": (_i32, [_P, _i32, _i32, _i32, _vp, _vp]),
+    "spark_select": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "spark_attn_fwd": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "spark_forward": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "spark_forward_host": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "spark_get_status": (_i32, [_vp]),
+    "spark_strerror": (ctypes.c_char_p, [_i32]),
+}
+
+
+def lib():
+    """The loaded libspark (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libspark.so not found at {LIB_PATH}; build it with "
+                               "`python -m block_sparse_attention_spark_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = L
+    return _LIB
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise SparkError(code, where)
+
+
+def params(B, H, N, d, topk_ratio=0.2, topk_blocks=0, layout="q_reuse_k",
+           summary="reweight") -> Params:
+    return Params(B, H, N, d, float(topk_ratio), int(topk_blocks), LAYOUTS[layout],
+                  SUMMARIES[summary], 0)
+
+
+def validate(p: Params) -> int:
+    return lib().spark_validate(ctypes.byref(p))
+
+
+def num_selected(p: Params) -> int:
+    return lib().spark_num_selected(ctypes.byref(p))
+
+
+def workspace_size(p: Params) -> int:
+    return lib().spark_workspace_size(ctypes.byref(p))
+
+
+def host_workspace_size(p: Params) -> int:
+    return lib().spark_host_workspace_size(ctypes.byref(p))
+
+
+def workspace_region(p: Params, name: str):
+    """(byte offset, byte size) of a named workspace region."""
+    n = _sz(0)
+    off = lib().spark_workspace_region(ctypes.byref(p), WS[name], ctypes.byref(n))
+    if off == ctypes.c_size_t(-1).value:
+        raise SparkError(1, "spark_workspace_region")
+    return off, n.value
+
+
+# ---------------------------------------------------------------- torch glue
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream():
+    return _torch().cuda.current_stream().cuda_stream
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _need(t, dtype, shape, name):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}, "
+                        f"got {t.dtype} {tuple(t.shape)}")
+
+
+def alloc_workspace(p: Params, host=False):
+    torch = _torch()
+    n = host_workspace_size(p) if host else workspace_size(p)
+    if n == 0:
+        _check(validate(p) or 1, "workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device="cuda")
+
+
+def ws_view(ws, p: Params, name: str, dtype, shape):
+    """A typed view of one workspace region (no copy)."""
+    off, n = workspace_region(p, name)
+    esz = _torch().tensor([], dtype=dtype).element_size()
+    count = 1
+    for s in shape:
+        count *= s
+    assert count * esz <= n
+    return ws[off:off + count * esz].view(dtype).view(*shape)
+
+
+def moments(p: Params, q, k, ws):
+    torch = _torch()
+    shp = (p.B, p.H, p.N, p.d)
+    _need(q, torch.bfloat16, shp, "q")
+    _need(k, torch.bfloat16, shp, "k")
+    MQ = torch.empty(p.B, p.H, p.d, p.d, dtype=torch.float64, device="cuda")
+    MK = torch.empty_like(MQ)
+    qmean = torch.empty(p.B, p.H, p.d, dtype=torch.float64, device="cuda")
+    _check(lib().spark_moments(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(MQ), _ptr(MK), _ptr(qmean),
+                               _ptr(ws), ws.numel(), _stream()), "spark_moments")
+    return MQ, MK, qmean
+
+
+def reblock(p: Params, q, k, MQ, MK, ws):
+    torch = _torch()
+    perm = torch.empty(p.B, p.H, p.N, dtype=torch.int32, device="cuda")
+    _check(lib().spark_reblock(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(MQ), _ptr(MK), _ptr(perm),
+                               _ptr(ws), ws.numel(), _stream()), "spark_reblock")
+    return perm
+
+
+def positional_perm(p: Params, grid):
+    torch = _torch()
+    F, Hl, Wl = grid
+    perm = torch.empty(p.B, p.H, p.N, dtype=torch.int32, device="cuda")
+    _check(lib().spark_positional_perm(ctypes.byref(p), F, Hl, Wl, _ptr(perm), _stream()),
+           "spark_positional_perm")
+    return perm
+
+
+def select(p: Params, q, k, v, perm, qmean, ws):
+    torch = _torch()
+    ksel = num_selected(p)
+    sel = torch.empty(p.B, p.H, p.N // 64, ksel, dtype=torch.int32, device="cuda")
+    _check(lib().spark_select(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(perm), _ptr(qmean),
+                              _ptr(sel), _ptr(ws), ws.numel(), _stream()), "spark_select")
+    return sel
+
+
+def attn_fwd(p: Params, perm, sel, ws, return_lse=False):
+    torch = _torch()
+    out = torch.empty(p.B, p.H, p.N, p.d, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(p.B, p.H, p.N, dtype=torch.float32, device="cuda") if return_lse else None
+    _check(lib().spark_attn_fwd(ctypes.byref(p), _ptr(perm), _ptr(sel), _ptr(out), _ptr(lse),
+                                _ptr(ws), ws.numel(), _stream()), "spark_attn_fwd")
+    return (out, lse) if return_lse else out
+
+
+def forward(p: Params, q, k, v, ws=None, out=None, lse=None, perm=None, sel=None):
+    """The whole pass on device tensors. Returns out (and writes lse/perm/sel
+    into the given tensors when they are passed)."""
+    torch = _torch()
+    shp = (p.B, p.H, p.N, p.d)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, shp, n)
+    if ws is None:
+        ws = alloc_workspace(p)
+    if out is None:
+        out = torch.empty(shp, dtype=torch.bfloat16, device="cuda")
+    _check(lib().spark_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                               _ptr(perm), _ptr(sel), _ptr(ws), ws.numel(), _stream()),
+           "spark_forward")
+    return out
+
+
+def forward_host(p: Params, q_host, k_host, v_host, out_host, ws, lse_host=None):
+    """The whole pass on host tensors (CPU torch tensors, pinned for speed)."""
+    _check(lib().spark_forward_host(ctypes.byref(p), _ptr(q_host), _ptr(k_host), _ptr(v_host),
+                                    _ptr(out_host), _ptr(lse_host), _ptr(ws), ws.numel(),
+                                    _stream()), "spark_forward_host")
+    return out_host
+
+
+def get_status():
+    """Synchronises the current stream and returns the device status code."""
+    return lib().spark_get_status(_stream())

@@ -1,0 +1,117 @@
+// Step a1: per-head second moments M_Q = E[q q^T], M_K = E[k k^T] and the
+// anchor qbar = E[q] ("MiniMax H3 Spark Attention (SM89)", "What it's doing
+// under the hood"; "Spark-H3" news post, Spark-Reweight bullet).
+//
+// Kernel 1 (moments_partial): grid (splits, B*H, 2 tensors). Each CTA streams
+// a contiguous token range of one head through shared memory (3-stage
+// cp.async pipeline, 16-byte loads) and forms the partial Gram X^T X plus the
+// column sums, float64-accumulated. Kernel 2 (moments_reduce) adds the
+// partials of a head in a fixed order (deterministic) and divides by N.
+#include "gram.cuh"
+#include "plan.h"
+
+namespace spark {
+
+template <int D, int STAGES>
+__global__ void __launch_bounds__(256, 1)
+moments_partial_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, int N,
+                       int blocks_per_split, double* __restrict__ part) {
+  using G = Gram<D>;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  double* acc64 = reinterpret_cast<double*>(smem_raw);
+  uint16_t* tiles = reinterpret_cast<uint16_t*>(smem_raw + sizeof(double) * G::ACC * G::THREADS);
+  __shared__ double colsum_sh[D];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int split = blockIdx.x, bh = blockIdx.y, t = blockIdx.z;
+  const int BH = gridDim.y, splits = gridDim.x;
+  const uint16_t* X = (t == 0 ? q : k) + (size_t)bh * N * D;
+  const int nb = N / BLK;
+  const int b0 = split * blocks_per_split;
+  const int b1 = min(nb, b0 + blocks_per_split);
+  const int ntiles = max(0, b1 - b0);
+
+  for (int j = tid; j < G::ACC * G::THREADS; j += G::THREADS) acc64[j] = 0.0;
+  float acc[G::ACC];
+#pragma unroll
+  for (int j = 0; j < G::ACC; ++j) acc[j] = 0.f;
+  double csum = 0.0;
+
+#pragma unroll
+  for (int s = 0; s < STAGES - 1; ++s) {
+    if (s < ntiles) G::load_tile(tiles + s * G::TILE, X, nullptr, (long)(b0 + s) * BLK, tid);
+    cp_async_commit();
+  }
+  for (int it = 0; it < ntiles; ++it) {
+    cp_async_wait<STAGES - 2>();
+    __syncthreads();
+    const int nxt = it + STAGES - 1;
+    if (nxt < ntiles) G::load_tile(tiles + (nxt % STAGES) * G::TILE, X, nullptr, (long)(b0 + nxt) * BLK, tid);
+    cp_async_commit();
+    const uint16_t* sm = tiles + (it % STAGES) * G::TILE;
+    G::tile_mma(sm, acc, warp, lane);
+    if (tid < D) {
+      double s = 0.0;
+#pragma unroll 8
+      for (int r = 0; r < BLK; ++r) s += (double)bf2f(sm[r * G::RS + tid]);
+      csum += s;
+    }
+    if ((it + 1) % G::FLUSH == 0 || it == ntiles - 1) G::flush(acc, acc64, tid);
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+
+  double* out = part + ((size_t)(t * BH + bh) * splits + split) * (size_t)(D * D + D);
+#pragma unroll 4
+  for (int j = 0; j < G::ACC; ++j) {
+    int row, col;
+    G::coord(j, warp, lane, row, col);
+    out[row * D + col] = acc64[j * G::THREADS + tid];
+  }
+  if (tid < D) out[D * D + tid] = csum;
+  (void)colsum_sh;
+}
+
+template <int D>
+__global__ void moments_reduce_kernel(const double* __restrict__ part, int splits, int N,
+                                      double* __restrict__ MQ, double* __restrict__ MK,
+                                      double* __restrict__ qmean) {
+  const int bh = blockIdx.x, t = blockIdx.y, BH = gridDim.x;
+  const double* src = part + (size_t)(t * BH + bh) * splits * (size_t)(D * D + D);
+  double* M = (t == 0 ? MQ : MK) + (size_t)bh * D * D;
+  const double invN = 1.0 / (double)N;
+  for (int e = threadIdx.x; e < D * D + D; e += blockDim.x) {
+    double s = 0.0;
+    for (int i = 0; i < splits; ++i) s += src[(size_t)i * (D * D + D) + e];
+    if (e < D * D) {
+      M[e] = s * invN;
+    } else if (t == 0) {
+      qmean[(size_t)bh * D + (e - D * D)] = s * invN;
+    }
+  }
+}
+
+template <int D>
+static cudaError_t run_moments(const Plan& pl, const uint16_t* q, const uint16_t* k, double* MQ,
+                               double* MK, double* qmean, void* ws, cudaStream_t s) {
+  constexpr int STAGES = 3;
+  using G = Gram<D>;
+  const size_t smem = sizeof(double) * G::ACC * G::THREADS + sizeof(uint16_t) * G::TILE * STAGES;
+  auto kern = moments_partial_kernel<D, STAGES>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int splits = pl.moment_splits;
+  const int bps = (pl.nb + splits - 1) / splits;
+  double* part = ws_at<double>(ws, pl.off_mpart);
+  kern<<<dim3(splits, pl.BH, 2), G::THREADS, smem, s>>>(q, k, pl.N, bps, part);
+  moments_reduce_kernel<D><<<dim3(pl.BH, 2), 256, 0, s>>>(part, splits, pl.N, MQ, MK, qmean);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_moments(const Plan& pl, const uint16_t* q, const uint16_t* k, double* MQ,
+                           double* MK, double* qmean, void* ws, cudaStream_t s) {
+  if (pl.d == 128) return run_moments<128>(pl, q, k, MQ, MK, qmean, ws, s);
+  return run_moments<64>(pl, q, k, MQ, MK, qmean, ws, s);
+}
+
+}  // namespace spark

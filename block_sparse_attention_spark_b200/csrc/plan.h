@@ -1,0 +1,61 @@
+// Host-side workspace plan and the launchers each kernel file exports.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "../../include/spark.h"
+
+namespace spark {
+
+// Number of token chunks each (head, tensor) is split into by the moments
+// kernel; partial Gram matrices are summed in float64 in a fixed order.
+constexpr int MOMENT_SPLITS_MAX = 64;
+
+struct Plan {
+  int B = 0, H = 0, N = 0, d = 0, BH = 0, nb = 0, ksel = 0, nb_pad = 0;
+  int nlevels = 0;
+  std::vector<int> level_count;   // nodes that split at each level
+  std::vector<int> level_off;     // offset of each level in the node table
+  std::vector<int> level_maxg;    // largest group (in blocks) at each level
+  int moment_splits = 1;
+  // byte offsets into the workspace
+  size_t off_MQ = 0, off_MK = 0, off_qmean = 0;
+  size_t off_mpart = 0;
+  size_t off_L = 0, off_uhat = 0, off_idx = 0, off_pval = 0, off_pidx = 0;
+  size_t off_nodes = 0;
+  size_t off_perm = 0, off_sel = 0;
+  size_t off_Qp = 0, off_Kp = 0, off_Vp = 0;
+  size_t off_qm = 0, off_km = 0;
+  size_t off_kt = 0, off_vt = 0, off_beta = 0;
+  size_t total = 0;
+  // extra device room used by spark_forward_host
+  size_t off_hq = 0, off_hk = 0, off_hv = 0, off_hout = 0, off_hlse = 0;
+  size_t host_total = 0;
+};
+
+// Fills plan from validated params. Returns false if the params are invalid.
+bool make_plan(const spark_params* p, Plan* plan);
+
+template <class T>
+inline T* ws_at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(reinterpret_cast<char*>(ws) + off);
+}
+
+// ---- launchers (each returns cudaGetLastError() of its launches)
+cudaError_t launch_moments(const Plan& pl, const uint16_t* q, const uint16_t* k, double* MQ,
+                           double* MK, double* qmean, void* ws, cudaStream_t s);
+cudaError_t launch_reblock(const Plan& pl, const uint16_t* x, const double* M, int32_t* perm,
+                           void* ws, int* status, cudaStream_t s);
+cudaError_t launch_positional(const Plan& pl, int F, int Hl, int Wl, int32_t* perm,
+                              cudaStream_t s);
+cudaError_t launch_select(const Plan& pl, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                          const int32_t* perm, const double* qmean, int32_t* sel, int summary,
+                          void* ws, int* status, cudaStream_t s);
+cudaError_t launch_attn(const Plan& pl, const int32_t* perm, const int32_t* sel, uint16_t* out,
+                        float* lse, void* ws, int* status, cudaStream_t s);
+
+}  // namespace spark

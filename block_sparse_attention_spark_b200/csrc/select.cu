@@ -1,0 +1,271 @@
+// Step a3 (block statistics, summaries) and a4 (top-K block selection).
+//
+// blockstats: one CTA per (key block, head). Gathers the block's 64 q, k, v
+//   rows by the permutation, writes the permuted copies the attention
+//   kernel streams, the float64 block means of q and k, and the block's
+//   summary ("Spark-H3" news post, Spark-Reweight bullet and figure caption;
+//   "MiniMax H3 Spark Attention (SM89)", under the hood): anchor logits
+//   x_j = qbar . k_j / sqrt(d), w = softmax(x), k~ = sum w k, v~ = sum w v,
+//   beta = ln sum e^x - qbar . k~ / sqrt(d) (k~ as stored in bf16), or the
+//   mean-pooling ablation (mean k, mean v, beta = ln 64).
+// select: one CTA per R query blocks of a head. Block scores
+//   s_ab = Qbar_a . Kbar_b / sqrt(d) in float64 ("Spark-H3" news post: the
+//   exact branch computes the top-ranked key/value blocks), then per row a
+//   warp-level radix select of the Ksel largest, ties to the lower b, written
+//   in ascending b order.
+#include <math.h>
+
+#include "common.cuh"
+#include "plan.h"
+
+namespace spark {
+
+template <int D>
+__global__ void __launch_bounds__(256)
+blockstats_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
+                  const uint16_t* __restrict__ v, const int32_t* __restrict__ perm,
+                  const double* __restrict__ qmean, int N, int nb, int nb_pad, int summary,
+                  uint16_t* __restrict__ Qp, uint16_t* __restrict__ Kp, uint16_t* __restrict__ Vp,
+                  double* __restrict__ qm, double* __restrict__ km, uint16_t* __restrict__ kt,
+                  uint16_t* __restrict__ vt, float* __restrict__ beta, int* status) {
+  constexpr int CH = D / 8;   // 16-byte chunks per row
+  __shared__ __align__(16) uint16_t ks[BLK * D];
+  __shared__ __align__(16) uint16_t vsm[BLK * D];
+  __shared__ float qb[D];
+  __shared__ float w[BLK];
+  __shared__ float red[8];
+  __shared__ float sh_m, sh_lz;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = blockIdx.x, bh = blockIdx.y;
+  const size_t hb = (size_t)bh * N * D;
+
+  if (b >= nb) {   // zero padding rows of the summary tables
+    for (int j = tid; j < D; j += blockDim.x) {
+      kt[((size_t)bh * nb_pad + b) * D + j] = 0;
+      vt[((size_t)bh * nb_pad + b) * D + j] = 0;
+    }
+    if (tid == 0) beta[(size_t)bh * nb_pad + b] = 0.f;
+    return;
+  }
+
+  // gather + permuted copies; q rows go straight to the column sums below
+  const int32_t* pr = perm + (size_t)bh * N + (size_t)b * BLK;
+  for (int c = tid; c < BLK * CH; c += blockDim.x) {
+    const int r = c / CH, ch = c % CH;
+    int row = pr[r];
+    if ((unsigned)row >= (unsigned)N) { set_status(status, STATUS_BAD_INPUT); row = 0; }
+    const size_t src = hb + (size_t)row * D + ch * 8;
+    const size_t dst = hb + ((size_t)b * BLK + r) * D + ch * 8;
+    const uint4 kk = *reinterpret_cast<const uint4*>(k + src);
+    const uint4 vv = *reinterpret_cast<const uint4*>(v + src);
+    const uint4 qq = *reinterpret_cast<const uint4*>(q + src);
+    *reinterpret_cast<uint4*>(Kp + dst) = kk;
+    *reinterpret_cast<uint4*>(Vp + dst) = vv;
+    *reinterpret_cast<uint4*>(Qp + dst) = qq;
+    *reinterpret_cast<uint4*>(ks + r * D + ch * 8) = kk;
+    *reinterpret_cast<uint4*>(vsm + r * D + ch * 8) = vv;
+  }
+  if (tid < D) qb[tid] = (float)qmean[(size_t)bh * D + tid];
+  __syncthreads();
+
+  // float64 block means (exact sums of 64 bf16 values). q is re-read from the
+  // permuted copy this CTA just wrote (same thread block, after the barrier).
+  if (tid < D) {
+    double s = 0.0;
+    for (int r = 0; r < BLK; ++r) s += (double)bf2f(Qp[hb + ((size_t)b * BLK + r) * D + tid]);
+    qm[((size_t)bh * nb + b) * D + tid] = s * (1.0 / BLK);
+  } else if (tid < 2 * D) {
+    const int j = tid - D;
+    double s = 0.0;
+    for (int r = 0; r < BLK; ++r) s += (double)bf2f(ks[r * D + j]);
+    km[((size_t)bh * nb + b) * D + j] = s * (1.0 / BLK);
+  }
+
+  const float scale = 1.0f / sqrtf((float)D);
+  if (summary == SPARK_SUMMARY_MEANPOOL) {
+    __syncthreads();
+    if (tid < D) {
+      float sk = 0.f, sv = 0.f;
+      for (int r = 0; r < BLK; ++r) { sk += bf2f(ks[r * D + tid]); sv += bf2f(vsm[r * D + tid]); }
+      kt[((size_t)bh * nb_pad + b) * D + tid] = f2bf(sk * (1.f / BLK));
+      vt[((size_t)bh * nb_pad + b) * D + tid] = f2bf(sv * (1.f / BLK));
+    }
+    if (tid == 0) beta[(size_t)bh * nb_pad + b] = logf((float)BLK);
+    return;
+  }
+
+  // anchor logits: warp w handles rows 8w..8w+7
+  for (int r = warp * 8; r < warp * 8 + 8; ++r) {
+    float s = 0.f;
+    for (int j = lane; j < D; j += 32) s = fmaf(qb[j], bf2f(ks[r * D + j]), s);
+    s = warp_sumf(s);
+    if (lane == 0) w[r] = s * scale;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const float x0 = w[lane], x1 = w[lane + 32];
+    const float m = warp_maxf(fmaxf(x0, x1));
+    const float e0 = expf(x0 - m), e1 = expf(x1 - m);
+    const float z = warp_sumf(e0 + e1);
+    w[lane] = e0 / z;
+    w[lane + 32] = e1 / z;
+    if (lane == 0) { sh_m = m; sh_lz = logf(z); }
+  }
+  __syncthreads();
+  float dotpart = 0.f;
+  if (tid < D) {
+    float sk = 0.f, sv = 0.f;
+    for (int r = 0; r < BLK; ++r) {
+      sk = fmaf(w[r], bf2f(ks[r * D + tid]), sk);
+      sv = fmaf(w[r], bf2f(vsm[r * D + tid]), sv);
+    }
+    const uint16_t kb = f2bf(sk);
+    kt[((size_t)bh * nb_pad + b) * D + tid] = kb;
+    vt[((size_t)bh * nb_pad + b) * D + tid] = f2bf(sv);
+    dotpart = qb[tid] * bf2f(kb);
+  }
+  dotpart = warp_sumf(dotpart);
+  if (lane == 0) red[warp] = dotpart;
+  __syncthreads();
+  if (tid == 0) {
+    float dsum = 0.f;
+    for (int i = 0; i < 8; ++i) dsum += red[i];
+    beta[(size_t)bh * nb_pad + b] = (sh_m + sh_lz) - dsum * scale;
+  }
+}
+
+// ------------------------------------------------------------------ selection
+template <int D>
+__global__ void __launch_bounds__(256)
+select_kernel(const double* __restrict__ qm, const double* __restrict__ km, int nb, int ksel,
+              int R, int32_t* __restrict__ sel) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  constexpr int KC = 64;          // key blocks staged per chunk
+  constexpr int KS = D + 1;       // padded row stride (doubles)
+  double* sc = reinterpret_cast<double*>(smem_raw);            // [R][nb]
+  double* qs = sc + (size_t)R * nb;                             // [R][D]
+  double* kc = qs + (size_t)R * D;                              // [KC][KS]
+  __shared__ int hist[8][256];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.y, a0 = blockIdx.x * R;
+  const int rows = min(R, nb - a0);
+  const double scale = 1.0 / sqrt((double)D);
+
+  for (int e = tid; e < rows * D; e += blockDim.x) qs[e] = qm[((size_t)bh * nb + a0) * D + e];
+  for (int c0 = 0; c0 < nb; c0 += KC) {
+    const int nk = min(KC, nb - c0);
+    __syncthreads();
+    for (int e = tid; e < nk * D; e += blockDim.x)
+      kc[(e / D) * KS + e % D] = km[((size_t)bh * nb + c0) * D + e];
+    __syncthreads();
+    for (int e = tid; e < rows * KC; e += blockDim.x) {
+      const int a = e / KC, bl = e % KC;
+      if (bl < nk) {
+        double s = 0.0;
+#pragma unroll 8
+        for (int j = 0; j < D; ++j) s = fma(qs[a * D + j], kc[bl * KS + j], s);
+        sc[(size_t)a * nb + c0 + bl] = s * scale;
+      }
+    }
+  }
+  __syncthreads();
+
+  // per row: the ksel largest scores, ties to the lower block index
+  int* h = hist[warp];
+  for (int a = warp; a < rows; a += 8) {
+    const double* srow = sc + (size_t)a * nb;
+    auto key = [&](int bb) -> uint64_t { return ordered_key(-srow[bb]); };
+    uint64_t prefix = 0, mask = 0;
+    int rank = ksel;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+      for (int i = lane; i < 256; i += 32) h[i] = 0;
+      __syncwarp();
+      for (int bb = lane; bb < nb; bb += 32) {
+        const uint64_t kk = key(bb);
+        if ((kk & mask) == prefix) atomicAdd(&h[(kk >> shift) & 255], 1);
+      }
+      __syncwarp();
+      int loc[8], s = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { loc[j] = h[lane * 8 + j]; s += loc[j]; }
+      int incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const int excl = incl - s;
+      int bucket = 0, newrank = 0;
+      const bool mine = (excl < rank && rank <= incl);
+      if (mine) {
+        int c = excl;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (c < rank && rank <= c + loc[j]) { bucket = lane * 8 + j; newrank = rank - c; }
+          c += loc[j];
+        }
+      }
+      const unsigned owner = __ballot_sync(0xffffffffu, mine);
+      const int src = __ffs(owner) - 1;
+      bucket = __shfl_sync(0xffffffffu, bucket, src);
+      newrank = __shfl_sync(0xffffffffu, newrank, src);
+      prefix |= ((uint64_t)bucket) << shift;
+      mask |= ((uint64_t)255) << shift;
+      rank = newrank;
+      __syncwarp();
+    }
+    const uint64_t kstar = prefix;
+    // members with key < kstar, plus the first `rank` members with key == kstar
+    int out = 0, ties = 0;
+    int32_t* dst = sel + ((size_t)bh * nb + a0 + a) * ksel;
+    for (int c0 = 0; c0 < nb; c0 += 32) {
+      const int bb = c0 + lane;
+      uint64_t kk = ~0ull;
+      if (bb < nb) kk = key(bb);
+      const bool less = bb < nb && kk < kstar;
+      const bool eq = bb < nb && kk == kstar;
+      const unsigned em = __ballot_sync(0xffffffffu, eq);
+      const int eq_before = ties + __popc(em & ((1u << lane) - 1u));
+      const bool take = less || (eq && eq_before < rank);
+      const unsigned tm = __ballot_sync(0xffffffffu, take);
+      const int at = out + __popc(tm & ((1u << lane) - 1u));
+      if (take && at < ksel) dst[at] = bb;
+      out += __popc(tm);
+      ties += __popc(em);
+    }
+  }
+}
+
+template <int D>
+static cudaError_t run_select(const Plan& pl, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                              const int32_t* perm, const double* qmean, int32_t* sel, int summary,
+                              void* ws, int* status, cudaStream_t s) {
+  uint16_t* Qp = ws_at<uint16_t>(ws, pl.off_Qp);
+  uint16_t* Kp = ws_at<uint16_t>(ws, pl.off_Kp);
+  uint16_t* Vp = ws_at<uint16_t>(ws, pl.off_Vp);
+  double* qm = ws_at<double>(ws, pl.off_qm);
+  double* km = ws_at<double>(ws, pl.off_km);
+  uint16_t* kt = ws_at<uint16_t>(ws, pl.off_kt);
+  uint16_t* vt = ws_at<uint16_t>(ws, pl.off_vt);
+  float* beta = ws_at<float>(ws, pl.off_beta);
+  blockstats_kernel<D><<<dim3(pl.nb_pad, pl.BH), 256, 0, s>>>(q, k, v, perm, qmean, pl.N, pl.nb,
+                                                              pl.nb_pad, summary, Qp, Kp, Vp, qm, km,
+                                                              kt, vt, beta, status);
+  const size_t fixed = sizeof(double) * (64 * (D + 1));
+  int R = (int)std::min<size_t>(8, (190000 - fixed) / (sizeof(double) * ((size_t)pl.nb + D)));
+  if (R < 1) R = 1;
+  const size_t smem = sizeof(double) * ((size_t)R * pl.nb + (size_t)R * D) + fixed;
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  select_kernel<D><<<dim3((pl.nb + R - 1) / R, pl.BH), 256, smem, s>>>(qm, km, pl.nb, pl.ksel, R, sel);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select(const Plan& pl, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                          const int32_t* perm, const double* qmean, int32_t* sel, int summary,
+                          void* ws, int* status, cudaStream_t s) {
+  if (pl.d == 128) return run_select<128>(pl, q, k, v, perm, qmean, sel, summary, ws, status, s);
+  return run_select<64>(pl, q, k, v, perm, qmean, sel, summary, ws, status, s);
+}
+
+}  // namespace spark

@@ -1,0 +1,315 @@
+// C ABI of libspark: argument validation, workspace planning and the launch
+// sequence of each step. See include/spark.h for the contract of each call.
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "plan.h"
+
+namespace spark {
+
+// Device status word: bounded waits and the Cholesky pivot check set bits
+// here; spark_get_status() reads and clears it.
+__device__ int g_spark_status = 0;
+
+static int* status_ptr() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_spark_status) != cudaSuccess) return nullptr;
+  return static_cast<int*>(p);
+}
+
+static int num_selected_impl(int nb, double ratio, int blocks) {
+  if (blocks > 0) return std::min(blocks, nb);
+  const int k = (int)ceil(ratio * (double)nb - 1e-9);
+  return std::max(1, std::min(nb, k));
+}
+
+static spark_status validate(const spark_params* p) {
+  if (p == nullptr) return SPARK_ERR_INVALID_ARG;
+  if (p->B < 1 || p->H < 1 || p->N < 1 || p->d < 1) return SPARK_ERR_INVALID_ARG;
+  if (p->topk_blocks < 0) return SPARK_ERR_INVALID_ARG;
+  if (p->layout != SPARK_LAYOUT_Q_REUSE_K && p->layout != SPARK_LAYOUT_K_REUSE_Q) return SPARK_ERR_INVALID_ARG;
+  if (p->summary != SPARK_SUMMARY_REWEIGHT && p->summary != SPARK_SUMMARY_MEANPOOL) return SPARK_ERR_INVALID_ARG;
+  if (p->tail != SPARK_TAIL_QUERY) return SPARK_ERR_INVALID_ARG;
+  if (p->N % SPARK_BLOCK != 0) return SPARK_ERR_UNSUPPORTED;
+  if (p->d != 64 && p->d != 128) return SPARK_ERR_UNSUPPORTED;
+  const long nb = p->N / SPARK_BLOCK;
+  if (nb < 2 || nb > SPARK_MAX_BLOCKS) return SPARK_ERR_UNSUPPORTED;
+  if (p->topk_blocks == 0 && !(p->topk_ratio > 0.0 && p->topk_ratio <= 1.0)) return SPARK_ERR_UNSUPPORTED;
+  if ((long)p->B * p->H > 65535) return SPARK_ERR_UNSUPPORTED;
+  return SPARK_OK;
+}
+
+static size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
+
+bool make_plan(const spark_params* p, Plan* pl) {
+  if (validate(p) != SPARK_OK) return false;
+  Plan& P = *pl;
+  P = Plan();
+  P.B = p->B; P.H = p->H; P.N = p->N; P.d = p->d;
+  P.BH = p->B * p->H;
+  P.nb = p->N / SPARK_BLOCK;
+  P.ksel = num_selected_impl(P.nb, p->topk_ratio, p->topk_blocks);
+  P.nb_pad = (P.nb + SPARK_BLOCK - 1) / SPARK_BLOCK * SPARK_BLOCK;
+  // tree: same recursion as the device tree builder
+  {
+    std::vector<std::pair<int, int>> cur{{0, P.nb}};
+    int off = 0;
+    while (!cur.empty()) {
+      int maxg = 0;
+      for (auto& n : cur) maxg = std::max(maxg, n.second);
+      P.level_count.push_back((int)cur.size());
+      P.level_off.push_back(off);
+      P.level_maxg.push_back(maxg);
+      off += (int)cur.size();
+      std::vector<std::pair<int, int>> nxt;
+      for (auto& n : cur) {
+        const int gl = n.second / 2, gr = n.second - gl;
+        if (gl >= 2) nxt.push_back({n.first, gl});
+        if (gr >= 2) nxt.push_back({n.first + gl, gr});
+      }
+      cur.swap(nxt);
+    }
+    P.nlevels = (int)P.level_count.size();
+  }
+  {
+    const int want = (600 + 2 * P.BH - 1) / (2 * P.BH);
+    P.moment_splits = std::max(1, std::min({want, MOMENT_SPLITS_MAX, P.nb}));
+  }
+  const size_t BH = P.BH, N = P.N, d = P.d, nb = P.nb, nbp = P.nb_pad;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { const size_t at = o; o = align_up(o + bytes); return at; };
+  P.off_MQ = take(BH * d * d * 8);
+  P.off_MK = take(BH * d * d * 8);
+  P.off_qmean = take(BH * d * 8);
+  P.off_mpart = take(BH * 2 * (size_t)P.moment_splits * (d * d + d) * 8);
+  P.off_L = take(BH * d * d * 4);
+  P.off_uhat = take(BH * N * d * 2);
+  P.off_idx = take(BH * N * 4);
+  P.off_pval = take(BH * N * 8);
+  P.off_pidx = take(BH * N * 4);
+  P.off_nodes = take(nb * 8);
+  P.off_perm = take(BH * N * 4);
+  P.off_sel = take(BH * nb * (size_t)P.ksel * 4);
+  P.off_Qp = take(BH * N * d * 2);
+  P.off_Kp = take(BH * N * d * 2);
+  P.off_Vp = take(BH * N * d * 2);
+  P.off_qm = take(BH * nb * d * 8);
+  P.off_km = take(BH * nb * d * 8);
+  P.off_kt = take(BH * nbp * d * 2);
+  P.off_vt = take(BH * nbp * d * 2);
+  P.off_beta = take(BH * nbp * 4);
+  P.total = o;
+  P.off_hq = take(BH * N * d * 2);
+  P.off_hk = take(BH * N * d * 2);
+  P.off_hv = take(BH * N * d * 2);
+  P.off_hout = take(BH * N * d * 2);
+  P.off_hlse = take(BH * N * 4);
+  P.host_total = o;
+  return true;
+}
+
+static bool aligned16(const void* ptr) { return ((uintptr_t)ptr & 15u) == 0; }
+
+static spark_status check_ws(const Plan& pl, const void* ws, size_t ws_bytes) {
+  if (ws == nullptr || !aligned16(ws)) return SPARK_ERR_INVALID_ARG;
+  if (ws_bytes < pl.total) return SPARK_ERR_WORKSPACE;
+  return SPARK_OK;
+}
+
+static spark_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA; }
+
+}  // namespace spark
+
+using namespace spark;
+
+extern "C" {
+
+spark_status spark_validate(const spark_params* p) { return validate(p); }
+
+int32_t spark_num_selected(const spark_params* p) {
+  if (validate(p) != SPARK_OK) return -1;
+  return num_selected_impl(p->N / SPARK_BLOCK, p->topk_ratio, p->topk_blocks);
+}
+
+size_t spark_workspace_size(const spark_params* p) {
+  Plan pl;
+  return make_plan(p, &pl) ? pl.total : 0;
+}
+
+size_t spark_host_workspace_size(const spark_params* p) {
+  Plan pl;
+  return make_plan(p, &pl) ? pl.host_total : 0;
+}
+
+spark_status spark_moments(const spark_params* p, const void* q, const void* k, double* MQ,
+                           double* MK, double* qmean, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const spark_status v = validate(p);
+  if (v != SPARK_OK) return v;
+  Plan pl;
+  make_plan(p, &pl);
+  if (!q || !k || !MQ || !MK || !qmean || !aligned16(q) || !aligned16(k)) return SPARK_ERR_INVALID_ARG;
+  const spark_status w = check_ws(pl, ws, ws_bytes);
+  if (w != SPARK_OK) return w;
+  return cuda_status(launch_moments(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, ws, stream));
+}
+
+spark_status spark_reblock(const spark_params* p, const void* q, const void* k, const double* MQ,
+                           const double* MK, int32_t* perm, void* ws, size_t ws_bytes,
+                           cudaStream_t stream) {
+  const spark_status v = validate(p);
+  if (v != SPARK_OK) return v;
+  Plan pl;
+  make_plan(p, &pl);
+  if (!q || !k || !MQ || !MK || !perm || !aligned16(q) || !aligned16(k)) return SPARK_ERR_INVALID_ARG;
+  const spark_status w = check_ws(pl, ws, ws_bytes);
+  if (w != SPARK_OK) return w;
+  const bool qside = p->layout == SPARK_LAYOUT_Q_REUSE_K;
+  const uint16_t* x = (const uint16_t*)(qside ? q : k);
+  const double* M = qside ? MK : MQ;
+  return cuda_status(launch_reblock(pl, x, M, perm, ws, status_ptr(), stream));
+}
+
+spark_status spark_positional_perm(const spark_params* p, int32_t F, int32_t Hl, int32_t Wl,
+                                   int32_t* perm, cudaStream_t stream) {
+  const spark_status v = validate(p);
+  if (v != SPARK_OK) return v;
+  if (!perm || F < 1 || Hl < 1 || Wl < 1) return SPARK_ERR_INVALID_ARG;
+  if ((long)F * Hl * Wl != p->N) return SPARK_ERR_INVALID_ARG;
+  if (F % 2 != 0 || Hl % 8 != 0 || Wl % 4 != 0) return SPARK_ERR_UNSUPPORTED;
+  Plan pl;
+  make_plan(p, &pl);
+  return cuda_status(launch_positional(pl, F, Hl, Wl, perm, stream));
+}
+
+spark_status spark_select(const spark_params* p, const void* q, const void* k, const void* v,
+                          const int32_t* perm, const double* qmean, int32_t* sel, void* ws,
+                          size_t ws_bytes, cudaStream_t stream) {
+  const spark_status vs = validate(p);
+  if (vs != SPARK_OK) return vs;
+  Plan pl;
+  make_plan(p, &pl);
+  if (!q || !k || !v || !perm || !qmean || !sel) return SPARK_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return SPARK_ERR_INVALID_ARG;
+  const spark_status w = check_ws(pl, ws, ws_bytes);
+  if (w != SPARK_OK) return w;
+  return cuda_status(launch_select(pl, (const uint16_t*)q, (const uint16_t*)k, (const uint16_t*)v,
+                                   perm, qmean, sel, p->summary, ws, status_ptr(), stream));
+}
+
+spark_status spark_attn_fwd(const spark_params* p, const int32_t* perm, const int32_t* sel, void* out,
+                            float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const spark_status v = validate(p);
+  if (v != SPARK_OK) return v;
+  Plan pl;
+  make_plan(p, &pl);
+  if (!perm || !sel || !out || !aligned16(out)) return SPARK_ERR_INVALID_ARG;
+  const spark_status w = check_ws(pl, ws, ws_bytes);
+  if (w != SPARK_OK) return w;
+  return cuda_status(launch_attn(pl, perm, sel, (uint16_t*)out, lse, ws, status_ptr(), stream));
+}
+
+spark_status spark_forward(const spark_params* p, const void* q, const void* k, const void* v,
+                           void* out, float* lse, int32_t* perm_out, int32_t* sel_out, void* ws,
+                           size_t ws_bytes, cudaStream_t stream) {
+  const spark_status vs = validate(p);
+  if (vs != SPARK_OK) return vs;
+  Plan pl;
+  make_plan(p, &pl);
+  if (!q || !k || !v || !out) return SPARK_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SPARK_ERR_INVALID_ARG;
+  const spark_status w = check_ws(pl, ws, ws_bytes);
+  if (w != SPARK_OK) return w;
+  double* MQ = ws_at<double>(ws, pl.off_MQ);
+  double* MK = ws_at<double>(ws, pl.off_MK);
+  double* qmean = ws_at<double>(ws, pl.off_qmean);
+  int32_t* perm = perm_out ? perm_out : ws_at<int32_t>(ws, pl.off_perm);
+  int32_t* sel = sel_out ? sel_out : ws_at<int32_t>(ws, pl.off_sel);
+  cudaError_t e = launch_moments(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, ws, stream);
+  if (e != cudaSuccess) return SPARK_ERR_CUDA;
+  const bool qside = p->layout == SPARK_LAYOUT_Q_REUSE_K;
+  e = launch_reblock(pl, (const uint16_t*)(qside ? q : k), qside ? MK : MQ, perm, ws, status_ptr(), stream);
+  if (e != cudaSuccess) return SPARK_ERR_CUDA;
+  e = launch_select(pl, (const uint16_t*)q, (const uint16_t*)k, (const uint16_t*)v, perm, qmean, sel,
+                    p->summary, ws, status_ptr(), stream);
+  if (e != cudaSuccess) return SPARK_ERR_CUDA;
+  e = launch_attn(pl, perm, sel, (uint16_t*)out, lse, ws, status_ptr(), stream);
+  return cuda_status(e);
+}
+
+spark_status spark_forward_host(const spark_params* p, const void* q_host, const void* k_host,
+                                const void* v_host, void* out_host, float* lse_host, void* ws,
+                                size_t ws_bytes, cudaStream_t stream) {
+  const spark_status vs = validate(p);
+  if (vs != SPARK_OK) return vs;
+  Plan pl;
+  make_plan(p, &pl);
+  if (!q_host || !k_host || !v_host || !out_host) return SPARK_ERR_INVALID_ARG;
+  if (ws == nullptr || !aligned16(ws)) return SPARK_ERR_INVALID_ARG;
+  if (ws_bytes < pl.host_total) return SPARK_ERR_WORKSPACE;
+  const size_t tb = (size_t)pl.BH * pl.N * pl.d * 2;
+  void* dq = ws_at<char>(ws, pl.off_hq);
+  void* dk = ws_at<char>(ws, pl.off_hk);
+  void* dv = ws_at<char>(ws, pl.off_hv);
+  void* dout = ws_at<char>(ws, pl.off_hout);
+  float* dlse = lse_host ? ws_at<float>(ws, pl.off_hlse) : nullptr;
+  if (cudaMemcpyAsync(dq, q_host, tb, cudaMemcpyHostToDevice, stream) != cudaSuccess) return SPARK_ERR_CUDA;
+  if (cudaMemcpyAsync(dk, k_host, tb, cudaMemcpyHostToDevice, stream) != cudaSuccess) return SPARK_ERR_CUDA;
+  if (cudaMemcpyAsync(dv, v_host, tb, cudaMemcpyHostToDevice, stream) != cudaSuccess) return SPARK_ERR_CUDA;
+  const spark_status r = spark_forward(p, dq, dk, dv, dout, dlse, nullptr, nullptr, ws, pl.total, stream);
+  if (r != SPARK_OK) return r;
+  if (cudaMemcpyAsync(out_host, dout, tb, cudaMemcpyDeviceToHost, stream) != cudaSuccess) return SPARK_ERR_CUDA;
+  if (lse_host && cudaMemcpyAsync(lse_host, dlse, (size_t)pl.BH * pl.N * 4, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return SPARK_ERR_CUDA;
+  return SPARK_OK;
+}
+
+size_t spark_workspace_region(const spark_params* p, int32_t region, size_t* bytes) {
+  Plan pl;
+  if (!make_plan(p, &pl)) return (size_t)-1;
+  const size_t BH = pl.BH, N = pl.N, d = pl.d, nb = pl.nb, nbp = pl.nb_pad;
+  size_t off, sz;
+  switch (region) {
+    case SPARK_WS_MQ: off = pl.off_MQ; sz = BH * d * d * 8; break;
+    case SPARK_WS_MK: off = pl.off_MK; sz = BH * d * d * 8; break;
+    case SPARK_WS_QMEAN: off = pl.off_qmean; sz = BH * d * 8; break;
+    case SPARK_WS_PERM: off = pl.off_perm; sz = BH * N * 4; break;
+    case SPARK_WS_SEL: off = pl.off_sel; sz = BH * nb * (size_t)pl.ksel * 4; break;
+    case SPARK_WS_QM: off = pl.off_qm; sz = BH * nb * d * 8; break;
+    case SPARK_WS_KM: off = pl.off_km; sz = BH * nb * d * 8; break;
+    case SPARK_WS_KT: off = pl.off_kt; sz = BH * nbp * d * 2; break;
+    case SPARK_WS_VT: off = pl.off_vt; sz = BH * nbp * d * 2; break;
+    case SPARK_WS_BETA: off = pl.off_beta; sz = BH * nbp * 4; break;
+    case SPARK_WS_UHAT: off = pl.off_uhat; sz = BH * N * d * 2; break;
+    default: return (size_t)-1;
+  }
+  if (bytes) *bytes = sz;
+  return off;
+}
+
+spark_status spark_get_status(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return SPARK_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpyFromSymbol(&h, g_spark_status, sizeof(int)) != cudaSuccess) return SPARK_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_spark_status, &zero, sizeof(int)) != cudaSuccess) return SPARK_ERR_CUDA;
+  if (h & STATUS_TIMEOUT) return SPARK_ERR_TIMEOUT;
+  if (h & (STATUS_BAD_PIVOT | STATUS_BAD_INPUT)) return SPARK_ERR_UNSUPPORTED;
+  return SPARK_OK;
+}
+
+const char* spark_strerror(spark_status s) {
+  switch (s) {
+    case SPARK_OK: return "ok";
+    case SPARK_ERR_INVALID_ARG: return "invalid argument";
+    case SPARK_ERR_UNSUPPORTED: return "unsupported input";
+    case SPARK_ERR_WORKSPACE: return "workspace too small";
+    case SPARK_ERR_CUDA: return "CUDA error";
+    case SPARK_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

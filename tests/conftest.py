@@ -17,3 +17,19 @@ def pytest_configure(config):
 def have_gpu():
     import torch
     return torch.cuda.is_available()
+
+
+def pytest_collection_modifyitems(config, items):
+    """GPU tests need a CUDA device; without one they are skipped (never run
+    on a CPU fallback: the library has none)."""
+    try:
+        import torch
+        ok = torch.cuda.is_available()
+    except Exception:
+        ok = False
+    if ok:
+        return
+    skip = pytest.mark.skip(reason="no CUDA device")
+    for it in items:
+        if "gpu" in it.keywords:
+            it.add_marker(skip)

@@ -1,0 +1,128 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry
+point include/spark.h declares, and validates arguments before launching
+anything. No GPU is needed (no compute call is made)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import block_sparse_attention_spark_b200 as spark
+from oracle import spark_oracle as so
+from spark_gen import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "spark.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(spark_[a-z_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = spark.lib()
+    names = declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", spark.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (spark_\w+)", out))
+    assert set(names) <= exported
+
+
+def test_params_struct_layout():
+    assert ctypes.sizeof(spark.Params) == 40
+    assert spark.Params.topk_ratio.offset == 16
+
+
+def P(**kw):
+    base = dict(B=1, H=2, N=4096, d=64, topk_ratio=0.2)
+    base.update(kw)
+    return spark.params(**base)
+
+
+def test_validate_accepts_workloads():
+    for w in WORKLOADS.values():
+        for r in w.sweep():
+            p = spark.params(w.B, w.H, w.N, w.d, r)
+            assert spark.validate(p) == 0
+            assert spark.num_selected(p) == so.num_selected(w.nb, r)
+            assert spark.workspace_size(p) > 0
+            assert spark.host_workspace_size(p) > spark.workspace_size(p)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(N=4100), 2), (dict(N=64), 2), (dict(d=96), 2), (dict(d=256), 2),
+    (dict(topk_ratio=0.0), 2), (dict(topk_ratio=1.5), 2), (dict(topk_ratio=float("nan")), 2),
+    (dict(N=64 * 8193), 2), (dict(B=0), 1), (dict(H=-1), 1),
+])
+def test_validate_rejects(kw, code):
+    p = P(**kw)
+    assert spark.validate(p) == code
+    assert spark.workspace_size(p) == 0
+    assert spark.num_selected(p) == -1
+
+
+def test_bad_enums_rejected():
+    p = P()
+    p.layout = 7
+    assert spark.validate(p) == 1
+    p = P()
+    p.summary = 3
+    assert spark.validate(p) == 1
+    p = P()
+    p.tail = 1
+    assert spark.validate(p) == 1
+    p = P(topk_blocks=-2)
+    assert spark.validate(p) == 1
+
+
+@pytest.mark.parametrize("nb,r,blocks", [(64, 0.2, 0), (1134, 0.1, 0), (1134, 0.3, 0), (2, 0.01, 0),
+                                         (10, 0.3, 0), (1000, 0.3, 0), (64, 0.2, 5), (64, 0.2, 99)])
+def test_num_selected_matches_oracle(nb, r, blocks):
+    p = P(N=64 * nb, topk_ratio=r, topk_blocks=blocks)
+    assert spark.num_selected(p) == so.num_selected(nb, r, blocks)
+
+
+def test_entry_points_reject_null_and_small_workspace_without_launching():
+    L = spark.lib()
+    p = P()
+    n = spark.workspace_size(p)
+    fake = ctypes.c_void_p(1 << 20)           # never dereferenced: validation fails first
+    assert L.spark_moments(ctypes.byref(p), None, fake, fake, fake, fake, fake, n, None) == 1
+    assert L.spark_moments(ctypes.byref(p), fake, fake, fake, fake, fake, fake, n - 1, None) == 3
+    assert L.spark_reblock(ctypes.byref(p), fake, fake, fake, fake, None, fake, n, None) == 1
+    assert L.spark_select(ctypes.byref(p), fake, fake, fake, fake, fake, None, fake, n, None) == 1
+    assert L.spark_attn_fwd(ctypes.byref(p), fake, fake, fake, None, None, n, None) == 1
+    assert L.spark_attn_fwd(ctypes.byref(p), fake, fake, fake, None, fake, 16, None) == 3
+    mis = ctypes.c_void_p((1 << 20) + 2)      # misaligned
+    assert L.spark_forward(ctypes.byref(p), mis, fake, fake, fake, None, None, None, fake, n, None) == 1
+    assert L.spark_forward_host(ctypes.byref(p), fake, fake, fake, fake, None, fake, n, None) == 3
+    bad = P(N=100)
+    assert L.spark_forward(ctypes.byref(bad), fake, fake, fake, fake, None, None, None, fake, n, None) == 2
+    assert L.spark_positional_perm(ctypes.byref(p), 4, 16, 63, fake, None) == 1   # 4*16*63 != N
+    assert L.spark_positional_perm(ctypes.byref(P(N=64 * 3 * 2 * 2)), 3, 8, 32, fake, None) == 2
+
+
+def test_workspace_regions_are_disjoint_and_inside():
+    p = P(B=2, H=3, N=64 * 37, d=128, topk_ratio=0.3)
+    total = spark.workspace_size(p)
+    spans = []
+    for name in spark.WS:
+        off, n = spark.workspace_region(p, name)
+        assert off % 256 == 0 and off + n <= total
+        spans.append((off, off + n))
+    spans.sort()
+    for (a0, a1), (b0, b1) in zip(spans, spans[1:]):
+        assert a1 <= b0
+
+
+def test_strerror():
+    L = spark.lib()
+    for c in range(6):
+        assert L.spark_strerror(c)
+    assert L.spark_strerror(99) == b"unknown status"

@@ -1,0 +1,287 @@
+"""CUDA path against the CPU oracle on seeded inputs (needs a B200).
+
+Every call goes through the C ABI (ctypes binding). Layered comparison: see
+tests/parity.py."""
+
+import math
+
+import numpy as np
+import pytest
+
+import block_sparse_attention_spark_b200 as spark
+from oracle import spark_oracle as so
+from spark_gen import WORKLOADS, bf16_bits_to_f64, make_inputs, tiny_workload
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def to_dev(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def bf16_to_f64(t):
+    import torch
+    return bf16_bits_to_f64(t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16))
+
+
+def run_stages(w, ratio=None, layout="q_reuse_k", summary="reweight", topk_blocks=0, qkv=None,
+               perm=None):
+    import torch
+    q, k, v = qkv if qkv is not None else make_inputs(w)
+    B, H, N, d = q.shape
+    p = spark.params(B, H, N, d, ratio if ratio is not None else w.ratio, topk_blocks, layout, summary)
+    ws = spark.alloc_workspace(p)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    MQ, MK, qmean = spark.moments(p, qd, kd, ws)
+    gperm = spark.reblock(p, qd, kd, MQ, MK, ws) if perm is None else perm
+    uhat = spark.ws_view(ws, p, "UHAT", torch.bfloat16, (B, H, N, d)).clone() if perm is None else None
+    sel = spark.select(p, qd, kd, vd, gperm, qmean, ws)
+    out, lse = spark.attn_fwd(p, gperm, sel, ws, return_lse=True)
+    nbp = (N // 64 + 63) // 64 * 64
+    res = dict(p=p, q=q, k=k, v=v, MQ=MQ.cpu().numpy(), MK=MK.cpu().numpy(), qmean=qmean.cpu().numpy(),
+               perm=gperm.cpu().numpy(), sel=sel.cpu().numpy(), out=bf16_to_f64(out),
+               lse=lse.cpu().numpy().astype(np.float64),
+               kt=bf16_to_f64(spark.ws_view(ws, p, "KT", torch.bfloat16, (B, H, nbp, d))),
+               vt=bf16_to_f64(spark.ws_view(ws, p, "VT", torch.bfloat16, (B, H, nbp, d))),
+               beta=spark.ws_view(ws, p, "BETA", torch.float32, (B, H, nbp)).cpu().numpy().astype(np.float64),
+               qm=spark.ws_view(ws, p, "QM", torch.float64, (B, H, N // 64, d)).cpu().numpy(),
+               km=spark.ws_view(ws, p, "KM", torch.float64, (B, H, N // 64, d)).cpu().numpy(),
+               uhat=None if uhat is None else bf16_to_f64(uhat))
+    assert spark.get_status() == 0
+    return res
+
+
+def check_head(r, b, h, layout="q_reuse_k", summary="reweight", rows=None, check_perm=True,
+               report=None):
+    q = bf16_bits_to_f64(r["q"][b, h])
+    k = bf16_bits_to_f64(r["k"][b, h])
+    v = bf16_bits_to_f64(r["v"][b, h])
+    N, d = q.shape
+    nb = N // 64
+    p = r["p"]
+    # a1 moments: float64-accumulated products of bf16 values
+    MQ, MK, qbar = so.second_moment(q), so.second_moment(k), so.anchor(q)
+    assert np.abs(r["MQ"][b, h] - MQ).max() <= 1e-6 * np.abs(MQ).max()
+    assert np.abs(r["MK"][b, h] - MK).max() <= 1e-6 * np.abs(MK).max()
+    assert np.abs(r["qmean"][b, h] - qbar).max() <= 1e-12 * (1 + np.abs(qbar).max())
+    perm = r["perm"][b, h].astype(np.int64)
+    xs, Ms = (q, MK) if layout == "q_reuse_k" else (k, MQ)
+    if check_perm:
+        # normalised whitened tokens: identical up to isolated 1-ulp roundings
+        # (float32 whitening: the error is relative to |u|, so an element far
+        # below |u| = 1 can move by more than its own ulp)
+        U = so.normalized_whitened(xs, so.whitening_factor(Ms))
+        diff = r["uhat"][b, h] != U
+        assert diff.mean() <= 1e-3, diff.mean()
+        if diff.any():
+            ref_ulp = np.ldexp(1.0, np.frexp(np.abs(U[diff]))[1] - 8)
+            dev = np.abs(r["uhat"][b, h][diff] - U[diff])
+            assert np.all(dev <= np.maximum(ref_ulp, 4e-6)), dev.max()
+        st = parity.certify_perm(xs, Ms, perm, U=r["uhat"][b, h])
+        print("perm", b, h, st)
+        assert st["failures"] == 0, st
+        if report is not None:
+            report.append(("perm", b, h, st["nodes"], st["mismatched"], st["certified"], st["worst"]))
+    else:
+        parity.check_perm_structure(perm, N)
+    # a3 block means (exact sums) and summaries, given the CUDA permutation
+    qm, km = so.block_means(q, perm), so.block_means(k, perm)
+    assert np.abs(r["qm"][b, h] - qm).max() <= 1e-14 * (1 + np.abs(qm).max())
+    assert np.abs(r["km"][b, h] - km).max() <= 1e-14 * (1 + np.abs(km).max())
+    kt, vt, beta = so.summaries(k, v, perm, qbar, summary)
+    gk, gv, gb = r["kt"][b, h, :nb], r["vt"][b, h, :nb], r["beta"][b, h, :nb]
+    assert np.all(np.abs(gk - kt) <= 2 ** -8 * np.abs(kt) + 1e-6 * np.abs(kt).max())
+    assert np.all(np.abs(gv - vt) <= 2 ** -8 * np.abs(vt) + 1e-6 * np.abs(vt).max())
+    assert np.abs(gb - beta).max() <= 1e-4 * (1 + np.abs(beta).max())
+    assert np.all(r["kt"][b, h, nb:] == 0) and np.all(r["beta"][b, h, nb:] == 0)
+    # a4 selection, given the CUDA permutation
+    ksel = spark.num_selected(p)
+    sel = r["sel"][b, h].astype(np.int64)
+    st = parity.certify_select(qm, km, ksel, sel)
+    assert st["failures"] == 0, st
+    if report is not None:
+        report.append(("sel", b, h, st["rows"], st["mismatched"], st["certified"]))
+    # a5-a7 outputs, given the CUDA permutation and selection
+    ref, ref_lse = so.attention(q, k, v, perm, sel, kt, vt, beta, rows=rows)
+    mask = ~np.isnan(ref[:, 0])
+    e = parity.out_errors(r["out"][b, h][mask], ref[mask])
+    assert e["max_rel_to_bound"] <= 1.0, e
+    # derived bound: bf16 output rounding plus bf16 P and summaries
+    assert e["max_abs"] <= 2 ** -7 * np.abs(ref[mask]).max() + 4e-3 * e["ref_rms"], e
+    assert np.abs(r["lse"][b, h][mask] - ref_lse[mask]).max() <= 1e-3 * (1 + np.abs(ref_lse[mask]).max())
+    return e
+
+
+def test_tiny_workload_all_stages():
+    w = WORKLOADS["tiny_4096"]
+    r = run_stages(w)
+    rep = []
+    for h in range(w.H):
+        check_head(r, 0, h, report=rep)
+    print(rep)
+
+
+def test_mid_workload_all_stages():
+    w = WORKLOADS["mid_16128"]
+    r = run_stages(w)
+    rep = []
+    for h in range(w.H):
+        check_head(r, 0, h, report=rep)
+    print(rep)
+
+
+@pytest.mark.parametrize("nb,d", [(2, 64), (3, 128), (5, 64), (7, 128), (13, 64), (33, 128)])
+def test_ragged_trees(nb, d):
+    w = tiny_workload(f"ragged{nb}", 2, (2, 8, 4 * nb), d, 0.3, seed_index=200 + nb)
+    r = run_stages(w)
+    for h in range(w.H):
+        check_head(r, 0, h)
+
+
+def test_density_one_is_dense_attention():
+    w = tiny_workload("dense", 2, (2, 16, 32), 128, 1.0, seed_index=300)
+    r = run_stages(w)
+    for h in range(2):
+        q, k, v = (bf16_bits_to_f64(r[t][0, h]) for t in ("q", "k", "v"))
+        ref, lse = so.dense_attention(q, k, v)
+        e = parity.out_errors(r["out"][0, h], ref)
+        assert e["max_rel_to_bound"] <= 1.0
+        assert e["max_abs"] <= 2 ** -7 * np.abs(ref).max() + 4e-3 * e["ref_rms"], e
+        assert np.abs(r["lse"][0, h] - lse).max() <= 1e-3 * (1 + np.abs(lse).max())
+
+
+@pytest.mark.parametrize("summary", ["reweight", "meanpool"])
+@pytest.mark.parametrize("layout", ["q_reuse_k", "k_reuse_q"])
+def test_layouts_and_summaries(layout, summary):
+    w = tiny_workload("lay", 2, (2, 16, 64), 64, 0.25, seed_index=400)
+    r = run_stages(w, layout=layout, summary=summary)
+    for h in range(2):
+        check_head(r, 0, h, layout=layout, summary=summary)
+
+
+def test_topk_blocks_and_batch():
+    w = tiny_workload("tb", 3, (2, 16, 32), 128, 0.2, seed_index=500, B=2)
+    r = run_stages(w, topk_blocks=5)
+    assert r["sel"].shape[-1] == 5
+    for b in range(2):
+        for h in range(3):
+            check_head(r, b, h)
+
+
+def test_positional_tiles_layout():
+    import torch
+    w = WORKLOADS["tiny_4096"]
+    q, k, v = make_inputs(w)
+    p = spark.params(1, 2, w.N, w.d, 0.2)
+    perm = spark.positional_perm(p, w.grid)
+    ref = so.positional_tiles(w.grid)
+    got = perm.cpu().numpy()
+    assert np.array_equal(got[0, 0], ref) and np.array_equal(got[0, 1], ref)
+    r = run_stages(w, summary="meanpool", qkv=(q, k, v), perm=perm)
+    for h in range(2):
+        check_head(r, 0, h, summary="meanpool", check_perm=False)
+    del torch
+
+
+def test_degenerate_inputs():
+    # identical keys inside every positional block, constant values, and an
+    # all-zero query head (zero whitened vectors: index order decides)
+    w = tiny_workload("deg", 2, (2, 8, 32), 64, 0.3, seed_index=600)
+    q, k, v = make_inputs(w)
+    N = w.N
+    k[0, 0] = np.repeat(k[0, 0, ::64], 64, axis=0)
+    v[0, 0] = v[0, 0, :1]
+    q[0, 1] = 0
+    r = run_stages(w, qkv=(q, k, v))
+    check_head(r, 0, 0)
+    check_head(r, 0, 1)
+    assert np.allclose(r["out"][0, 0], bf16_bits_to_f64(v[0, 0, :1]), atol=0, rtol=2 ** -8)
+    perm1 = r["perm"][0, 1]
+    assert np.array_equal(perm1, np.arange(N))       # zero vectors: index order
+    del N
+
+
+def test_forward_matches_stages_and_is_deterministic():
+    import torch
+    w = WORKLOADS["mid_16128"]
+    q, k, v = make_inputs(w, heads=[0, 1, 2])
+    p = spark.params(1, 3, w.N, w.d, w.ratio)
+    ws = spark.alloc_workspace(p)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    outs = []
+    for _ in range(2):
+        out = spark.forward(p, qd, kd, vd, ws=ws)
+        outs.append(out.clone())
+    assert torch.equal(outs[0], outs[1])
+    r = run_stages(w, qkv=(q, k, v))
+    assert np.array_equal(bf16_to_f64(outs[0]), r["out"])
+    # host-buffer entry point
+    hws = spark.alloc_workspace(p, host=True)
+    qh, kh, vh = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in (q, k, v))
+    oh = torch.empty_like(qh).pin_memory()
+    spark.forward_host(p, qh, kh, vh, oh, hws)
+    assert spark.get_status() == 0
+    assert torch.equal(oh, outs[0].cpu())
+
+
+def test_reference_size_sampled():
+    """The 72,576-token workload in the configuration bench.py times
+    (spark_forward, ratio 0.2, all 40 heads); the oracle checks two heads
+    (one temporal, one spatial) fully for layout and selection, and sampled
+    query blocks for the outputs."""
+    import torch
+    w = WORKLOADS["ref_72576"]
+    heads = [0, 17]
+    qh, kh, vh = make_inputs(w)
+    p = spark.params(w.B, w.H, w.N, w.d, 0.2)
+    ws = spark.alloc_workspace(p)
+    out = spark.forward(p, to_dev(qh), to_dev(kh), to_dev(vh), ws=ws)
+    assert spark.get_status() == 0
+    nb, d = w.nb, w.d
+    nbp = (nb + 63) // 64 * 64
+    view = lambda n, dt, sh: spark.ws_view(ws, p, n, dt, sh).cpu().numpy()  # noqa: E731
+    r = dict(p=p, q=qh[:, heads], k=kh[:, heads], v=vh[:, heads],
+             MQ=view("MQ", torch.float64, (1, 40, d, d))[:, heads],
+             MK=view("MK", torch.float64, (1, 40, d, d))[:, heads],
+             qmean=view("QMEAN", torch.float64, (1, 40, d))[:, heads],
+             perm=view("PERM", torch.int32, (1, 40, w.N))[:, heads],
+             sel=view("SEL", torch.int32, (1, 40, nb, 227))[:, heads],
+             out=bf16_to_f64(out[:, heads]),
+             lse=np.zeros((1, 2, w.N)),
+             kt=bf16_to_f64(spark.ws_view(ws, p, "KT", torch.bfloat16, (1, 40, nbp, d))[:, heads]),
+             vt=bf16_to_f64(spark.ws_view(ws, p, "VT", torch.bfloat16, (1, 40, nbp, d))[:, heads]),
+             beta=view("BETA", torch.float32, (1, 40, nbp))[:, heads].astype(np.float64),
+             qm=view("QM", torch.float64, (1, 40, nb, d))[:, heads],
+             km=view("KM", torch.float64, (1, 40, nb, d))[:, heads],
+             uhat=bf16_to_f64(spark.ws_view(ws, p, "UHAT", torch.bfloat16, (1, 40, w.N, d))[:, heads]))
+    rng = np.random.default_rng(7)
+    rep = []
+    for j in range(2):
+        rows = sorted(rng.choice(nb, 12, replace=False).tolist()) + [nb - 1]
+        # lse is not requested on this path; compare outputs only
+        r["lse"][0, j] = np.nan
+        q = bf16_bits_to_f64(r["q"][0, j])
+        k = bf16_bits_to_f64(r["k"][0, j])
+        v = bf16_bits_to_f64(r["v"][0, j])
+        perm = r["perm"][0, j].astype(np.int64)
+        Kk = so.second_moment(k)
+        U = so.normalized_whitened(q, so.whitening_factor(Kk))
+        diff = r["uhat"][0, j] != U
+        assert diff.mean() <= 1e-3, diff.mean()
+        own = parity.certify_perm(q, Kk, perm)
+        st = parity.certify_perm(q, Kk, perm, U=r["uhat"][0, j])
+        print("head", heads[j], "uhat flips", int(diff.sum()), "own-uhat replay", own, "gpu-uhat replay", st)
+        assert st["failures"] == 0, st
+        rep.append(st)
+        qm, km = so.block_means(q, perm), so.block_means(k, perm)
+        sst = parity.certify_select(qm, km, 227, r["sel"][0, j].astype(np.int64))
+        assert sst["failures"] == 0, sst
+        kt, vt, beta = so.summaries(k, v, perm, so.anchor(q))
+        ref, _ = so.attention(q, k, v, perm, r["sel"][0, j].astype(np.int64), kt, vt, beta, rows=rows)
+        mask = ~np.isnan(ref[:, 0])
+        e = parity.out_errors(r["out"][0, j][mask], ref[mask])
+        assert e["max_rel_to_bound"] <= 1.0, e
+        assert e["max_abs"] <= 2 ** -7 * np.abs(ref[mask]).max() + 4e-3 * e["ref_rms"], e
+    print(rep)

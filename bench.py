@@ -1,0 +1,444 @@
+#!/usr/bin/env python
+"""Benchmark of the Spark-Attn forward pass on B200.
+
+One step = one attention layer of the pages' reference size (B=1, H=40,
+N=72,576 tokens = 18x48x84 latent grid = 1,134 blocks of 64, d=128, bf16,
+topk_ratio 0.2, q_reuse_k, reweighted summaries): moments -> reblock ->
+select -> exact + compressed branches -> merge, all through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl spark|reference]
+
+Prints one JSON line (rank 0). value = effective TFLOP/s of the whole job
+(dense-equivalent 4*B*H*N^2*d per layer, summed over ranks, divided by the
+max-over-ranks time); ms_per_step = ms per layer. With N > 1 (torchrun) every
+rank runs an independent replica of the layer (the pass shards by head and
+batch with no exchange step), so scaling is weak.
+
+--impl reference times the CPU oracle (float64 NumPy) on the host cores on a
+bounded sample of the same workload per step and scales it to the same unit.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import multiprocessing as mp
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from spark_gen import WORKLOADS  # noqa: E402
+
+METRIC = "Spark-Attn fwd ms/layer & eff. TFLOP/s at N=72,576, density 0.1/0.2/0.3, 1 B200"
+UNIT = "TFLOP/s (effective, dense-equivalent)"
+DATA = ("synthetic: seeded Fourier-feature Q/K on the 18x48x84 latent grid (10% temporal / "
+        "90% spatial heads, noise 0.2), V~N(0,1), bf16")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["spark", "reference"], default="spark")
+    ap.add_argument("--workload", default="ref_72576")
+    ap.add_argument("--ratio", type=float, default=0.2)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="use only the first H heads (smaller case for profiling)")
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+
+def _gen_head(args):
+    from spark_gen import make_head
+    name, b, h = args
+    return make_head(WORKLOADS[name], b, h)
+
+
+def make_inputs_parallel(w):
+    """All heads of the workload, drawn in a spawn process pool (before any
+    CUDA call in this process)."""
+    import numpy as np
+    jobs = [(w.name, b, h) for b in range(w.B) for h in range(w.H)]
+    procs = max(1, min(len(jobs), len(os.sched_getaffinity(0))))
+    with mp.get_context("spawn").Pool(procs) as pool:
+        res = pool.map(_gen_head, jobs)
+    shape = (w.B, w.H, w.N, w.d)
+    q = np.empty(shape, np.uint16)
+    k = np.empty(shape, np.uint16)
+    v = np.empty(shape, np.uint16)
+    for (_, b, h), (qq, kk, vv) in zip(jobs, res):
+        q[b, h], k[b, h], v[b, h] = qq, kk, vv
+    return q, k, v
+
+
+def flops(w, ksel):
+    BH = w.B * w.H
+    exact = 4.0 * BH * w.N * 64 * ksel * w.d
+    comp = 4.0 * BH * w.N * (w.nb - ksel) * w.d
+    dense = 4.0 * BH * float(w.N) * w.N * w.d
+    return exact, comp, dense
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu_id)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], 0.0, set()
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = max(smax, float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+
+def oracle_sample(w, ratio, heads, rows_per_head, q=None, k=None, v=None):
+    """Time the oracle on `heads` (full moments, reblock, selection and
+    summaries) plus attention for `rows_per_head` query blocks of each, and
+    scale to one whole layer. Returns (seconds per layer, sample text)."""
+    import numpy as np
+    from oracle import spark_oracle as so
+    from spark_gen import bf16_bits_to_f64, make_head
+    ksel = so.num_selected(w.nb, ratio)
+    t_head, t_rows, nrows = 0.0, 0.0, 0
+    for h in heads:
+        qq, kk, vv = make_head(w, 0, h) if q is None else (q[0, h], k[0, h], v[0, h])
+        qf, kf, vf = bf16_bits_to_f64(qq), bf16_bits_to_f64(kk), bf16_bits_to_f64(vv)
+        t0 = time.perf_counter()
+        MK, qbar = so.second_moment(kf), so.anchor(qf)
+        so.second_moment(qf)
+        perm = so.reblock(qf, MK)
+        qm, km = so.block_means(qf, perm), so.block_means(kf, perm)
+        sel = so.select(qm, km, ksel)
+        kt, vt, beta = so.summaries(kf, vf, perm, qbar)
+        t1 = time.perf_counter()
+        rows = np.linspace(0, w.nb - 1, rows_per_head).astype(int)
+        so.attention(qf, kf, vf, perm, sel, kt, vt, beta, rows=rows)
+        t2 = time.perf_counter()
+        t_head += t1 - t0
+        t_rows += t2 - t1
+        nrows += len(rows)
+    per_layer = (t_head / len(heads)) * w.H * w.B + (t_rows / nrows) * w.nb * w.H * w.B
+    sample = (f"heads {list(heads)} of {w.name}: full moments+reblock+select+summaries, attention "
+              f"for {rows_per_head} query blocks each; scaled to {w.B * w.H} heads x {w.nb} blocks")
+    return per_layer, sample
+
+
+def attn_traffic(w):
+    """DRAM bytes per attention launch from the committed ncu capture
+    (profiles/attn_traffic.json), scaled from the captured head count to this
+    launch's; None when the kernel source changed since the capture."""
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "attn_traffic.json")))
+        src = open(os.path.join(ROOT, rec["source"]), "rb").read()
+        if hashlib.sha256(src).hexdigest() != rec["source_sha256"]:
+            return None
+        per_head = rec["dram_bytes_per_launch_8_heads"] / rec["heads_captured"]
+        return per_head * w.H * w.B
+    except Exception:
+        return None
+
+
+def cpu_cores():
+    return len(os.sched_getaffinity(0))
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = workload(a)
+    from oracle import spark_oracle as so
+    ksel = so.num_selected(w.nb, a.ratio)
+    _, _, dense = flops(w, ksel)
+    times = []
+    sample = ""
+    for step in range(a.warmup + a.steps):
+        h = step % w.H
+        t, sample = oracle_sample(w, a.ratio, [h], 16)
+        if step >= a.warmup:
+            times.append(t)
+    per_layer = statistics.mean(times)
+    value = dense / per_layer / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": per_layer * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": DATA,
+        "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} topk_ratio={a.ratio}",
+                   "seq_len": w.N, "heads": w.H, "head_dim": w.d, "topk_ratio": a.ratio},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                         "sample": "per step: " + sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ CUDA arm
+
+def workload(a):
+    import dataclasses
+    w = WORKLOADS[a.workload]
+    if a.heads:
+        w = dataclasses.replace(w, H=a.heads)
+    return w
+
+
+def run_spark(a):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = workload(a)
+    qh, kh, vh = make_inputs_parallel(w)          # before the first CUDA call
+
+    import numpy as np
+    import torch
+    import block_sparse_attention_spark_b200 as spark
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+
+    def up(x):
+        return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k, v = up(qh), up(kh), up(vh)
+    p = spark.params(w.B, w.H, w.N, w.d, a.ratio)
+    ksel = spark.num_selected(p)
+    ws = spark.alloc_workspace(p)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        MQ, MK, qmean = spark.moments(p, q, k, ws)
+        if evs is not None:
+            evs[1].record(stream)
+        perm = spark.reblock(p, q, k, MQ, MK, ws)
+        if evs is not None:
+            evs[2].record(stream)
+        sel = spark.select(p, q, k, v, perm, qmean, ws)
+        if evs is not None:
+            evs[3].record(stream)
+        out = spark.attn_fwd(p, perm, sel, ws)
+        if evs is not None:
+            evs[4].record(stream)
+        return out
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(a.warmup):
+        step()
+    if spark.get_status() != 0:
+        raise RuntimeError("device status not OK after warm-up")
+
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = str(local)
+    clocks = ClockSampler(gpu_id)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(a.steps)]
+    barrier()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(a.steps):
+        step(evs[i])
+    t_end.record(stream)
+    barrier()
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    if spark.get_status() != 0:
+        raise RuntimeError("device status not OK after the timed steps")
+    stage = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(4)]
+
+    t_max = total_ms
+    if dist is not None:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = float(tt.item())
+
+    exact, comp, dense = flops(w, ksel)
+    ms_per_layer = t_max / a.steps
+    value = world * dense / (ms_per_layer * 1e-3) / 1e12
+
+    # dominant kernel: the attention (exact + compressed branches, one launch)
+    attn_ms = stage[3]
+    achieved = (exact + comp) / (attn_ms * 1e-3) / 1e12
+    traffic = attn_traffic(w)
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        peak, peak_src = float(peaks["bf16_tflops_sustained"]), "measured (sustained bf16)"
+    except Exception:
+        peak, peak_src = 1400.0, "fallback (sustained bf16)"
+
+    # ratio sweep (same run, fewer steps)
+    sweep = {}
+    if not a.no_sweep:
+        for r in (0.1, 0.2, 0.3):
+            pr = spark.params(w.B, w.H, w.N, w.d, r)
+            ws_r = spark.alloc_workspace(pr)
+            ks = spark.num_selected(pr)
+
+            def fwd():
+                return spark.forward(pr, q, k, v, ws=ws_r)
+            for _ in range(2):
+                fwd()
+            barrier()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(3):
+                fwd()
+            e1.record(stream)
+            barrier()
+            ms = e0.elapsed_time(e1) / 3
+            if dist is not None:
+                tt = torch.tensor([ms], dtype=torch.float64, device=dev)
+                dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+                ms = float(tt.item())
+            ex, cp, dn = flops(w, ks)
+            sweep[str(r)] = {"ksel": ks, "ms_per_layer": round(ms, 3),
+                             "eff_tflops": round(dn / (ms * 1e-3) / 1e12, 2),
+                             "algorithmic_tflops": round((ex + cp) / (ms * 1e-3) / 1e12, 2)}
+            del ws_r
+
+    # end to end through the host-buffer entry point (copies inside the timed region)
+    e2e = None
+    if not a.no_e2e:
+        hws = spark.alloc_workspace(p, host=True)
+        qp = torch.from_numpy(qh.view(np.int16)).view(torch.bfloat16).pin_memory()
+        kp = torch.from_numpy(kh.view(np.int16)).view(torch.bfloat16).pin_memory()
+        vp = torch.from_numpy(vh.view(np.int16)).view(torch.bfloat16).pin_memory()
+        op = torch.empty_like(qp).pin_memory()
+        spark.forward_host(p, qp, kp, vp, op, hws)
+        barrier()
+        ne = max(3, a.steps // 4)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(ne):
+            spark.forward_host(p, qp, kp, vp, op, hws)
+        e1.record(stream)
+        barrier()
+        ms = e0.elapsed_time(e1) / ne
+        if dist is not None:
+            tt = torch.tensor([ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ms = float(tt.item())
+        e2e = {"value": world * dense / (ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms,
+               "h2d_bytes_per_step": 3 * qh.nbytes, "d2h_bytes_per_step": qh.nbytes,
+               "api": "spark_forward_host (pinned host buffers)"}
+        del hws
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        per_layer, sample = oracle_sample(w, a.ratio, [0, 17, 33], 64, qh, kh, vh)
+        cpu = {"value": dense / per_layer / 1e12, "unit": UNIT, "cores": cpu_cores(),
+               "kind": "oracle", "sample": sample, "seconds_per_layer": per_layer}
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms_per_layer, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
+        "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} (18x48x84) d={w.d} "
+                               f"topk_ratio={a.ratio} Ksel={ksel} q_reuse_k reweight",
+                   "global_batch": w.B * world, "seq_len": w.N, "heads": w.H, "head_dim": w.d,
+                   "topk_ratio": a.ratio, "parallelism": f"replicas x{world}",
+                   "l2": "inputs (2.2 GB q/k/v) exceed the 126 MB L2; not flushed"},
+        "ms_per_layer": ms_per_layer,
+        "stages_ms": {"moments": stage[0], "reblock": stage[1], "select": stage[2],
+                      "attention": stage[3]},
+        "algorithmic_tflops": (exact + comp) / (ms_per_layer * 1e-3) / 1e12,
+        "sweep": sweep,
+        "roofline": {"bound": "tensor", "kernel": "attention (exact + compressed, one launch)",
+                     "achieved": achieved, "peak": peak, "peak_source": peak_src,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                     "algorithmic_flops_per_launch": exact + comp},
+        "clocks": clk,
+        "e2e": e2e,
+        "gpu_launches": spark.forward_launches(p) * a.steps,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    a = parse()
+    if a.impl == "reference":
+        return run_reference(a)
+    return run_spark(a)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -57,6 +57,7 @@ _SIGS = {
     "spark_num_selected": (_i32, [_P]),
     "spark_workspace_size": (_sz, [_P]),
     "spark_host_workspace_size": (_sz, [_P]),
+    "spark_forward_launches": (_i32, [_P]),
     "spark_workspace_region": (_sz, [_P, _i32, ctypes.POINTER(_sz)]),
     "spark_moments": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "spark_reblock": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -107,6 +108,11 @@ def num_selected(p: Params) -> int:
 
 def workspace_size(p: Params) -> int:
     return lib().spark_workspace_size(ctypes.byref(p))
+
+
+def forward_launches(p: Params) -> int:
+    """Kernel launches one spark_forward call makes."""
+    return lib().spark_forward_launches(ctypes.byref(p))
 
 
 def host_workspace_size(p: Params) -> int:

@@ -139,6 +139,12 @@ size_t spark_workspace_size(const spark_params* p) {
   return make_plan(p, &pl) ? pl.total : 0;
 }
 
+int32_t spark_forward_launches(const spark_params* p) {
+  Plan pl;
+  if (!make_plan(p, &pl)) return -1;
+  return 2 + (5 + pl.nlevels) + 2 + 1;
+}
+
 size_t spark_host_workspace_size(const spark_params* p) {
   Plan pl;
   return make_plan(p, &pl) ? pl.host_total : 0;

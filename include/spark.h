@@ -170,6 +170,10 @@ spark_status spark_forward(const spark_params* p, const void* q, const void* k, 
                            void* out, float* lse, int32_t* perm_out, int32_t* sel_out,
                            void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* Number of kernel launches one spark_forward call makes for these params
+ * (moments 2, reblock 5 + tree depth, select 2, attention 1); -1 if invalid. */
+int32_t spark_forward_launches(const spark_params* p);
+
 /* Device bytes spark_forward_host needs: spark_workspace_size() plus room
  * for device copies of q, k, v, out and lse. */
 size_t spark_host_workspace_size(const spark_params* p);

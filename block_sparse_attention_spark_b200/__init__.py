@@ -60,6 +60,7 @@ _SIGS = {
     "spark_forward_launches": (_i32, [_P]),
     "spark_workspace_region": (_sz, [_P, _i32, ctypes.POINTER(_sz)]),
     "spark_moments": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "spark_moments_noalloc": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp]),
     "spark_reblock": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "spark_positional_perm": (_i32, [_P, _i32, _i32, _i32, _vp, _vp]),
     "spark_select": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -183,6 +184,22 @@ def moments(p: Params, q, k, ws):
     qmean = torch.empty(p.B, p.H, p.d, dtype=torch.float64, device="cuda")
     _check(lib().spark_moments(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(MQ), _ptr(MK), _ptr(qmean),
                                _ptr(ws), ws.numel(), _stream()), "spark_moments")
+    return MQ, MK, qmean
+
+
+def moments_noalloc(p: Params, q, k, MQ, MK, qmean):
+    """spark_moments without a workspace: the library's own fixed device
+    array holds the partial sums (see include/spark.h for its limit and the
+    rules on overlapping calls). Outputs are written into the given tensors."""
+    torch = _torch()
+    shp = (p.B, p.H, p.N, p.d)
+    _need(q, torch.bfloat16, shp, "q")
+    _need(k, torch.bfloat16, shp, "k")
+    _need(MQ, torch.float64, (p.B, p.H, p.d, p.d), "MQ")
+    _need(MK, torch.float64, (p.B, p.H, p.d, p.d), "MK")
+    _need(qmean, torch.float64, (p.B, p.H, p.d), "qmean")
+    _check(lib().spark_moments_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(MQ), _ptr(MK),
+                                       _ptr(qmean), _stream()), "spark_moments_noalloc")
     return MQ, MK, qmean
 
 

@@ -115,3 +115,84 @@ cudaError_t launch_moments(const Plan& pl, const uint16_t* q, const uint16_t* k,
 }
 
 }  // namespace spark
+
+// ------------------------------------------------------------------ allocation-free variant
+// spark_moments_noalloc: the same two kernels, with the per-chunk partial
+// sums kept in a fixed file-scope device array instead of the caller's
+// workspace, for callers that cannot hand over or allocate device memory.
+#include <mutex>
+
+namespace spark {
+
+constexpr size_t NOALLOC_SCRATCH_BYTES = (size_t)SPARK_NOALLOC_SCRATCH_BYTES;
+
+// One copy per device that loads the library, alive until the process exits.
+// Host code must not pass this name to a kernel: on the host it is only a
+// stand-in symbol; the device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) double g_moment_scratch[NOALLOC_SCRATCH_BYTES / sizeof(double)];
+
+constexpr int NOALLOC_MAX_DEVICES = 128;
+static std::mutex g_scratch_mutex;
+static double* g_scratch_addr[NOALLOC_MAX_DEVICES] = {};
+
+// Device address of g_moment_scratch on the current device. Looked up once
+// per device (on that device's first call) and cached.
+static cudaError_t moment_scratch_address(double** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_moment_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = static_cast<double*>(p);
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+template <int D>
+static cudaError_t run_moments_static(const Plan& pl, const uint16_t* q, const uint16_t* k, double* MQ,
+                                      double* MK, double* qmean, double* part, int splits,
+                                      cudaStream_t s) {
+  constexpr int STAGES = 3;
+  using G = Gram<D>;
+  const size_t smem = sizeof(double) * G::ACC * G::THREADS + sizeof(uint16_t) * G::TILE * STAGES;
+  auto kern = moments_partial_kernel<D, STAGES>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int bps = (pl.nb + splits - 1) / splits;
+  kern<<<dim3(splits, pl.BH, 2), G::THREADS, smem, s>>>(q, k, pl.N, bps, part);
+  moments_reduce_kernel<D><<<dim3(pl.BH, 2), 256, 0, s>>>(part, splits, pl.N, MQ, MK, qmean);
+  return cudaGetLastError();
+}
+
+}  // namespace spark
+
+extern "C" spark_status spark_moments_noalloc(const spark_params* p, const void* q, const void* k,
+                                              double* MQ, double* MK, double* qmean,
+                                              cudaStream_t stream) {
+  using namespace spark;
+  const spark_status v = spark_validate(p);
+  if (v != SPARK_OK) return v;
+  Plan pl;
+  make_plan(p, &pl);
+  if (!q || !k || !MQ || !MK || !qmean) return SPARK_ERR_INVALID_ARG;
+  if (((uintptr_t)q & 15u) != 0 || ((uintptr_t)k & 15u) != 0) return SPARK_ERR_INVALID_ARG;
+  // every (head, tensor) needs at least one partial of d*d + d doubles
+  const size_t per_partial = ((size_t)pl.d * pl.d + pl.d) * sizeof(double);
+  const size_t fit = NOALLOC_SCRATCH_BYTES / per_partial;
+  const size_t min_need = 2 * (size_t)pl.BH;
+  if (min_need > fit) return SPARK_ERR_UNSUPPORTED;
+  const int splits = (int)std::max<size_t>(1, std::min<size_t>((size_t)pl.moment_splits, fit / min_need));
+  double* scratch = nullptr;
+  if (moment_scratch_address(&scratch) != cudaSuccess) return SPARK_ERR_CUDA;
+  const cudaError_t e =
+      pl.d == 128 ? run_moments_static<128>(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean,
+                                            scratch, splits, stream)
+                  : run_moments_static<64>(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean,
+                                           scratch, splits, stream);
+  return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
+}

@@ -112,6 +112,33 @@ spark_status spark_moments(const spark_params* p, const void* q, const void* k,
                            double* MQ, double* MK, double* qmean,
                            void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* Allocation-free variant of spark_moments. The pages have no counterpart:
+ * this is a convenience of this library for callers that cannot allocate or
+ * lend device memory - for example code embedded in a host framework that
+ * owns every device allocation and forbids new ones on its hot path, or a
+ * caller with a fixed memory plan and no workspace to hand over. It computes
+ * exactly what spark_moments computes (same kernels), but keeps the partial
+ * sums in a fixed device array inside the library instead of a workspace.
+ *   - The array is SPARK_NOALLOC_SCRATCH_BYTES (16 MiB) per device; every GPU
+ *     that loads the library holds it until the process exits.
+ *   - Limit: 2 * B * H partial sums of (d*d + d) doubles must fit, i.e.
+ *     B*H <= 63 for d = 128 and B*H <= 252 for d = 64; larger inputs return
+ *     SPARK_ERR_UNSUPPORTED without launching anything. Within the limit the
+ *     token range of a head is split into fewer chunks than spark_moments
+ *     uses, so it can be slower.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents (nothing in it needs to start at zero: each call writes every
+ *     partial before reading it). Calls whose kernels may overlap on the GPU
+ *     (other streams, other host threads) race on it: serialise them.
+ *   - Never allocates or frees memory (no cudaMalloc / cudaFree).
+ * Arguments as for spark_moments, minus the workspace. */
+#define SPARK_NOALLOC_SCRATCH_BYTES (16u << 20)
+spark_status spark_moments_noalloc(const spark_params* p, const void* q, const void* k,
+                                   double* MQ, double* MK, double* qmean, cudaStream_t stream);
+
 /* Step 2 - reblock ([P1] Spark-Reblock bullet; [P2] under the hood):
  * recursive bisection of the partitioned side (queries for q_reuse_k, keys
  * for k_reuse_q) along the top principal direction of its whitened,

@@ -55,7 +55,7 @@ cudaError_t launch_positional(const Plan& pl, int F, int Hl, int Wl, int32_t* pe
 cudaError_t launch_select(const Plan& pl, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                           const int32_t* perm, const double* qmean, int32_t* sel, int summary,
                           void* ws, int* status, cudaStream_t s);
-cudaError_t launch_attn(const Plan& pl, const int32_t* perm, const int32_t* sel, uint16_t* out,
-                        float* lse, void* ws, int* status, cudaStream_t s);
+cudaError_t launch_attn_tc(const Plan& pl, const int32_t* perm, const int32_t* sel, uint16_t* out,
+                           float* lse, void* ws, int* status, cudaStream_t s);
 
 }  // namespace spark

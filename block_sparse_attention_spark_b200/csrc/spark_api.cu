@@ -214,7 +214,7 @@ spark_status spark_attn_fwd(const spark_params* p, const int32_t* perm, const in
   if (!perm || !sel || !out || !aligned16(out)) return SPARK_ERR_INVALID_ARG;
   const spark_status w = check_ws(pl, ws, ws_bytes);
   if (w != SPARK_OK) return w;
-  return cuda_status(launch_attn(pl, perm, sel, (uint16_t*)out, lse, ws, status_ptr(), stream));
+  return cuda_status(launch_attn_tc(pl, perm, sel, (uint16_t*)out, lse, ws, status_ptr(), stream));
 }
 
 spark_status spark_forward(const spark_params* p, const void* q, const void* k, const void* v,
@@ -241,7 +241,7 @@ spark_status spark_forward(const spark_params* p, const void* q, const void* k, 
   e = launch_select(pl, (const uint16_t*)q, (const uint16_t*)k, (const uint16_t*)v, perm, qmean, sel,
                     p->summary, ws, status_ptr(), stream);
   if (e != cudaSuccess) return SPARK_ERR_CUDA;
-  e = launch_attn(pl, perm, sel, (uint16_t*)out, lse, ws, status_ptr(), stream);
+  e = launch_attn_tc(pl, perm, sel, (uint16_t*)out, lse, ws, status_ptr(), stream);
   return cuda_status(e);
 }
 

@@ -52,7 +52,7 @@ bool make_plan(const spark_params* p, Plan* pl) {
   P.BH = p->B * p->H;
   P.nb = p->N / SPARK_BLOCK;
   P.ksel = num_selected_impl(P.nb, p->topk_ratio, p->topk_blocks);
-  P.nb_pad = (P.nb + SPARK_BLOCK - 1) / SPARK_BLOCK * SPARK_BLOCK;
+  P.nb_pad = (P.nb + 2 * SPARK_BLOCK - 1) / (2 * SPARK_BLOCK) * (2 * SPARK_BLOCK);   // summary tiles of 128
   // tree: same recursion as the device tree builder
   {
     std::vector<std::pair<int, int>> cur{{0, P.nb}};

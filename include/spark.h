@@ -221,7 +221,7 @@ spark_status spark_forward_host(const spark_params* p, const void* q_host, const
  * (spark_forward's moments), SPARK_WS_PERM [B,H,N] i32 and SPARK_WS_SEL
  * [B,H,nb,Ksel] i32 (spark_forward's layout and selection), SPARK_WS_QM/KM
  * [B,H,nb,d] f64 block means, SPARK_WS_KT/VT [B,H,nbp,d] bf16 summaries and
- * SPARK_WS_BETA [B,H,nbp] f32 biases with nbp = nb rounded up to 64 (rows
+ * SPARK_WS_BETA [B,H,nbp] f32 biases with nbp = nb rounded up to 128 (rows
  * past nb are zero), SPARK_WS_UHAT [B,H,N,d] bf16 normalised whitened
  * tokens of the partitioned side (original token order). */
 enum {

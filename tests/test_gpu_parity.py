@@ -39,7 +39,7 @@ def run_stages(w, ratio=None, layout="q_reuse_k", summary="reweight", topk_block
     uhat = spark.ws_view(ws, p, "UHAT", torch.bfloat16, (B, H, N, d)).clone() if perm is None else None
     sel = spark.select(p, qd, kd, vd, gperm, qmean, ws)
     out, lse = spark.attn_fwd(p, gperm, sel, ws, return_lse=True)
-    nbp = (N // 64 + 63) // 64 * 64
+    nbp = spark.workspace_region(p, "BETA")[1] // (4 * B * H)
     res = dict(p=p, q=q, k=k, v=v, MQ=MQ.cpu().numpy(), MK=MK.cpu().numpy(), qmean=qmean.cpu().numpy(),
                perm=gperm.cpu().numpy(), sel=sel.cpu().numpy(), out=bf16_to_f64(out),
                lse=lse.cpu().numpy().astype(np.float64),
@@ -240,7 +240,7 @@ def test_reference_size_sampled():
     out = spark.forward(p, to_dev(qh), to_dev(kh), to_dev(vh), ws=ws)
     assert spark.get_status() == 0
     nb, d = w.nb, w.d
-    nbp = (nb + 63) // 64 * 64
+    nbp = spark.workspace_region(p, "BETA")[1] // (4 * w.B * w.H)
     view = lambda n, dt, sh: spark.ws_view(ws, p, n, dt, sh).cpu().numpy()  # noqa: E731
     r = dict(p=p, q=qh[:, heads], k=kh[:, heads], v=vh[:, heads],
              MQ=view("MQ", torch.float64, (1, 40, d, d))[:, heads],

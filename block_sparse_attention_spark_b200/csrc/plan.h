@@ -22,11 +22,14 @@ struct Plan {
   std::vector<int> level_off;     // offset of each level in the node table
   std::vector<int> level_maxg;    // largest group (in blocks) at each level
   int moment_splits = 1;
+  int sub_level = 0;              // first level whose nodes are split by the in-shared-memory subtree kernel
+  std::vector<int> level_chunks;  // > 0: the level's groups are spread over this many chunk CTAs each
   // byte offsets into the workspace
   size_t off_MQ = 0, off_MK = 0, off_qmean = 0;
   size_t off_mpart = 0;
   size_t off_L = 0, off_uhat = 0, off_idx = 0, off_pval = 0, off_pidx = 0;
   size_t off_nodes = 0;
+  size_t off_bigpart = 0, off_biginfo = 0, off_bigcand = 0;
   size_t off_perm = 0, off_sel = 0;
   size_t off_Qp = 0, off_Kp = 0, off_Vp = 0;
   size_t off_qm = 0, off_km = 0;

@@ -205,9 +205,15 @@ __device__ uint64_t radix_select_u64(int n, int rank, int nbits, GetKey getkey, 
   for (int shift = nbits - 8; shift >= 0; shift -= 8) {
     for (int b = tid; b < 256; b += blockDim.x) hist[b] = 0;
     __syncthreads();
-    for (int i = tid; i < n; i += blockDim.x) {
-      const uint64_t k = getkey(i);
-      if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255], 1);
+    for (int i0 = 0; i0 < n; i0 += blockDim.x) {   // uniform trip count: warp-aggregated adds
+      const int i = i0 + tid;
+      int bkt = -1;
+      if (i < n) {
+        const uint64_t k = getkey(i);
+        if ((k & mask) == prefix) bkt = (int)((k >> shift) & 255);
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, bkt);
+      if (bkt >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bkt], __popc(peers));
     }
     __syncthreads();
     if (tid < 32) {
@@ -237,6 +243,142 @@ __device__ uint64_t radix_select_u64(int n, int rank, int nbits, GetKey getkey, 
     __syncthreads();
   }
   return prefix;
+}
+
+// Power iteration v <- S v / |S v| (float64), POWER_ITERS steps from the
+// all-ones direction; S is a D x D row-major matrix in shared memory (the
+// buffer is reused as scratch afterwards). Thread (rg, cg) holds rows
+// rg*RPT.. and columns cg*CPT.. of S in registers and its own copy of v on
+// those columns; z goes through a padded, double-buffered shared array (one
+// slot of padding per column group: conflict-free reads) and |z|^2 through
+// per-warp partials, so a step needs one barrier. Writes v to vs.
+template <int D>
+__device__ void power_iterate(double* acc64, double* vs) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int RPT = D / 32, CPT = D / 8, ZP = D + D / CPT;
+  const int rg = tid >> 3, cg = tid & 7;
+  double Sr[RPT][CPT];
+#pragma unroll
+  for (int i = 0; i < RPT; ++i)
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) Sr[i][j] = acc64[(rg * RPT + i) * D + cg * CPT + j];
+  double vloc[CPT];
+#pragma unroll
+  for (int j = 0; j < CPT; ++j) vloc[j] = 1.0 / sqrt((double)D);
+  double* zb = acc64;                        // S has been copied to registers: reuse as z buffers
+  __syncthreads();
+  auto zpad = [](int c) { return c + c / CPT; };
+  bool zero_dir = false;
+  double* nparts = zb + 2 * ZP;               // [2][8] per-warp partial |z|^2
+  for (int iter = 0; iter < POWER_ITERS; ++iter) {
+    double* z = zb + (iter & 1) * ZP;
+    double sq = 0.0;
+    double zr[RPT];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) zr[i] = 0.0;
+#pragma unroll
+    for (int j = 0; j < CPT; ++j)
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) zr[i] = fma(Sr[i][j], vloc[j], zr[i]);
+#pragma unroll
+    for (int o = 1; o <= 4; o <<= 1)
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) zr[i] += __shfl_xor_sync(0xffffffffu, zr[i], o);
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+      if (cg == 0) z[zpad(rg * RPT + i)] = zr[i];
+      sq = fma(zr[i], zr[i], sq);
+    }
+    // lanes 0, 8, 16, 24 of each warp hold the warp's four row groups
+    sq += __shfl_xor_sync(0xffffffffu, sq, 8);
+    sq += __shfl_xor_sync(0xffffffffu, sq, 16);
+    if (lane == 0) nparts[(iter & 1) * 8 + warp] = sq;
+    __syncthreads();
+    double nn = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) nn += nparts[(iter & 1) * 8 + w];
+    const double nrm = sqrt(nn);
+    if (nrm == 0.0) { zero_dir = true; break; }   // uniform: every thread saw the same partials
+    const double inv = 1.0 / nrm;
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) vloc[j] = z[zpad(cg * CPT + j)] * inv;
+  }
+  if (zero_dir) {
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) vloc[j] = 0.0;
+  }
+  if (rg == 0) {
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) vs[cg * CPT + j] = vloc[j];
+  }
+  __syncthreads();
+
+}
+
+// The cut of one group: the key of rank nL among the (sgn * p, index) keys
+// (block radix select on the ordered float64 projection, then index ties),
+// then a stable partition written over the group's index slice: the nL
+// smallest keys left, the rest right. pv/pi: the group's projections and
+// token indices (global scratch), ids: the group's index slice (output).
+__device__ void cut_and_partition(int n, int nL, double sgn, const double* pv, const int32_t* pi,
+                                  int32_t* ids, int* hist, int* sh_sel, int* warp_tot, int* red_i,
+                                  int* status) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // ---- phase 5: the cut - key of rank nL among (sgn * p) keys, then index ties
+  auto pkey = [&](int i) -> uint64_t { return ordered_key(sgn * pv[i]); };
+  const uint64_t kstar = radix_select_u64(n, nL, 64, pkey, hist, sh_sel);
+  int c_less = 0, c_eq = 0;
+  for (int i = tid; i < n; i += blockDim.x) {
+    const uint64_t k = pkey(i);
+    c_less += (k < kstar);
+    c_eq += (k == kstar);
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    c_less += __shfl_xor_sync(0xffffffffu, c_less, o);
+    c_eq += __shfl_xor_sync(0xffffffffu, c_eq, o);
+  }
+  if (lane == 0) { red_i[warp] = c_less; warp_tot[warp] = c_eq; }
+  __syncthreads();
+  if (tid == 0) {
+    int a = 0, b = 0;
+    for (int w = 0; w < 8; ++w) { a += red_i[w]; b += warp_tot[w]; }
+    sh_sel[0] = a;
+    sh_sel[1] = b;
+  }
+  __syncthreads();
+  const int need = nL - sh_sel[0];
+  const int ties = sh_sel[1];
+  __syncthreads();
+  int32_t istar = 0x7fffffff;
+  if (need < ties) {   // several tokens share the cut value: lowest indices go left
+    auto ikey = [&](int i) -> uint64_t {
+      return (pkey(i) == kstar) ? (uint64_t)(uint32_t)pi[i] : 0xffffffffull;
+    };
+    istar = (int32_t)radix_select_u64(n, need, 32, ikey, hist, sh_sel);
+  }
+
+  // ---- phase 6: stable partition, written in place over the group's indices
+  int left_done = 0, right_done = 0;
+  for (int base = 0; base < n; base += blockDim.x) {
+    const int i = base + tid;
+    int goleft = 0;
+    int32_t id = 0;
+    if (i < n) {
+      const uint64_t k = pkey(i);
+      id = pi[i];
+      goleft = (k < kstar) || (k == kstar && id <= istar);
+    }
+    int tot;
+    const int lpos = block_excl_scan_256(goleft, warp_tot, tot);
+    if (i < n) {
+      const int dst = goleft ? left_done + lpos : nL + right_done + (tid - lpos);
+      const bool in_side = goleft ? (dst < nL) : (dst < n);
+      if (in_side) ids[dst] = id;
+      else set_status(status, STATUS_BAD_INPUT);
+    }
+    left_done += tot;
+    right_done += min((int)blockDim.x, n - base) - tot;
+  }
 }
 
 // ------------------------------------------------------------------ one split level
@@ -297,17 +439,29 @@ split_level_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restr
     cp_async_commit();
     const uint16_t* sm = tiles + (it % STAGES) * G::TILE;
     G::tile_mma(sm, acc, warp, lane);
-    if (tid < D) {
-      double s = 0.0;
-#pragma unroll 8
-      for (int r = 0; r < BLK; ++r) s += (double)bf2f(sm[r * G::RS + tid]);
-      csum += s;
+    {
+      // column sums: thread covers column tid % D over rows (tid / D) + k * (256 / D)
+      constexpr int RSTEP = 256 / D;
+      float c4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int r = tid / D, k = 0; r < BLK; r += RSTEP, ++k) c4[k & 3] += bf2f(sm[r * G::RS + (tid % D)]);
+      csum += (double)((c4[0] + c4[1]) + (c4[2] + c4[3]));
     }
     if ((it + 1) % G::FLUSH == 0 || it == ntiles - 1) G::flush(acc, acc64, tid);
   }
   cp_async_wait<0>();
   const double invn = 1.0 / (double)n;
-  if (tid < D) mus[tid] = csum * invn;
+  {
+    double* cs = reinterpret_cast<double*>(tiles);   // tiles are drained: reuse for the column reduction
+    __syncthreads();                                  // every warp is done with the last tile
+    cs[tid] = csum;
+    __syncthreads();
+    if (tid < D) {
+      double t = 0.0;
+      for (int k = 0; k < 256 / D; ++k) t += cs[tid + k * D];
+      mus[tid] = t * invn;
+    }
+  }
   __syncthreads();
 
   // ---- phase 2: S = G/n - mu mu^T, written over the accumulators as a D x D matrix
@@ -325,56 +479,20 @@ split_level_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restr
   }
   __syncthreads();
 
-  // ---- phase 3: power iteration v <- S v / |S v| (float64, S in registers)
-  constexpr int RPT = D / 32, CPT = D / 8;
-  const int rg = tid >> 3, cg = tid & 7;
-  double Sr[RPT][CPT];
-#pragma unroll
-  for (int i = 0; i < RPT; ++i)
-#pragma unroll
-    for (int j = 0; j < CPT; ++j) Sr[i][j] = acc64[(rg * RPT + i) * D + cg * CPT + j];
-  if (tid < D) vs[tid] = 1.0 / sqrt((double)D);
-  __syncthreads();
-  for (int iter = 0; iter < POWER_ITERS; ++iter) {
-    double z[RPT];
-#pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-      double s = 0.0;
-#pragma unroll
-      for (int j = 0; j < CPT; ++j) s = fma(Sr[i][j], vs[cg * CPT + j], s);
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      s += __shfl_xor_sync(0xffffffffu, s, 2);
-      s += __shfl_xor_sync(0xffffffffu, s, 4);
-      z[i] = s;
-    }
-    if (cg == 0) {
-#pragma unroll
-      for (int i = 0; i < RPT; ++i) zs[rg * RPT + i] = z[i];
-    }
-    __syncthreads();
-    if (warp == 0) {
-      double s = 0.0;
-      for (int c = lane; c < D; c += 32) s = fma(zs[c], zs[c], s);
-      s = warp_sum(s);
-      if (lane == 0) sh_scalar = s;
-    }
-    __syncthreads();
-    const double nrm = sqrt(sh_scalar);
-    if (nrm == 0.0) {
-      if (tid < D) vs[tid] = 0.0;
-      __syncthreads();
-      break;
-    }
-    if (tid < D) vs[tid] = zs[tid] / nrm;
-    __syncthreads();
-  }
+  power_iterate<D>(acc64, vs);
 
-  // ---- phase 4: projections p_i = v . (u_i - mu) (float64); best |p|, lowest index
+  // ---- phase 4: projections p_i = v . u_i - v . mu (float64); best |p|, lowest index
   double best_abs = -1.0, best_p = 0.0;
   int best_id = 0x7fffffff;
   {
     constexpr int QD = D / 4;
     const int tok = tid >> 2, qd = tid & 3;
+    double vr[QD];
+#pragma unroll
+    for (int j = 0; j < QD; ++j) vr[j] = vs[qd * QD + j];
+    double vmu = 0.0;
+#pragma unroll 8
+    for (int j = 0; j < D; ++j) vmu = fma(vs[j], mus[j], vmu);
 #pragma unroll
     for (int s = 0; s < STAGES - 1; ++s) {
       if (s < ntiles) G::load_tile(tiles + s * G::TILE, X, ids + s * BLK, 0, tid);
@@ -387,12 +505,22 @@ split_level_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restr
       if (nxt < ntiles) G::load_tile(tiles + (nxt % STAGES) * G::TILE, X, ids + nxt * BLK, 0, tid);
       cp_async_commit();
       const uint16_t* sm = tiles + (it % STAGES) * G::TILE;
-      double s = 0.0;
-#pragma unroll 8
-      for (int j = qd * QD; j < (qd + 1) * QD; ++j)
-        s = fma(vs[j], (double)bf2f(sm[tok * G::RS + j]) - mus[j], s);
+      const uint4* rr = reinterpret_cast<const uint4*>(sm + tok * G::RS + qd * QD);
+      double s4[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+      for (int c = 0; c < QD / 8; ++c) {
+        const uint4 w = rr[c];
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          s4[e] = fma(vr[8 * c + 2 * e], (double)bf_lo(ws[e]), s4[e]);
+          s4[e] = fma(vr[8 * c + 2 * e + 1], (double)bf_hi(ws[e]), s4[e]);
+        }
+      }
+      double s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       s += __shfl_xor_sync(0xffffffffu, s, 1);
       s += __shfl_xor_sync(0xffffffffu, s, 2);
+      s -= vmu;
       if (qd == 0) {
         const int pos = it * BLK + tok;
         const int id = ids[pos];
@@ -425,61 +553,556 @@ split_level_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restr
   __syncthreads();
   const double sgn = sh_scalar;
 
-  // ---- phase 5: the cut - key of rank nL among (sgn * p) keys, then index ties
-  auto pkey = [&](int i) -> uint64_t { return ordered_key(sgn * pv[i]); };
-  const uint64_t kstar = radix_select_u64(n, nL, 64, pkey, hist, sh_sel);
-  int c_less = 0, c_eq = 0;
-  for (int i = tid; i < n; i += blockDim.x) {
-    const uint64_t k = pkey(i);
-    c_less += (k < kstar);
-    c_eq += (k == kstar);
+  cut_and_partition(n, nL, sgn, pv, pi, ids, hist, sh_sel, warp_tot, red_i, status);
+}
+
+// ------------------------------------------------------------------ large groups over many CTAs
+// For the top levels (few, large groups) one group is spread over a grid of
+// chunk CTAs: partial Gram matrices (float64 sums of float32 tile sums), one
+// CTA per group to reduce them and run the power iteration, chunk CTAs for
+// the projections (with each chunk's best |p| candidate), and one CTA per
+// group for orientation, cut and partition. Same arithmetic as
+// split_level_kernel, so both paths give the same split.
+constexpr int BIG_CHUNK_TILES = 32;
+
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+big_gram_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restrict__ nodes, int nnodes,
+                int chunks, const int32_t* __restrict__ idx, double* __restrict__ part) {
+  using G = Gram<D>;
+  using SM = SplitSmem<D>;
+  constexpr int STAGES = SM::STAGES;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  double* acc64 = reinterpret_cast<double*>(smem_raw);
+  uint16_t* tiles = reinterpret_cast<uint16_t*>(smem_raw + SM::acc_bytes);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x, k = blockIdx.y, bh = blockIdx.z;
+  const int2 node = nodes[k];
+  const int t0 = c * BIG_CHUNK_TILES, t1 = min(node.y, t0 + BIG_CHUNK_TILES);
+  const int ntiles = max(0, t1 - t0);
+  const uint16_t* X = uhat + (size_t)bh * N * D;
+  const int32_t* ids = idx + (size_t)bh * N + (size_t)node.x * BLK + (size_t)t0 * BLK;
+
+  for (int j = tid; j < G::ACC * G::THREADS; j += G::THREADS) acc64[j] = 0.0;
+  float acc[G::ACC];
+#pragma unroll
+  for (int j = 0; j < G::ACC; ++j) acc[j] = 0.f;
+  double csum = 0.0;
+#pragma unroll
+  for (int st = 0; st < STAGES - 1; ++st) {
+    if (st < ntiles) G::load_tile(tiles + st * G::TILE, X, ids + st * BLK, 0, tid);
+    cp_async_commit();
   }
+  for (int it = 0; it < ntiles; ++it) {
+    cp_async_wait<STAGES - 2>();
+    __syncthreads();
+    const int nxt = it + STAGES - 1;
+    if (nxt < ntiles) G::load_tile(tiles + (nxt % STAGES) * G::TILE, X, ids + nxt * BLK, 0, tid);
+    cp_async_commit();
+    const uint16_t* sm = tiles + (it % STAGES) * G::TILE;
+    G::tile_mma(sm, acc, warp, lane);
+    {
+      constexpr int RSTEP = 256 / D;
+      float c4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int r = tid / D, kk = 0; r < BLK; r += RSTEP, ++kk) c4[kk & 3] += bf2f(sm[r * G::RS + (tid % D)]);
+      csum += (double)((c4[0] + c4[1]) + (c4[2] + c4[3]));
+    }
+    if ((it + 1) % G::FLUSH == 0 || it == ntiles - 1) G::flush(acc, acc64, tid);
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  double* out = part + ((size_t)(bh * nnodes + k) * chunks + c) * (size_t)(D * D + D);
+#pragma unroll 4
+  for (int j = 0; j < G::ACC; ++j) {
+    int row, col;
+    G::coord(j, warp, lane, row, col);
+    out[row * D + col] = acc64[j * G::THREADS + tid];
+  }
+  double* cs = reinterpret_cast<double*>(tiles);
+  cs[tid] = csum;
+  __syncthreads();
+  if (tid < D) {
+    double t = 0.0;
+    for (int kk = 0; kk < 256 / D; ++kk) t += cs[tid + kk * D];
+    out[D * D + tid] = t;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+big_solve_kernel(const int2* __restrict__ nodes, int nnodes, int chunks, const double* __restrict__ part,
+                 double* __restrict__ info) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  double* Smat = reinterpret_cast<double*>(smem_raw);      // D x D
+  __shared__ double mus[D], vs[D];
+  const int tid = threadIdx.x, k = blockIdx.x, bh = blockIdx.y;
+  const int2 node = nodes[k];
+  const int n = node.y * BLK;
+  const int used = (node.y + BIG_CHUNK_TILES - 1) / BIG_CHUNK_TILES;
+  const double* src = part + (size_t)(bh * nnodes + k) * chunks * (size_t)(D * D + D);
+  const double invn = 1.0 / (double)n;
+  if (tid < D) {
+    double t = 0.0;
+    for (int c = 0; c < used; ++c) t += src[(size_t)c * (D * D + D) + D * D + tid];
+    mus[tid] = t * invn;
+  }
+  __syncthreads();
+  for (int e = tid; e < D * D; e += blockDim.x) {
+    double t = 0.0;
+    for (int c = 0; c < used; ++c) t += src[(size_t)c * (D * D + D) + e];
+    Smat[e] = t * invn - mus[e / D] * mus[e % D];
+  }
+  __syncthreads();
+  power_iterate<D>(Smat, vs);
+  double* out = info + (size_t)(bh * nnodes + k) * (D + 1);
+  if (tid < D) out[tid] = vs[tid];
+  if (tid == 0) {
+    double vmu = 0.0;
+    for (int j = 0; j < D; ++j) vmu = fma(vs[j], mus[j], vmu);
+    out[D] = vmu;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256)
+big_project_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restrict__ nodes, int nnodes,
+                   int chunks, const int32_t* __restrict__ idx, const double* __restrict__ info,
+                   double* __restrict__ pval, int32_t* __restrict__ pidx, double* __restrict__ cand) {
+  using G = Gram<D>;
+  constexpr int STAGES = 3;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  uint16_t* tiles = reinterpret_cast<uint16_t*>(smem_raw);
+  __shared__ double red_a[8], red_p[8];
+  __shared__ int red_id[8];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x, k = blockIdx.y, bh = blockIdx.z;
+  const int2 node = nodes[k];
+  const int t0 = c * BIG_CHUNK_TILES, t1 = min(node.y, t0 + BIG_CHUNK_TILES);
+  const int ntiles = max(0, t1 - t0);
+  const uint16_t* X = uhat + (size_t)bh * N * D;
+  const size_t gpos = (size_t)bh * N + (size_t)node.x * BLK + (size_t)t0 * BLK;
+  const int32_t* ids = idx + gpos;
+  const double* v = info + (size_t)(bh * nnodes + k) * (D + 1);
+  constexpr int QD = D / 4;
+  const int tok = tid >> 2, qd = tid & 3;
+  double vr[QD];
+#pragma unroll
+  for (int j = 0; j < QD; ++j) vr[j] = v[qd * QD + j];
+  const double vmu = v[D];
+  double best_abs = -1.0, best_p = 0.0;
+  int best_id = 0x7fffffff;
+#pragma unroll
+  for (int st = 0; st < STAGES - 1; ++st) {
+    if (st < ntiles) G::load_tile(tiles + st * G::TILE, X, ids + st * BLK, 0, tid);
+    cp_async_commit();
+  }
+  for (int it = 0; it < ntiles; ++it) {
+    cp_async_wait<STAGES - 2>();
+    __syncthreads();
+    const int nxt = it + STAGES - 1;
+    if (nxt < ntiles) G::load_tile(tiles + (nxt % STAGES) * G::TILE, X, ids + nxt * BLK, 0, tid);
+    cp_async_commit();
+    const uint16_t* sm = tiles + (it % STAGES) * G::TILE;
+    const uint4* rr = reinterpret_cast<const uint4*>(sm + tok * G::RS + qd * QD);
+    double s4[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+    for (int cc = 0; cc < QD / 8; ++cc) {
+      const uint4 w = rr[cc];
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        s4[e] = fma(vr[8 * cc + 2 * e], (double)bf_lo(ws[e]), s4[e]);
+        s4[e] = fma(vr[8 * cc + 2 * e + 1], (double)bf_hi(ws[e]), s4[e]);
+      }
+    }
+    double sv = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+    sv += __shfl_xor_sync(0xffffffffu, sv, 1);
+    sv += __shfl_xor_sync(0xffffffffu, sv, 2);
+    sv -= vmu;
+    if (qd == 0) {
+      const int pos = it * BLK + tok;
+      const int id = ids[pos];
+      pval[gpos + pos] = sv;
+      pidx[gpos + pos] = id;
+      const double a = fabs(sv);
+      if (a > best_abs || (a == best_abs && id < best_id)) { best_abs = a; best_p = sv; best_id = id; }
+    }
+  }
+  cp_async_wait<0>();
+#pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    c_less += __shfl_xor_sync(0xffffffffu, c_less, o);
-    c_eq += __shfl_xor_sync(0xffffffffu, c_eq, o);
+    const double oa = __shfl_xor_sync(0xffffffffu, best_abs, o);
+    const double op = __shfl_xor_sync(0xffffffffu, best_p, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, best_id, o);
+    if (oa > best_abs || (oa == best_abs && oi < best_id)) { best_abs = oa; best_p = op; best_id = oi; }
   }
-  if (lane == 0) { red_i[warp] = c_less; warp_tot[warp] = c_eq; }
+  if (lane == 0) { red_a[warp] = best_abs; red_p[warp] = best_p; red_id[warp] = best_id; }
   __syncthreads();
   if (tid == 0) {
-    int a = 0, b = 0;
-    for (int w = 0; w < 8; ++w) { a += red_i[w]; b += warp_tot[w]; }
-    sh_sel[0] = a;
-    sh_sel[1] = b;
+    double ba = red_a[0], bp = red_p[0];
+    int bi = red_id[0];
+    for (int w = 1; w < 8; ++w)
+      if (red_a[w] > ba || (red_a[w] == ba && red_id[w] < bi)) { ba = red_a[w]; bp = red_p[w]; bi = red_id[w]; }
+    double* o = cand + ((size_t)(bh * nnodes + k) * chunks + c) * 3;
+    o[0] = ba;
+    o[1] = bp;
+    o[2] = (double)bi;
   }
-  __syncthreads();
-  const int need = nL - sh_sel[0];
-  const int ties = sh_sel[1];
-  __syncthreads();
-  int32_t istar = 0x7fffffff;
-  if (need < ties) {   // several tokens share the cut value: lowest indices go left
-    auto ikey = [&](int i) -> uint64_t {
-      return (pkey(i) == kstar) ? (uint64_t)(uint32_t)pi[i] : 0xffffffffull;
-    };
-    istar = (int32_t)radix_select_u64(n, need, 32, ikey, hist, sh_sel);
-  }
+}
 
-  // ---- phase 6: stable partition, written in place over the group's indices
-  int left_done = 0, right_done = 0;
-  for (int base = 0; base < n; base += blockDim.x) {
-    const int i = base + tid;
-    int goleft = 0;
-    int32_t id = 0;
-    if (i < n) {
-      const uint64_t k = pkey(i);
-      id = pi[i];
-      goleft = (k < kstar) || (k == kstar && id <= istar);
+__global__ void __launch_bounds__(256)
+big_select_kernel(int N, const int2* __restrict__ nodes, int nnodes, int chunks, const double* __restrict__ cand,
+                  int32_t* __restrict__ idx, const double* __restrict__ pval, const int32_t* __restrict__ pidx,
+                  int* status) {
+  __shared__ int hist[256];
+  __shared__ int sh_sel[2];
+  __shared__ int warp_tot[8];
+  __shared__ int red_i[8];
+  __shared__ double sh_sgn;
+  const int tid = threadIdx.x, k = blockIdx.x, bh = blockIdx.y;
+  const int2 node = nodes[k];
+  const int n = node.y * BLK, nL = BLK * (node.y / 2);
+  const int used = (node.y + BIG_CHUNK_TILES - 1) / BIG_CHUNK_TILES;
+  if (tid == 0) {
+    const double* cd = cand + (size_t)(bh * nnodes + k) * chunks * 3;
+    double ba = -1.0, bp = 0.0;
+    double bi = 4.0e9;
+    for (int c = 0; c < used; ++c) {
+      const double a = cd[3 * c], pp = cd[3 * c + 1], id = cd[3 * c + 2];
+      if (a > ba || (a == ba && id < bi)) { ba = a; bp = pp; bi = id; }
     }
-    int tot;
-    const int lpos = block_excl_scan_256(goleft, warp_tot, tot);
-    if (i < n) {
-      const int dst = goleft ? left_done + lpos : nL + right_done + (tid - lpos);
-      const bool in_side = goleft ? (dst < nL) : (dst < n);
-      if (in_side) ids[dst] = id;
-      else set_status(status, STATUS_BAD_INPUT);
-    }
-    left_done += tot;
-    right_done += min((int)blockDim.x, n - base) - tot;
+    sh_sgn = (bp < 0.0) ? -1.0 : 1.0;
   }
+  __syncthreads();
+  const size_t gpos = (size_t)bh * N + (size_t)node.x * BLK;
+  cut_and_partition(n, nL, sh_sgn, pval + gpos, pidx + gpos, idx + gpos, hist, sh_sel, warp_tot, red_i, status);
+}
+
+// ------------------------------------------------------------------ whole small subtrees
+// One CTA per node of at most SUB_BLOCKS blocks at the first level where all
+// nodes are that small: the node's normalised whitened rows are staged in
+// shared memory once and every remaining split of its subtree is done
+// on-chip (same split rule as split_level_kernel): Gram by mma.sync with
+// per-lane gathered ldmatrix rows, float64 covariance and power iteration in
+// the MMA fragment layout, float64 projections, orientation, and the cut by
+// exact ranks of (projection, index) - the node's slice of the local order
+// is rewritten in ascending rank, so children are contiguous slices.
+constexpr int SUB_BLOCKS = 9;
+
+template <int D>
+struct SubSmem {
+  static constexpr int RS = D + 8;                       // padded row (elements): conflict-free ldmatrix
+  static constexpr int TMAX = SUB_BLOCKS * BLK;
+  static constexpr size_t off_rows = 0;
+  static constexpr size_t off_pv = off_rows + sizeof(uint16_t) * TMAX * RS;
+  static constexpr size_t off_ids = off_pv + sizeof(double) * TMAX;
+  static constexpr int SORTN = 1024;                     // power of two >= TMAX
+  static_assert(SORTN >= TMAX, "sort buffer must hold a whole subtree");
+  static constexpr size_t off_loc = off_ids + sizeof(int32_t) * TMAX;
+  static constexpr size_t off_skey = (off_loc + sizeof(uint16_t) * TMAX + 15) & ~(size_t)15;
+  static constexpr size_t off_sid = off_skey + sizeof(uint64_t) * SORTN;
+  static constexpr size_t off_stok = off_sid + sizeof(int32_t) * SORTN;
+  static constexpr size_t off_zp = (off_stok + sizeof(uint16_t) * SORTN + 15) & ~(size_t)15;
+  static constexpr size_t zp_bytes = sizeof(double) * 2 * 2 * D > sizeof(int32_t) * TMAX ? sizeof(double) * 2 * 2 * D : sizeof(int32_t) * TMAX;
+  static constexpr size_t bytes = off_zp + (zp_bytes > sizeof(double) * 256 ? zp_bytes : sizeof(double) * 256);
+};
+
+template <int D>
+__device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* ids, uint16_t* loc,
+                              uint64_t* skey, int32_t* sid, uint16_t* stok, double* zp, double* mus,
+                              double* vs, double* npart, double* red_d, int* red_i, double* sh_sgn, int s0,
+                              int nn) {
+  using G = Gram<D>;
+  using SM = SubSmem<D>;
+  constexpr int RS = SM::RS;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wm = warp % 4, wn = warp / 4;
+  const int m0 = wm * G::WM, n0 = wn * G::WN;
+  const int ntiles = nn / BLK;
+  const uint16_t* lo = loc + s0;
+
+  // Gram of the node (float32 over at most SUB_BLOCKS tiles) and column sums
+  float acc[G::ACC];
+#pragma unroll
+  for (int j = 0; j < G::ACC; ++j) acc[j] = 0.f;
+  for (int t = 0; t < ntiles; ++t) {
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      const int t0 = t * BLK + ks * 16;
+      uint32_t a[G::MT][4];
+      const uint16_t* ra = rows + (size_t)lo[t0 + (lane & 7) + (lane >> 4) * 8] * RS;
+#pragma unroll
+      for (int mt = 0; mt < G::MT; ++mt)
+        ldsm_x4_t(a[mt][0], a[mt][1], a[mt][2], a[mt][3], ra + m0 + mt * 16 + ((lane >> 3) & 1) * 8);
+      const uint16_t* rb = rows + (size_t)lo[t0 + (lane & 7) + ((lane >> 3) & 1) * 8] * RS;
+#pragma unroll
+      for (int np = 0; np < G::NT / 2; ++np) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(b0, b1, b2, b3, rb + n0 + np * 16 + (lane >> 4) * 8);
+#pragma unroll
+        for (int mt = 0; mt < G::MT; ++mt) {
+          mma_bf16(&acc[(mt * G::NT + 2 * np) * 4], a[mt], b0, b1);
+          mma_bf16(&acc[(mt * G::NT + 2 * np + 1) * 4], a[mt], b2, b3);
+        }
+      }
+    }
+  }
+  {
+    // column sums: thread covers column tid % D over tokens (tid / D) + k * (256 / D)
+    constexpr int RSTEP = 256 / D;
+    float c4[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int t = tid / D, k = 0; t < nn; t += RSTEP, ++k) c4[k & 3] += bf2f(rows[(size_t)lo[t] * RS + (tid % D)]);
+    double* cs = zp;   // scratch before the power iteration uses it
+    cs[tid] = (double)((c4[0] + c4[1]) + (c4[2] + c4[3]));
+    __syncthreads();
+    if (tid < D) {
+      double t = 0.0;
+      for (int k = 0; k < RSTEP; ++k) t += cs[tid + k * D];
+      mus[tid] = t / (double)nn;
+    }
+  }
+  __syncthreads();
+  // S = G / n - mu mu^T on this thread's fragment entries (float64)
+  const double invn = 1.0 / (double)nn;
+  double S[G::ACC];
+#pragma unroll
+  for (int j = 0; j < G::ACC; ++j) {
+    int row, col;
+    G::coord(j, warp, lane, row, col);
+    S[j] = (double)acc[j] * invn - mus[row] * mus[col];
+  }
+  // power iteration in the fragment layout: rows m0 + mt*16 + lane/4 + 8h,
+  // columns n0 + nt*8 + 2 (lane % 4) + e
+  double vl[G::NT * 2];
+#pragma unroll
+  for (int j = 0; j < G::NT * 2; ++j) vl[j] = 1.0 / sqrt((double)D);
+  bool zero_dir = false;
+  for (int iter = 0; iter < POWER_ITERS; ++iter) {
+    double* z = zp + (iter & 1) * 2 * D;        // [wn][row]
+    double zr[G::MT][2];
+#pragma unroll
+    for (int mt = 0; mt < G::MT; ++mt) { zr[mt][0] = 0.0; zr[mt][1] = 0.0; }
+#pragma unroll
+    for (int nt = 0; nt < G::NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+#pragma unroll
+        for (int mt = 0; mt < G::MT; ++mt)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) zr[mt][h] = fma(S[(mt * G::NT + nt) * 4 + 2 * h + e], vl[nt * 2 + e], zr[mt][h]);
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1)
+#pragma unroll
+      for (int mt = 0; mt < G::MT; ++mt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) zr[mt][h] += __shfl_xor_sync(0xffffffffu, zr[mt][h], o);
+    if ((lane & 3) == 0) {
+#pragma unroll
+      for (int mt = 0; mt < G::MT; ++mt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) z[wn * D + m0 + mt * 16 + (lane >> 2) + 8 * h] = zr[mt][h];
+    }
+    __syncthreads();
+    // |z|^2 from the warps of column half 0 (each row once)
+    double sq = 0.0;
+    if (wn == 0 && (lane & 3) == 0) {
+#pragma unroll
+      for (int mt = 0; mt < G::MT; ++mt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int row = m0 + mt * 16 + (lane >> 2) + 8 * h;
+          const double zz = z[row] + z[D + row];
+          sq = fma(zz, zz, sq);
+        }
+    }
+    sq += __shfl_xor_sync(0xffffffffu, sq, 4);
+    sq += __shfl_xor_sync(0xffffffffu, sq, 8);
+    sq += __shfl_xor_sync(0xffffffffu, sq, 16);
+    if (wn == 0 && lane == 0) npart[(iter & 1) * 4 + wm] = sq;
+    __syncthreads();
+    const double nrm = sqrt((npart[(iter & 1) * 4 + 0] + npart[(iter & 1) * 4 + 1]) +
+                            (npart[(iter & 1) * 4 + 2] + npart[(iter & 1) * 4 + 3]));
+    if (nrm == 0.0) { zero_dir = true; break; }
+    const double inv = 1.0 / nrm;
+#pragma unroll
+    for (int nt = 0; nt < G::NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int col = n0 + nt * 8 + 2 * (lane & 3) + e;
+        vl[nt * 2 + e] = (z[col] + z[D + col]) * inv;
+      }
+  }
+  if (wm == 0 && lane < 4) {
+#pragma unroll
+    for (int nt = 0; nt < G::NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) vs[n0 + nt * 8 + 2 * lane + e] = zero_dir ? 0.0 : vl[nt * 2 + e];
+  }
+  __syncthreads();
+  // projections p_t = v . (u_t - mu), float64; best |p| (lowest index on ties)
+  double best_abs = -1.0, best_p = 0.0;
+  int best_id = 0x7fffffff;
+  {
+    constexpr int QD = D / 4;
+    const int tk = tid >> 2, qd = tid & 3;
+    double vr[QD];
+#pragma unroll
+    for (int j = 0; j < QD; ++j) vr[j] = vs[qd * QD + j];
+    double vmu = 0.0;
+#pragma unroll 8
+    for (int j = 0; j < D; ++j) vmu = fma(vs[j], mus[j], vmu);
+    for (int b0 = 0; b0 < nn; b0 += 64) {
+      const int t = b0 + tk;
+      const uint4* rr = reinterpret_cast<const uint4*>(rows + (size_t)lo[t] * RS + qd * QD);
+      double s4[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+      for (int c = 0; c < QD / 8; ++c) {
+        const uint4 w = rr[c];
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          s4[e] = fma(vr[8 * c + 2 * e], (double)bf_lo(ws[e]), s4[e]);
+          s4[e] = fma(vr[8 * c + 2 * e + 1], (double)bf_hi(ws[e]), s4[e]);
+        }
+      }
+      double sacc = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+      sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
+      sacc += __shfl_xor_sync(0xffffffffu, sacc, 2);
+      sacc -= vmu;
+      if (qd == 0) {
+        pv[t] = sacc;
+        const int id = ids[lo[t]];
+        const double a = fabs(sacc);
+        if (a > best_abs || (a == best_abs && id < best_id)) { best_abs = a; best_p = sacc; best_id = id; }
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const double oa = __shfl_xor_sync(0xffffffffu, best_abs, o);
+    const double op = __shfl_xor_sync(0xffffffffu, best_p, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, best_id, o);
+    if (oa > best_abs || (oa == best_abs && oi < best_id)) { best_abs = oa; best_p = op; best_id = oi; }
+  }
+  if (lane == 0) { red_d[warp] = best_abs; red_d[8 + warp] = best_p; red_i[warp] = best_id; }
+  __syncthreads();
+  if (tid == 0) {
+    double ba = red_d[0], bp = red_d[8];
+    int bi = red_i[0];
+    for (int w = 1; w < 8; ++w) {
+      if (red_d[w] > ba || (red_d[w] == ba && red_i[w] < bi)) { ba = red_d[w]; bp = red_d[8 + w]; bi = red_i[w]; }
+    }
+    *sh_sgn = (bp < 0.0) ? -1.0 : 1.0;
+  }
+  __syncthreads();
+  const double sgn = *sh_sgn;
+  // ascending order of (sgn * p, index): bitonic sort of the node's keys
+  int P2 = 64;
+  while (P2 < nn) P2 <<= 1;
+  for (int t = tid; t < P2; t += blockDim.x) {
+    if (t < nn) {
+      skey[t] = ordered_key(sgn * pv[t]);
+      sid[t] = ids[lo[t]];
+      stok[t] = lo[t];
+    } else {
+      skey[t] = ~0ull;
+      sid[t] = 0x7fffffff;
+      stok[t] = 0;
+    }
+  }
+  __syncthreads();
+  for (int kk = 2; kk <= P2; kk <<= 1) {
+    for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+      for (int i = tid; i < P2; i += blockDim.x) {
+        const int ixj = i ^ jj;
+        if (ixj > i) {
+          const uint64_t ka = skey[i], kb = skey[ixj];
+          const int32_t ia = sid[i], ib = sid[ixj];
+          const bool a_gt = (ka > kb) || (ka == kb && ia > ib);
+          if (a_gt == ((i & kk) == 0)) {
+            skey[i] = kb; skey[ixj] = ka;
+            sid[i] = ib; sid[ixj] = ia;
+            const uint16_t ta = stok[i];
+            stok[i] = stok[ixj]; stok[ixj] = ta;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int t = tid; t < nn; t += blockDim.x) loc[s0 + t] = stok[t];
+  __syncthreads();
+}
+
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+subtree_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restrict__ nodes,
+               int32_t* __restrict__ idx, int* status) {
+  using SM = SubSmem<D>;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  uint16_t* rows = reinterpret_cast<uint16_t*>(smem_raw + SM::off_rows);
+  double* pv = reinterpret_cast<double*>(smem_raw + SM::off_pv);
+  int32_t* ids = reinterpret_cast<int32_t*>(smem_raw + SM::off_ids);
+  uint16_t* loc = reinterpret_cast<uint16_t*>(smem_raw + SM::off_loc);
+  uint64_t* skey = reinterpret_cast<uint64_t*>(smem_raw + SM::off_skey);
+  int32_t* sid = reinterpret_cast<int32_t*>(smem_raw + SM::off_sid);
+  uint16_t* stok = reinterpret_cast<uint16_t*>(smem_raw + SM::off_stok);
+  double* zp = reinterpret_cast<double*>(smem_raw + SM::off_zp);
+  __shared__ double mus[D], vs[D], npart[8], red_d[16];
+  __shared__ int red_i[8];
+  __shared__ double sh_sgn;
+  __shared__ int2 lvl[2][SUB_BLOCKS];
+  __shared__ int lvl_n[2];
+
+  const int tid = threadIdx.x;
+  const int2 node = nodes[blockIdx.x];
+  const int bh = blockIdx.y;
+  const int g0 = node.y, n = g0 * BLK, pos0 = node.x * BLK;
+  if (g0 > SUB_BLOCKS) {   // never launched that way; keep the shared arrays in bounds regardless
+    if (tid == 0) set_status(status, STATUS_BAD_INPUT);
+    return;
+  }
+  int32_t* gidx = idx + (size_t)bh * N + pos0;
+  const uint16_t* X = uhat + (size_t)bh * N * D;
+  for (int t = tid; t < n; t += blockDim.x) {
+    ids[t] = gidx[t];
+    loc[t] = (uint16_t)t;
+  }
+  __syncthreads();
+  constexpr int CH = D / 8;
+  for (int c = tid; c < n * CH; c += blockDim.x) {
+    const int t = c / CH, ch = c % CH;
+    cp_async16(rows + (size_t)t * SM::RS + ch * 8, X + (size_t)ids[t] * D + ch * 8);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  if (tid == 0) { lvl[0][0] = make_int2(0, g0); lvl_n[0] = 1; }
+  __syncthreads();
+  int cur = 0;
+  while (lvl_n[cur] > 0) {
+    const int cnt = lvl_n[cur];
+    for (int i = 0; i < cnt; ++i) {
+      const int2 nd = lvl[cur][i];
+      if (nd.y >= 2)
+        subtree_split<D>(rows, pv, ids, loc, skey, sid, stok, zp, mus, vs, npart, red_d, red_i, &sh_sgn,
+                         nd.x * BLK, nd.y * BLK);
+    }
+    if (tid == 0) {
+      int m = 0;
+      for (int i = 0; i < cnt; ++i) {
+        const int2 nd = lvl[cur][i];
+        if (nd.y < 2) continue;
+        const int gl = nd.y / 2, gr = nd.y - gl;
+        if (gl >= 2) lvl[cur ^ 1][m++] = make_int2(nd.x, gl);
+        if (gr >= 2) lvl[cur ^ 1][m++] = make_int2(nd.x + gl, gr);
+      }
+      lvl_n[cur ^ 1] = m;
+    }
+    __syncthreads();
+    cur ^= 1;
+  }
+  for (int t = tid; t < n; t += blockDim.x) gidx[t] = ids[loc[t]];
 }
 
 // ------------------------------------------------------------------ leaves -> perm
@@ -545,7 +1168,36 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
   const size_t smem_s = SplitSmem<D>::bytes;
   e = cudaFuncSetAttribute(split_level_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s);
   if (e != cudaSuccess) return e;
+  const size_t smem_t = SubSmem<D>::bytes;
+  e = cudaFuncSetAttribute(subtree_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_t);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(big_gram_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s);
+  if (e != cudaSuccess) return e;
+  const size_t smem_solve = sizeof(double) * D * D;
+  e = cudaFuncSetAttribute(big_solve_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_solve);
+  if (e != cudaSuccess) return e;
+  const size_t smem_proj = sizeof(uint16_t) * Gram<D>::TILE * 3;
+  e = cudaFuncSetAttribute(big_project_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_proj);
+  if (e != cudaSuccess) return e;
+  double* bpart = ws_at<double>(ws, pl.off_bigpart);
+  double* binfo = ws_at<double>(ws, pl.off_biginfo);
+  double* bcand = ws_at<double>(ws, pl.off_bigcand);
   for (int lv = 0; lv < pl.nlevels; ++lv) {
+    if (pl.level_chunks[lv] > 0) {   // few large groups: spread each over chunk CTAs
+      const int cnt = pl.level_count[lv], ch = pl.level_chunks[lv];
+      const int2* nd = nodes + pl.level_off[lv];
+      big_gram_kernel<D><<<dim3(ch, cnt, pl.BH), 256, smem_s, s>>>(uhat, pl.N, nd, cnt, ch, idx, bpart);
+      big_solve_kernel<D><<<dim3(cnt, pl.BH), 256, smem_solve, s>>>(nd, cnt, ch, bpart, binfo);
+      big_project_kernel<D><<<dim3(ch, cnt, pl.BH), 256, smem_proj, s>>>(uhat, pl.N, nd, cnt, ch, idx, binfo, pval,
+                                                                        pidx, bcand);
+      big_select_kernel<<<dim3(cnt, pl.BH), 256, 0, s>>>(pl.N, nd, cnt, ch, bcand, idx, pval, pidx, status);
+      continue;
+    }
+    if (pl.level_maxg[lv] <= SUB_BLOCKS) {   // this level and everything below it, in shared memory
+      subtree_kernel<D><<<dim3(pl.level_count[lv], pl.BH), 256, smem_t, s>>>(uhat, pl.N, nodes + pl.level_off[lv],
+                                                                            idx, status);
+      break;
+    }
     split_level_kernel<D><<<dim3(pl.level_count[lv], pl.BH), 256, smem_s, s>>>(
         uhat, pl.N, nodes + pl.level_off[lv], idx, pval, pidx, status);
   }

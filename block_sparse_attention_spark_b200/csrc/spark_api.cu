@@ -73,6 +73,15 @@ bool make_plan(const spark_params* p, Plan* pl) {
       cur.swap(nxt);
     }
     P.nlevels = (int)P.level_count.size();
+    P.sub_level = P.nlevels;
+    for (int lv = 0; lv < P.nlevels; ++lv)
+      if (P.level_maxg[lv] <= 9) { P.sub_level = lv; break; }
+    // few large groups (fewer than two waves of CTAs) are spread over chunks of 32 tiles
+    P.level_chunks.assign(P.nlevels, 0);
+    for (int lv = 0; lv < P.sub_level; ++lv) {
+      const int ch = (P.level_maxg[lv] + 31) / 32;
+      if ((long)P.level_count[lv] * P.BH < 296 && ch >= 2) P.level_chunks[lv] = ch;
+    }
   }
   {
     const int want = (600 + 2 * P.BH - 1) / (2 * P.BH);
@@ -91,6 +100,19 @@ bool make_plan(const spark_params* p, Plan* pl) {
   P.off_pval = take(BH * N * 8);
   P.off_pidx = take(BH * N * 4);
   P.off_nodes = take(nb * 8);
+  {
+    size_t part = 0, info = 0, cand = 0;
+    for (int lv = 0; lv < P.nlevels; ++lv) {
+      if (P.level_chunks[lv] == 0) continue;
+      const size_t groups = (size_t)P.BH * P.level_count[lv];
+      part = std::max(part, groups * P.level_chunks[lv] * (d * d + d) * 8);
+      info = std::max(info, groups * (d + 1) * 8);
+      cand = std::max(cand, groups * P.level_chunks[lv] * 3 * 8);
+    }
+    P.off_bigpart = take(std::max<size_t>(part, 8));
+    P.off_biginfo = take(std::max<size_t>(info, 8));
+    P.off_bigcand = take(std::max<size_t>(cand, 8));
+  }
   P.off_perm = take(BH * N * 4);
   P.off_sel = take(BH * nb * (size_t)P.ksel * 4);
   P.off_Qp = take(BH * N * d * 2);
@@ -142,7 +164,11 @@ size_t spark_workspace_size(const spark_params* p) {
 int32_t spark_forward_launches(const spark_params* p) {
   Plan pl;
   if (!make_plan(p, &pl)) return -1;
-  return 2 + (5 + pl.nlevels) + 2 + 1;
+  // moments 2; reblock: whiten, normalise, tree, init, split levels, subtree, leaves; select 2; attention 1
+  int split_launches = 0;
+  for (int lv = 0; lv < pl.sub_level; ++lv) split_launches += pl.level_chunks[lv] > 0 ? 4 : 1;
+  const int reblock = 4 + split_launches + (pl.sub_level < pl.nlevels ? 1 : 0) + 1;
+  return 2 + reblock + 2 + 1;
 }
 
 size_t spark_host_workspace_size(const spark_params* p) {

@@ -198,7 +198,10 @@ spark_status spark_forward(const spark_params* p, const void* q, const void* k, 
                            void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Number of kernel launches one spark_forward call makes for these params
- * (moments 2, reblock 5 + tree depth, select 2, attention 1); -1 if invalid. */
+ * (moments 2; reblock 5, plus 1 per tree level above the first level whose
+ * groups all have at most 9 blocks - 4 for a level of few large groups that
+ * are spread over chunk CTAs - plus 1 for the subtree pass; select 2;
+ * attention 1); -1 if invalid. */
 int32_t spark_forward_launches(const spark_params* p);
 
 /* Device bytes spark_forward_host needs: spark_workspace_size() plus room

@@ -14,20 +14,28 @@
 // selected. One running softmax over both term sets = the log-sum-exp merge
 // of the two branches.
 //
-// Roles (352 threads):
-//   warps 0-7  softmax: row r = 32 (w mod 4) + lane is TMEM lane r; warp w
-//              takes columns 64 (w / 4) .. +63 of every 128-key S tile, so
-//              the two threads of a row exchange their partial row maxima
-//              through shared memory once per tile. Lazy-rescaled online
-//              softmax (the reference max moves only when the row max grows
-//              by more than 2^8); P (bf16 pairs) goes to TMEM.
-//   warp 8     TMA producer of Q (once) and the K (or k~) tiles.
-//   warp 10    TMA producer of the V (or v~) tiles.
-//   warp 9     TMEM allocator + the MMA-issuing thread:
-//              S_j = Q K_j^T (M128 N128 K=d, K-major smem operands) into one of
-//              two TMEM S buffers; O += P_j V_j (M128 N=d K=128) with P read
-//              from TMEM and V an MN-major smem operand.
-// TMEM columns: S0 [0,128) S1 [128,256) O [256,256+d) P0 [384,448) P1 [448,512).
+// A CTA runs two such units side by side in two independent slots (pairs
+// 2c and 2c+1), each with its own Q, K and V buffers and its own TMEM
+// columns, so that one slot's softmax overlaps the other slot's MMAs.
+//
+// Roles (384 threads = three warpgroups):
+//   warps 0-3  softmax of slot 0, warps 4-7 softmax of slot 1: one thread
+//              per query row (TMEM lane = row), all 128 columns of a tile.
+//              Lazy-rescaled online softmax (the reference max moves only
+//              when the row max grows by more than 2^8); P (bf16 pairs) is
+//              written over the first 64 columns of the slot's S buffer.
+//   warp 8 / 9 TMA producer of slot 0 / 1: Q once, then K_j and V_j of
+//              every tile into the slot's single K and V buffers.
+//   warp 10    TMEM allocator + the MMA-issuing thread (warp 11 idles). Per slot and tile:
+//              O += P_j V_j (M128 N=d K=128, P read from TMEM, V an MN-major
+//              smem operand), then S_{j+1} = Q K_{j+1}^T (M128 N128 K=d,
+//              K-major smem operands) into the same S columns, then one
+//              commit. The MMAs of a CTA complete in issue order, so the
+//              arrival of S_{j+1} also means that P_j and O are free: the
+//              softmax needs one wait per tile, and O can be rescaled in
+//              place without another.
+// TMEM columns: S of slot s at 128 s (P aliased on its first 64), O of slot
+// s at 256 + 128 s.
 // Every mbarrier wait is bounded (about 2 s); on expiry the kernel records
 // a timeout in the status word, drains its own copies and MMAs (again with a
 // bound), frees TMEM and returns.
@@ -42,15 +50,23 @@ namespace tc {
 
 constexpr int ROWS = 128;
 constexpr int KEYS = 128;                // keys (or summaries) per tile
-constexpr int KSTAGES = 2;
-constexpr int VSTAGES = 3;
-constexpr int THREADS = 352;
+constexpr int SLOTS = 2;
+constexpr int THREADS = 384;
+// Register split (setmaxnreg, per warpgroup): the block is launched with
+// LAUNCH_REGS per thread; the producer/MMA warpgroup gives registers back so
+// that each softmax thread can hold a whole 128-column S row.
+// 2*128*SOFTMAX_REGS + 128*OTHER_REGS equals THREADS*LAUNCH_REGS, so every
+// increase is covered by the decrease.
+constexpr int LAUNCH_REGS = 168;
+constexpr int SOFTMAX_REGS = 192;
+constexpr int OTHER_REGS = 120;
+static_assert(2 * 128 * SOFTMAX_REGS + 128 * OTHER_REGS == THREADS * LAUNCH_REGS, "register split must balance");
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t S_COL = 0;            // S buffer i at S_COL + 128 i
-constexpr uint32_t O_COL = 256;
-constexpr uint32_t P_COL = 384;          // P buffer i at P_COL + 64 i
+constexpr uint32_t S_COL = 0;            // S (and P) of slot s at S_COL + 128 s
+constexpr uint32_t O_COL = 256;          // O of slot s at O_COL + 128 s
 constexpr float LAZY_RESCALE = 8.0f;     // log2 units
 constexpr unsigned long long WAIT_NS = 2000000000ull;
+constexpr int MASK_WORDS = SPARK_MAX_BLOCKS / 32;
 
 template <int D>
 struct Layout {
@@ -59,10 +75,12 @@ struct Layout {
   static constexpr int KV_ATOM = KEYS * 128;           // 128 rows x 128 B
   static constexpr int Q_BYTES = Q_ATOM * KATOMS;
   static constexpr int KV_TILE = KV_ATOM * KATOMS;
+  // per slot: Q, K, V
+  static constexpr int SLOT_BYTES = Q_BYTES + 2 * KV_TILE;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + KSTAGES * KV_TILE;
-  static constexpr int BYTES = OFF_V + VSTAGES * KV_TILE;
+  static constexpr int OFF_K = Q_BYTES;
+  static constexpr int OFF_V = Q_BYTES + KV_TILE;
+  static constexpr int BYTES = SLOTS * SLOT_BYTES;
   static constexpr int SMEM = BYTES + 1024;            // slack for 1024-byte alignment
   static constexpr uint32_t IDESC_S = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(KEYS >> 3) << 17) |
                                       ((uint32_t)(ROWS >> 4) << 24);
@@ -89,6 +107,17 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred P;\n\tmbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Non-blocking look at a phase (for polling several barriers in turn).
+__device__ __forceinline__ bool mbar_probe(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\tmbarrier.test_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, P;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -144,7 +173,7 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");
 }
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_ld32p(uint32_t taddr, uint32_t* r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
       "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
@@ -155,7 +184,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_st32p(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
       "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
@@ -229,373 +258,428 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
                int nb_pad, int ksel, uint16_t* __restrict__ out, float* __restrict__ lse, int* status) {
   using L = Layout<D>;
   extern __shared__ unsigned char smem_raw[];
-  __shared__ uint32_t selm[2][SPARK_MAX_BLOCKS / 32];
-  __shared__ uint32_t unionm[SPARK_MAX_BLOCKS / 32];
-  __shared__ __align__(8) uint64_t bars[2 * KSTAGES + 2 * VSTAGES + 8];
-  __shared__ float red_max[2][2][ROWS];   // [tile parity][column half][row]
-  __shared__ float red_l[2][ROWS];
+  __shared__ uint32_t selm[SLOTS][2][MASK_WORDS];
+  __shared__ uint32_t unionm[SLOTS][MASK_WORDS];
+  // per slot: q_full, k_full, k_empty, v_full, v_empty, s_full, p_full; then drain
+  __shared__ __align__(8) uint64_t bars[7 * SLOTS + 1];
   __shared__ uint32_t tmem_base_sh;
-  __shared__ int count_sh[12];
-  __shared__ int abort_sh;
-  __shared__ int issued_sh[2], consumed_sh[2], q_seen_sh, mma_used_sh;
+  __shared__ int count_sh[THREADS / 32][SLOTS];
+  __shared__ int abort_sh, mma_used_sh;
+  __shared__ int issued_sh[SLOTS][2], consumed_sh[SLOTS][2], q_seen_sh[SLOTS];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int pair = blockIdx.x, bh = blockIdx.y;
-  const int a0 = 2 * pair, a1 = 2 * pair + 1;
-  const bool half1_valid = a1 < nb;
+  const int bh = blockIdx.y;
+  const int npairs = (nb + 1) >> 1;
   const int nwords = (nb + 31) >> 5;
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sQ = base + L::OFF_Q, sK = base + L::OFF_K, sV = base + L::OFF_V;
   const uint32_t bar0 = smem_u32(&bars[0]);
-  auto k_full = [&](int s) { return bar0 + 8u * s; };
-  auto k_empty = [&](int s) { return bar0 + 8u * (KSTAGES + s); };
-  auto v_full = [&](int s) { return bar0 + 8u * (2 * KSTAGES + s); };
-  auto v_empty = [&](int s) { return bar0 + 8u * (2 * KSTAGES + VSTAGES + s); };
-  const uint32_t bx = bar0 + 8u * (2 * KSTAGES + 2 * VSTAGES);
-  const uint32_t q_full = bx;
-  auto s_full = [&](int i) { return bx + 8u * (1 + i); };
-  auto p_full = [&](int i) { return bx + 8u * (3 + i); };
-  const uint32_t o_done = bx + 8u * 5;
-  const uint32_t drain = bx + 8u * 6;
+  auto q_full = [&](int s) { return bar0 + 8u * (7 * s + 0); };
+  auto k_full = [&](int s) { return bar0 + 8u * (7 * s + 1); };
+  auto k_empty = [&](int s) { return bar0 + 8u * (7 * s + 2); };
+  auto v_full = [&](int s) { return bar0 + 8u * (7 * s + 3); };
+  auto v_empty = [&](int s) { return bar0 + 8u * (7 * s + 4); };
+  auto s_full = [&](int s) { return bar0 + 8u * (7 * s + 5); };
+  auto p_full = [&](int s) { return bar0 + 8u * (7 * s + 6); };
+  const uint32_t drain = bar0 + 8u * (7 * SLOTS);
+  auto sQ = [&](int s) { return base + (uint32_t)(s * L::SLOT_BYTES + L::OFF_Q); };
+  auto sK = [&](int s) { return base + (uint32_t)(s * L::SLOT_BYTES + L::OFF_K); };
+  auto sV = [&](int s) { return base + (uint32_t)(s * L::SLOT_BYTES + L::OFF_V); };
 
-  // ---- prologue: selection masks of both query blocks, their union
-  for (int i = tid; i < SPARK_MAX_BLOCKS / 32; i += THREADS) { selm[0][i] = 0u; selm[1][i] = 0u; }
+  // ---- prologue: selection masks of the four query blocks, per-slot unions
+  for (int i = tid; i < SLOTS * 2 * MASK_WORDS; i += THREADS) (&selm[0][0][0])[i] = 0u;
   if (tid == 0) {
-    abort_sh = 0; q_seen_sh = 0; mma_used_sh = 0;
-    issued_sh[0] = issued_sh[1] = 0; consumed_sh[0] = consumed_sh[1] = 0;
-    for (int s = 0; s < KSTAGES; ++s) { mbar_init(k_full(s), 1); mbar_init(k_empty(s), 1); }
-    for (int s = 0; s < VSTAGES; ++s) { mbar_init(v_full(s), 1); mbar_init(v_empty(s), 1); }
-    mbar_init(q_full, 1);
-    mbar_init(s_full(0), 1); mbar_init(s_full(1), 1);
-    mbar_init(p_full(0), 256); mbar_init(p_full(1), 256);
-    mbar_init(o_done, 1);
+    abort_sh = 0;
+    mma_used_sh = 0;
+    for (int s = 0; s < SLOTS; ++s) {
+      q_seen_sh[s] = 0;
+      issued_sh[s][0] = issued_sh[s][1] = 0;
+      consumed_sh[s][0] = consumed_sh[s][1] = 0;
+      mbar_init(q_full(s), 1);
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
+      mbar_init(v_full(s), 1);
+      mbar_init(v_empty(s), 1);
+      mbar_init(s_full(s), 1);
+      mbar_init(p_full(s), ROWS);
+    }
     mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 9) {
+  if (warp == 10) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_sh)),
                  "r"(TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   __syncthreads();
-  {
-    const int32_t* s0 = sel + ((size_t)bh * nb + a0) * ksel;
+  for (int qb = 0; qb < 2 * SLOTS; ++qb) {
+    const int blk = 2 * SLOTS * blockIdx.x + qb;
+    if (blk >= nb) break;
+    const int32_t* sp = sel + ((size_t)bh * nb + blk) * ksel;
+    uint32_t* m = selm[qb >> 1][qb & 1];
     for (int i = tid; i < ksel; i += THREADS) {
-      const int b = s0[i];
-      if ((unsigned)b < (unsigned)nb) atomicOr(&selm[0][b >> 5], 1u << (b & 31));
+      const int b = sp[i];
+      if ((unsigned)b < (unsigned)nb) atomicOr(&m[b >> 5], 1u << (b & 31));
       else set_status(status, STATUS_BAD_INPUT);
-    }
-    if (half1_valid) {
-      const int32_t* s1 = sel + ((size_t)bh * nb + a1) * ksel;
-      for (int i = tid; i < ksel; i += THREADS) {
-        const int b = s1[i];
-        if ((unsigned)b < (unsigned)nb) atomicOr(&selm[1][b >> 5], 1u << (b & 31));
-        else set_status(status, STATUS_BAD_INPUT);
-      }
     }
   }
   fence_before();
   __syncthreads();
   fence_after();
-  int cnt = 0;
-  for (int w = tid; w < nwords; w += THREADS) {
-    const uint32_t u = selm[0][w] | selm[1][w];
-    unionm[w] = u;
-    cnt += __popc(u);
+  {
+    int c0 = 0, c1 = 0;
+    for (int w = tid; w < nwords; w += THREADS) {
+      const uint32_t u0 = selm[0][0][w] | selm[0][1][w];
+      const uint32_t u1 = selm[1][0][w] | selm[1][1][w];
+      unionm[0][w] = u0;
+      unionm[1][w] = u1;
+      c0 += __popc(u0);
+      c1 += __popc(u1);
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      c0 += __shfl_xor_sync(0xffffffffu, c0, o);
+      c1 += __shfl_xor_sync(0xffffffffu, c1, o);
+    }
+    if (lane == 0) {
+      count_sh[warp][0] = c0;
+      count_sh[warp][1] = c1;
+    }
   }
-  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-  if (lane == 0) count_sh[warp] = cnt;
   __syncthreads();
-  int U = 0;
-  for (int w = 0; w < THREADS / 32; ++w) U += count_sh[w];
-  const int TE = (U + 1) >> 1;                         // exact tiles (two union blocks each)
-  const int T = TE + (nb + KEYS - 1) / KEYS;           // plus summary tiles
+  int TE[SLOTS], T[SLOTS];
+  const int TS = (nb + KEYS - 1) / KEYS;               // summary tiles
+#pragma unroll
+  for (int s = 0; s < SLOTS; ++s) {
+    int U = 0;
+    for (int w = 0; w < THREADS / 32; ++w) U += count_sh[w][s];
+    TE[s] = (U + 1) >> 1;                                // exact tiles (two union blocks each)
+    T[s] = (SLOTS * blockIdx.x + s < npairs) ? TE[s] + TS : 0;
+  }
   const uint32_t tmem = tmem_base_sh;
   constexpr int NONE = 1 << 30;
 
-  if (warp == 8 || warp == 10) {
-    // ------------------------------------------------ TMA producers (warp 8: Q and K, warp 10: V)
-    const int pidx = warp == 8 ? 0 : 1;
-    if (lane == 0) {
-      const bool isk = pidx == 0;
-      const int stages = isk ? KSTAGES : VSTAGES;
-      if (isk) {
-        const int qrow = bh * N + a0 * BLK;
-        mbar_arrive_tx(q_full, L::Q_BYTES);
+  if (warp < 8) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(SOFTMAX_REGS));
+    // ------------------------------------------------ softmax of slot warp / 4, one thread per row
+    const int s = warp >> 2;
+    const int Ts = T[s], TEs = TE[s];
+    if (Ts > 0) {
+      const int a0 = 2 * (SLOTS * blockIdx.x + s);
+      const int r = (warp & 3) * 32 + lane;              // query row 0..127 of the pair
+      const int qh = r >> 6;                             // which of the two query blocks
+      const bool row_valid = qh == 0 || a0 + 1 < nb;     // uniform per warp
+      const uint32_t* mymask = selm[s][qh];
+      const uint32_t* um = unionm[s];
+      const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+      const uint32_t sc = tmem + lane_base + S_COL + 128u * (uint32_t)s;
+      const uint32_t oc = tmem + lane_base + O_COL + 128u * (uint32_t)s;
+      const float sl2 = (1.0f / sqrtf((float)D)) * 1.4426950408889634f;
+      const uint64_t sc2 = f2(sl2, sl2);
+      float m_ref = -INFINITY, l = 0.f;
+      int cur = next_block(um, 0, nwords);
+      bool ok = true;
+      for (int j = 0; j < Ts; ++j) {
+        // the tile's blocks (or summary range) and this row's masks, before the wait
+        const bool comp = j >= TEs;
+        bool t0 = false, t1 = false;
+        uint32_t ex[4] = {~0u, ~0u, ~0u, ~0u};
+        int c0 = 0;
+        if (!comp) {
+          const int b0 = cur;
+          const int b1 = next_block(um, b0 + 1, nwords);
+          cur = b1 < NONE ? next_block(um, b1 + 1, nwords) : NONE;
+          t0 = row_valid && ((mymask[b0 >> 5] >> (b0 & 31)) & 1u);
+          t1 = row_valid && b1 < NONE && ((mymask[b1 >> 5] >> (b1 & 31)) & 1u);
+        } else {
+          c0 = (j - TEs) * KEYS;
+          if (row_valid) {
 #pragma unroll
-        for (int a = 0; a < L::KATOMS; ++a) tma_load_2d(sQ + a * L::Q_ATOM, &maps.q, 64 * a, qrow, q_full);
+            for (int w = 0; w < 4; ++w) {
+              const int lo = c0 + 32 * w;
+              uint32_t e = (lo >> 5) < nwords ? mymask[lo >> 5] : ~0u;
+              if (lo + 32 > nb) e |= lo >= nb ? ~0u : (~0u << (nb - lo));
+              ex[w] = e;
+            }
+          }
+        }
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full(s), j & 1, status));
+        fence_after();
+        const bool ld0 = ok && (comp || t0), ld1 = ok && (comp || t1);   // uniform per warp
+        uint32_t sa[64], sb[64];                         // columns 0..63 / 64..127 of S_j
+        if (ld0) {
+          tmem_ld32p(sc, sa);
+          tmem_ld32p(sc + 32u, sa + 32);
+        }
+        if (ld1) {
+          tmem_ld32p(sc + 64u, sb);
+          tmem_ld32p(sc + 96u, sb + 32);
+        }
+        if (ld0 || ld1) tmem_ld_wait();
+        float mt = -INFINITY;
+        const float* brow = beta + (size_t)bh * nb_pad + c0;   // summary tiles only
+        if (!comp) {
+          float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          if (ld0) {
+#pragma unroll
+            for (int c = 0; c < 64; c += 8)
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                mc[i] = max3(mc[i], __uint_as_float(sa[c + 2 * i]), __uint_as_float(sa[c + 2 * i + 1]));
+          }
+          if (ld1) {
+#pragma unroll
+            for (int c = 0; c < 64; c += 8)
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                mc[i] = max3(mc[i], __uint_as_float(sb[c + 2 * i]), __uint_as_float(sb[c + 2 * i + 1]));
+          }
+          mt = fmaxf(max3(mc[0], mc[1], mc[2]), mc[3]) * sl2;
+        } else if (ok) {
+          // x = s / sqrt(d) + beta (log2 units), -inf where the row selected the block
+#pragma unroll
+          for (int c4 = 0; c4 < 32; ++c4) {
+            const float4 bb = __ldg(reinterpret_cast<const float4*>(brow) + c4);
+            const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = 4 * c4 + e;
+              uint32_t& sv = c < 64 ? sa[c] : sb[c - 64];
+              const float x = ((ex[c >> 5] >> (c & 31)) & 1u)
+                                  ? -INFINITY
+                                  : fmaf(__uint_as_float(sv), sl2, bv[e] * 1.4426950408889634f);
+              sv = __float_as_uint(x);
+              mt = fmaxf(mt, x);
+            }
+          }
+        }
+        // lazy reference maximum
+        float m_new = m_ref, corr = 1.f;
+        bool resc = false;
+        if (mt > -INFINITY) {
+          if (m_ref == -INFINITY) {
+            m_new = mt;
+          } else if (mt > m_ref + LAZY_RESCALE) {
+            m_new = mt;
+            corr = ex2(m_ref - mt);
+            resc = true;
+          }
+        }
+        if (ok && __any_sync(0xffffffffu, resc)) {
+          // O is idle here: S_j completing means P_{j-1} V_{j-1} has completed
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32p(oc + 32u * cc, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
+            tmem_st32p(oc + 32u * cc, o);
+          }
+        }
+        // P_j over the first 64 columns of the S buffer, one 64-key half at a time
+        float rs = 0.f;
+        const bool live = comp ? (m_new != -INFINITY && ok) : true;
+        const uint64_t mul2 = comp ? f2(1.f, 1.f) : sc2, nm2 = f2(-m_new, -m_new);
+        auto make_p = [&](const uint32_t(&sv)[64], int hh, bool take) {
+          uint32_t pw[32];
+          if (take) {
+            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+            for (int c = 0; c < 64; c += 2) {
+              float u0, u1;
+              unf2(ffma2(f2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), mul2, nm2), u0, u1);
+              const float p0 = ex2(u0), p1 = ex2(u1);
+              acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], f2(p0, p1));
+              pw[c >> 1] = cvt_bf2(p0, p1);
+            }
+            float r0, r1, r2, r3;
+            unf2(fadd2(acc[0], acc[1]), r0, r1);
+            unf2(fadd2(acc[2], acc[3]), r2, r3);
+            rs += (r0 + r2) + (r1 + r3);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) pw[c] = 0u;
+          }
+          if (ok) tmem_st32p(sc + 32u * hh, pw);
+        };
+        make_p(sa, 0, comp ? live : ld0);     // uniform per warp
+        make_p(sb, 1, comp ? live : ld1);
+        l = l * corr + rs;
+        m_ref = m_new;
+        if (ok) {
+          tmem_st_wait();
+          fence_before();
+          mbar_arrive(p_full(s));
+        }
       }
-      const uint32_t ring = isk ? sK : sV;
-      int cur = next_block(unionm, 0, nwords);
-      int issued = 0;
-      for (int j = 0; j < T; ++j) {
-        const int st = j % stages;
-        const uint32_t empty = isk ? k_empty(st) : v_empty(st);
-        const uint32_t full = isk ? k_full(st) : v_full(st);
-        if (j >= stages && !mbar_wait(empty, ((j / stages) - 1) & 1, status)) {
+      // ---- epilogue: O / l -> out[perm[row]]
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full(s), Ts & 1, status));
+      if (!ok) atomicExch(&abort_sh, 1);
+      fence_after();
+      ok = __all_sync(0xffffffffu, ok && !(*(volatile int*)&abort_sh));
+      if (ok && row_valid) {
+        const int pos = a0 * BLK + r;
+        const int orig = perm[(size_t)bh * N + pos];
+        const bool dst_ok = (unsigned)orig < (unsigned)N;
+        if (!dst_ok) set_status(status, STATUS_BAD_INPUT);
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)bh * N + (dst_ok ? orig : 0)) * D);
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32p(oc + 32u * cc, o);
+          tmem_ld_wait();
+          if (dst_ok) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e2 = 0; e2 < 4; ++e2) {
+                const int e = 8 * q4 + 2 * e2;
+                w[e2] = cvt_bf2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
+              }
+              dst[cc * 4 + q4] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
+        }
+        if (lse != nullptr && dst_ok) lse[(size_t)bh * N + orig] = (m_ref + log2f(l)) * 0.6931471805599453f;
+      }
+    }
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(OTHER_REGS));
+  if (warp == 8 || warp == 9) {
+    // ------------------------------------------------ TMA producer of slot warp - 8
+    const int s = warp - 8;
+    if (lane == 0 && T[s] > 0) {
+      const int a0 = 2 * (SLOTS * blockIdx.x + s);
+      mbar_arrive_tx(q_full(s), L::Q_BYTES);
+#pragma unroll
+      for (int a = 0; a < L::KATOMS; ++a)
+        tma_load_2d(sQ(s) + a * L::Q_ATOM, &maps.q, 64 * a, bh * N + a0 * BLK, q_full(s));
+      const uint32_t* um = unionm[s];
+      int cur = next_block(um, 0, nwords);
+      int ik = 0, iv = 0;
+      for (int j = 0; j < T[s]; ++j) {
+        const CUtensorMap *mk, *mv;
+        int row0, row1;
+        if (j < TE[s]) {
+          const int b0 = cur;
+          int b1 = next_block(um, b0 + 1, nwords);
+          cur = b1 < NONE ? next_block(um, b1 + 1, nwords) : NONE;
+          if (b1 >= NONE) b1 = b0;                     // odd count: the second half repeats, masked
+          row0 = bh * N + b0 * BLK;
+          row1 = bh * N + b1 * BLK;
+          mk = &maps.k;
+          mv = &maps.v;
+        } else {
+          row0 = bh * nb_pad + (j - TE[s]) * KEYS;
+          row1 = row0 + BLK;
+          mk = &maps.kt;
+          mv = &maps.vt;
+        }
+        // K_j once S_{j-1} has read the buffer
+        if (j > 0 && !mbar_wait(k_empty(s), (j - 1) & 1, status)) {
           atomicExch(&abort_sh, 1);
           break;
         }
         if (*(volatile int*)&abort_sh) break;
-        const uint32_t dst = ring + st * L::KV_TILE;
-        mbar_arrive_tx(full, L::KV_TILE);
-        const CUtensorMap* m;
-        int row0, row1;
-        if (j < TE) {
-          const int b0 = cur;
-          int b1 = next_block(unionm, b0 + 1, nwords);
-          cur = b1 < NONE ? next_block(unionm, b1 + 1, nwords) : NONE;
-          if (b1 >= NONE) b1 = b0;                   // odd count: the second half repeats, masked
-          row0 = bh * N + b0 * BLK;
-          row1 = bh * N + b1 * BLK;
-          m = isk ? &maps.k : &maps.v;
-        } else {
-          row0 = bh * nb_pad + (j - TE) * KEYS;
-          row1 = row0 + BLK;
-          m = isk ? &maps.kt : &maps.vt;
-        }
+        mbar_arrive_tx(k_full(s), L::KV_TILE);
 #pragma unroll
         for (int a = 0; a < L::KATOMS; ++a) {
-          tma_load_2d(dst + a * L::KV_ATOM, m, 64 * a, row0, full);
-          tma_load_2d(dst + a * L::KV_ATOM + BLK * 128, m, 64 * a, row1, full);
+          tma_load_2d(sK(s) + a * L::KV_ATOM, mk, 64 * a, row0, k_full(s));
+          tma_load_2d(sK(s) + a * L::KV_ATOM + BLK * 128, mk, 64 * a, row1, k_full(s));
         }
-        issued = j + 1;
+        ik = j + 1;
+        // V_j once P_{j-1} V_{j-1} has read the buffer
+        if (j > 0 && !mbar_wait(v_empty(s), (j - 1) & 1, status)) {
+          atomicExch(&abort_sh, 1);
+          break;
+        }
+        if (*(volatile int*)&abort_sh) break;
+        mbar_arrive_tx(v_full(s), L::KV_TILE);
+#pragma unroll
+        for (int a = 0; a < L::KATOMS; ++a) {
+          tma_load_2d(sV(s) + a * L::KV_ATOM, mv, 64 * a, row0, v_full(s));
+          tma_load_2d(sV(s) + a * L::KV_ATOM + BLK * 128, mv, 64 * a, row1, v_full(s));
+        }
+        iv = j + 1;
       }
-      issued_sh[pidx] = issued;
+      issued_sh[s][0] = ik;
+      issued_sh[s][1] = iv;
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------ MMA issuer
+  } else if (warp == 10) {
+    // ------------------------------------------------ MMA issuer, both slots
     if (lane == 0) {
-      bool ok = mbar_wait(q_full, 0, status);
-      if (ok) q_seen_sh = 1;
-      int kc = 0, vc = 0;   // K / V tiles whose arrival was observed
-      const uint64_t dQ0 = sdesc(sQ, 16, 1024);
-      const uint64_t dK0 = sdesc(sK, 16, 1024);
-      const uint64_t dV0 = sdesc(sV, L::KV_ATOM, 1024);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % KSTAGES;
-        if (!mbar_wait(k_full(st), (j / KSTAGES) & 1, status)) return false;
-        kc = j + 1;
-        fence_after();
-        const uint32_t d = tmem + S_COL + 128u * (uint32_t)(j & 1);
-        const uint64_t dk = dK0 + (uint64_t)((st * L::KV_TILE) >> 4);
+      bool ok = true;
+      int jp[SLOTS] = {0, 0};                          // next P V product per slot
+      int kc[SLOTS] = {0, 0}, vc[SLOTS] = {0, 0};      // K / V arrivals observed
+      auto issue_s = [&](int s) {
+        const uint32_t d = tmem + S_COL + 128u * (uint32_t)s;
+        const uint64_t dq = sdesc(sQ(s), 16, 1024), dk = sdesc(sK(s), 16, 1024);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t qo = (uint64_t)(((ks >> 2) * L::Q_ATOM + (ks & 3) * 32) >> 4);
           const uint64_t ko = (uint64_t)(((ks >> 2) * L::KV_ATOM + (ks & 3) * 32) >> 4);
-          mma_f16(d, dQ0 + qo, dk + ko, L::IDESC_S, ks > 0 ? 1u : 0u);
+          mma_f16(d, dq + qo, dk + ko, L::IDESC_S, ks > 0 ? 1u : 0u);
         }
-        mma_commit(s_full(j & 1));
-        mma_commit(k_empty(st));
-        mma_used_sh = 1;
-        return true;
+        mma_commit(k_empty(s));
       };
-      if (ok && T > 0) ok = issue_s(0);
-      if (ok && T > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < T; ++j) {
-        const int st = j % VSTAGES;
-        if (!mbar_wait(p_full(j & 1), (j >> 1) & 1, status)) { ok = false; break; }
-        if (!mbar_wait(v_full(st), (j / VSTAGES) & 1, status)) { ok = false; break; }
-        vc = j + 1;
+      for (int s = 0; s < SLOTS && ok; ++s) {
+        if (T[s] == 0) continue;
+        if (!mbar_wait(q_full(s), 0, status)) { ok = false; break; }
+        q_seen_sh[s] = 1;
+        if (!mbar_wait(k_full(s), 0, status)) { ok = false; break; }
+        kc[s] = 1;
         fence_after();
-        const uint64_t dv = dV0 + (uint64_t)((st * L::KV_TILE) >> 4);
-        const uint32_t pa = tmem + P_COL + 64u * (uint32_t)(j & 1);
-        const uint32_t acc0 = j > 0 ? 1u : 0u;
-#pragma unroll
-        for (int kk = 0; kk < KEYS / 16; ++kk)
-          mma_ts(tmem + O_COL, pa + 8u * kk, dv + (uint64_t)((kk * 2048) >> 4), L::IDESC_O, kk > 0 ? 1u : acc0);
-        mma_commit(o_done);
-        mma_commit(v_empty(st));
-        // S buffer j&1 is free again (the softmax read S_j before releasing P_j)
-        if (j + 2 < T && !issue_s(j + 2)) { ok = false; break; }
+        issue_s(s);
+        mma_commit(s_full(s));
+        mma_used_sh = 1;
       }
-      if (ok && T > 0) {
-        // the last commit must land before this CTA's shared memory is released
-        const int jl = T - 1;
-        ok = mbar_wait(v_empty(jl % VSTAGES), (jl / VSTAGES) & 1, status);
+      unsigned long long t_last = globaltimer();
+      while (ok && (jp[0] < T[0] || jp[1] < T[1])) {
+        bool progressed = false;
+        for (int s = 0; s < SLOTS && ok; ++s) {
+          const int j = jp[s];
+          if (j >= T[s] || !mbar_probe(p_full(s), j & 1)) continue;
+          if (!mbar_wait(v_full(s), j & 1, status)) { ok = false; break; }
+          vc[s] = j + 1;
+          fence_after();
+          const uint64_t dv = sdesc(sV(s), L::KV_ATOM, 1024);
+          const uint32_t pa = tmem + S_COL + 128u * (uint32_t)s;
+          const uint32_t od = tmem + O_COL + 128u * (uint32_t)s;
+#pragma unroll
+          for (int kk = 0; kk < KEYS / 16; ++kk)
+            mma_ts(od, pa + 8u * kk, dv + (uint64_t)((kk * 2048) >> 4), L::IDESC_O, (kk > 0 || j > 0) ? 1u : 0u);
+          mma_commit(v_empty(s));
+          if (j + 1 < T[s]) {
+            if (!mbar_wait(k_full(s), (j + 1) & 1, status)) { ok = false; break; }
+            kc[s] = j + 2;
+            fence_after();
+            issue_s(s);
+          }
+          // S_{j+1} ready, or (after the last tile) O complete
+          mma_commit(s_full(s));
+          jp[s] = j + 1;
+          progressed = true;
+        }
+        if (progressed) {
+          t_last = globaltimer();
+        } else if (globaltimer() - t_last > WAIT_NS) {
+          set_status(status, STATUS_TIMEOUT);
+          ok = false;
+        }
+      }
+      // the last arrivals must land before this CTA's shared memory is released
+      for (int s = 0; s < SLOTS && ok; ++s) {
+        if (T[s] == 0) continue;
+        ok = mbar_wait(v_empty(s), (T[s] - 1) & 1, status) && mbar_wait(k_empty(s), (T[s] - 1) & 1, status);
       }
       if (!ok) atomicExch(&abort_sh, 1);
-      consumed_sh[0] = kc;
-      consumed_sh[1] = vc;
-    }
-  } else {
-    // ------------------------------------------------ softmax warps 0-7
-    const int h = warp >> 2;                 // column half of the 128-key tile
-    const int r = (warp & 3) * 32 + lane;    // query row 0..127 of the pair
-    const int qh = r >> 6;                   // which of the two query blocks
-    const bool row_valid = qh == 0 || half1_valid;   // uniform per warp
-    const uint32_t* mymask = selm[qh];
-    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const float sl2 = (1.0f / sqrtf((float)D)) * 1.4426950408889634f;
-    float m_ref = -INFINITY, l = 0.f;
-    int cur = next_block(unionm, 0, nwords);
-    bool ok = true;
-    for (int j = 0; j < T; ++j) {
-      // (a warp that gave up keeps taking part in the named barriers)
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full(j & 1), (j >> 1) & 1, status));
-      fence_after();
-      uint32_t sa[32], sb[32];
-      if (ok) {
-        tmem_ld32(tmem + lane_base + S_COL + 128u * (uint32_t)(j & 1) + 64u * h, sa);
-        tmem_ld32(tmem + lane_base + S_COL + 128u * (uint32_t)(j & 1) + 64u * h + 32u, sb);
-        tmem_ld_wait();
-      } else {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) { sa[c] = 0u; sb[c] = 0u; }
-      }
-      auto sv = [&](int c) { return __uint_as_float(c < 32 ? sa[c] : sb[c - 32]); };
-      bool take = false, comp = j >= TE;
-      uint64_t excl = 0;
-      float x[64];
-      float mx = -INFINITY;
-      if (!comp) {
-        const int b0 = cur;
-        const int b1 = next_block(unionm, b0 + 1, nwords);
-        cur = b1 < NONE ? next_block(unionm, b1 + 1, nwords) : NONE;
-        const int blk = h == 0 ? b0 : b1;
-        take = row_valid && blk < NONE && ((mymask[blk >> 5] >> (blk & 31)) & 1u);   // uniform per warp
-        if (take) {
-          float mc[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) mc[i] = fmaxf(sv(2 * i), sv(2 * i + 1));
-#pragma unroll
-          for (int c = 8; c < 64; c += 8) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) mc[i] = max3(mc[i], sv(c + 2 * i), sv(c + 2 * i + 1));
-          }
-          mx = fmaxf(max3(mc[0], mc[1], mc[2]), mc[3]) * sl2;
-        }
-      } else {
-        const int c0 = (j - TE) * KEYS + 64 * h;
-        if (c0 < nb) {
-          excl = (uint64_t)mymask[c0 >> 5];
-          if ((c0 >> 5) + 1 < nwords) excl |= (uint64_t)mymask[(c0 >> 5) + 1] << 32;
-          if (c0 + BLK > nb) excl |= ~0ull << (nb - c0);
-        } else {
-          excl = ~0ull;
-        }
-        if (!row_valid) excl = ~0ull;
-        const float4* bt = reinterpret_cast<const float4*>(beta + (size_t)bh * nb_pad + c0);
-#pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const float4 bb = __ldg(bt + c4);
-          const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 4 * c4 + e;
-            const float v = fmaf(sv(c), sl2, bv[e] * 1.4426950408889634f);
-            x[c] = ((excl >> c) & 1ull) ? -INFINITY : v;
-            mx = fmaxf(mx, x[c]);
-          }
-        }
-      }
-      // row max over both column halves
-      red_max[j & 1][h][r] = mx;
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      const float mt = fmaxf(red_max[j & 1][0][r], red_max[j & 1][1][r]);
-      float m_new = m_ref, corr = 1.f;
-      bool resc = false;
-      if (mt > -INFINITY) {
-        if (m_ref == -INFINITY) {
-          m_new = mt;
-        } else if (mt > m_ref + LAZY_RESCALE) {
-          m_new = mt;
-          corr = ex2(m_ref - mt);
-          resc = true;
-        }
-      }
-      uint32_t pw[32];
-      float rs = 0.f;
-      if (!comp && take) {
-        const uint64_t sc2 = f2(sl2, sl2), nm2 = f2(-m_new, -m_new);
-        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          float t0, t1;
-          unf2(ffma2(f2(sv(c), sv(c + 1)), sc2, nm2), t0, t1);
-          const float p0 = ex2(t0), p1 = ex2(t1);
-          acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], f2(p0, p1));
-          pw[c >> 1] = cvt_bf2(p0, p1);
-        }
-        float r0, r1, r2, r3;
-        unf2(fadd2(acc[0], acc[1]), r0, r1);
-        unf2(fadd2(acc[2], acc[3]), r2, r3);
-        rs = (r0 + r2) + (r1 + r3);
-      } else if (comp && m_new != -INFINITY) {
-        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float p0 = ex2(x[c] - m_new), p1 = ex2(x[c + 1] - m_new);
-          rs4[(c >> 1) & 3] += p0 + p1;
-          pw[c >> 1] = cvt_bf2(p0, p1);
-        }
-        rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-      } else {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) pw[c] = 0u;
-      }
-      l = l * corr + rs;
-      m_ref = m_new;
-      // previous P V product complete: O may be rescaled, P buffer j&1 reused
-      if (ok && j > 0) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, status));
-      fence_after();
-      if (ok) {
-        if (__any_sync(0xffffffffu, resc)) {
-#pragma unroll 1
-          for (int cc = 0; cc < 2; ++cc) {
-            const uint32_t oc = tmem + lane_base + O_COL + 64u * h + 32u * cc;
-            if (64 * h + 32 * cc < D) {
-              uint32_t o[32];
-              tmem_ld32(oc, o);
-              tmem_ld_wait();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
-              tmem_st32(oc, o);
-            }
-          }
-          tmem_st_wait();
-        }
-        tmem_st32(tmem + lane_base + P_COL + 64u * (uint32_t)(j & 1) + 32u * h, pw);
-        tmem_st_wait();
-        fence_before();
-        mbar_arrive(p_full(j & 1));
+      for (int s = 0; s < SLOTS; ++s) {
+        consumed_sh[s][0] = kc[s];
+        consumed_sh[s][1] = vc[s];
       }
     }
-    // ---- epilogue: O / l -> out[perm[row]], each thread its 64 columns
-    if (ok && T > 0) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (T - 1) & 1, status));
-    if (!ok) atomicExch(&abort_sh, 1);
-    fence_after();
-    red_l[h][r] = l;
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    const float lt = red_l[0][r] + red_l[1][r];
-    ok = ok && !(*(volatile int*)&abort_sh);
-    if (ok && row_valid && 64 * h < D) {
-      const int pos = a0 * BLK + r;
-      const int orig = perm[(size_t)bh * N + pos];
-      const bool dst_ok = (unsigned)orig < (unsigned)N;
-      if (!dst_ok) set_status(status, STATUS_BAD_INPUT);
-      const float inv = lt > 0.f ? 1.f / lt : 0.f;
-      uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)bh * N + (dst_ok ? orig : 0)) * D + 64 * h);
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(tmem + lane_base + O_COL + 64u * h + 32u * cc, o);
-        tmem_ld_wait();
-        if (dst_ok) {
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e2 = 0; e2 < 4; ++e2) {
-              const int e = 8 * q4 + 2 * e2;
-              w[e2] = cvt_bf2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
-            }
-            dst[cc * 4 + q4] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
-      }
-      if (h == 0 && lse != nullptr && dst_ok) lse[(size_t)bh * N + orig] = (m_ref + log2f(lt)) * 0.6931471805599453f;
-    }
+  }
   }
 
   // ---- teardown: drain own copies / MMAs (bounded), free TMEM
@@ -603,15 +687,14 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
   __syncthreads();
   fence_after();
   if (abort_sh) {
-    if ((warp == 8 || warp == 10) && lane == 0) {
+    if ((warp == 8 || warp == 9) && lane == 0) {
       // copies issued but never observed by the MMA thread
-      const int pi = warp == 8 ? 0 : 1;
-      const int stages = pi == 0 ? KSTAGES : VSTAGES;
-      if (pi == 0 && !q_seen_sh) mbar_wait(q_full, 0, status);
-      for (int j = consumed_sh[pi]; j < issued_sh[pi]; ++j)
-        mbar_wait(pi == 0 ? k_full(j % stages) : v_full(j % stages), (j / stages) & 1, status);
+      const int s = warp - 8;
+      if (T[s] > 0 && !q_seen_sh[s]) mbar_wait(q_full(s), 0, status);
+      for (int j = consumed_sh[s][0]; j < issued_sh[s][0]; ++j) mbar_wait(k_full(s), j & 1, status);
+      for (int j = consumed_sh[s][1]; j < issued_sh[s][1]; ++j) mbar_wait(v_full(s), j & 1, status);
     }
-    if (warp == 9 && lane == 0 && mma_used_sh) {
+    if (warp == 10 && lane == 0 && mma_used_sh) {
       mma_commit(drain);
       mbar_wait(drain, 0, status);
     }
@@ -619,7 +702,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
     __syncthreads();
     fence_after();
   }
-  if (warp == 9) {
+  if (warp == 10) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
   }
 }
@@ -668,9 +751,18 @@ static cudaError_t run(const Plan& pl, const int32_t* perm, const int32_t* sel, 
       !make_map(&maps.vt, ws_at<void>(ws, pl.off_vt), srows, D, 64))
     return cudaErrorInvalidValue;
   auto kern = attn_tc_kernel<D>;
+  // the register split is only sound with exactly LAUNCH_REGS per thread at launch
+  static int regs_ok = -1;
+  if (regs_ok < 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
+    regs_ok = fa.numRegs == LAUNCH_REGS ? 1 : 0;
+  }
+  if (!regs_ok) return cudaErrorInvalidDeviceFunction;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<dim3((pl.nb + 1) / 2, pl.BH), THREADS, Lay::SMEM, s>>>(maps, ws_at<float>(ws, pl.off_beta), perm, sel,
+  const int npairs = (pl.nb + 1) / 2;
+  kern<<<dim3((npairs + SLOTS - 1) / SLOTS, pl.BH), THREADS, Lay::SMEM, s>>>(maps, ws_at<float>(ws, pl.off_beta), perm, sel,
                                                                  pl.N, pl.nb, pl.nb_pad, pl.ksel, out, lse, status);
   return cudaGetLastError();
 }

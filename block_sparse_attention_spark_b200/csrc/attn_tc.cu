@@ -5,37 +5,34 @@
 // query rows, the M of one tcgen05 MMA. The exact branch ("Spark-H3" news
 // post, "What Spark-Attn changed": the exact branch fully computes the
 // top-ranked key/value blocks) runs over the UNION of the two blocks'
-// selected key blocks in ascending order, two 64-key blocks per 128-key
-// tile; a row only keeps the columns of blocks its own query block selected
-// (the others get zero weight; that MMA work is not counted as
-// algorithmic). The compressed branch ("MiniMax H3 Spark Attention (SM89)",
-// under the hood: a real Q per query, K/V downsampled) follows over the
-// summary table, 128 summaries per tile, each row masking the blocks it
-// selected. One running softmax over both term sets = the log-sum-exp merge
-// of the two branches.
+// selected key blocks in ascending order, one 64-key block per tile; the
+// rows of a query block that did not select the tile's block give it zero
+// weight (that MMA work is not counted as algorithmic). The compressed
+// branch ("MiniMax H3 Spark Attention (SM89)", under the hood: a real Q per
+// query, K/V downsampled) follows over the summary table, 64 summaries per
+// tile, each row masking the blocks it selected. One running softmax over
+// both term sets = the log-sum-exp merge of the two branches.
 //
 // A CTA runs two such units side by side in two independent slots (pairs
-// 2c and 2c+1), each with its own Q, K and V buffers and its own TMEM
-// columns, so that one slot's softmax overlaps the other slot's MMAs.
+// 2c and 2c+1), each with its own Q, K and V buffers and TMEM columns. Each
+// slot double-buffers S in TMEM, so the tensor cores compute S_{j+1} (and
+// P_{j-1} V_{j-1}) while the slot's softmax works on S_j.
 //
-// Roles (384 threads = three warpgroups):
+// Roles (384 threads):
 //   warps 0-3  softmax of slot 0, warps 4-7 softmax of slot 1: one thread
-//              per query row (TMEM lane = row), all 128 columns of a tile.
+//              per query row (TMEM lane = row), the 64 columns of a tile.
 //              Lazy-rescaled online softmax (the reference max moves only
 //              when the row max grows by more than 2^8); P (bf16 pairs) is
-//              written over the first 64 columns of the slot's S buffer.
+//              written over the first 32 columns of the tile's S buffer.
 //   warp 8 / 9 TMA producer of slot 0 / 1: Q once, then K_j and V_j of
-//              every tile into the slot's single K and V buffers.
-//   warp 10    TMEM allocator + the MMA-issuing thread (warp 11 idles). Per slot and tile:
-//              O += P_j V_j (M128 N=d K=128, P read from TMEM, V an MN-major
-//              smem operand), then S_{j+1} = Q K_{j+1}^T (M128 N128 K=d,
-//              K-major smem operands) into the same S columns, then one
-//              commit. The MMAs of a CTA complete in issue order, so the
-//              arrival of S_{j+1} also means that P_j and O are free: the
-//              softmax needs one wait per tile, and O can be rescaled in
-//              place without another.
-// TMEM columns: S of slot s at 128 s (P aliased on its first 64), O of slot
-// s at 256 + 128 s.
+//              every tile into two-stage K and V rings.
+//   warp 10/11 MMA-issuing thread of slot 0 / 1 (warp 10 also allocates
+//              TMEM): S_j = Q K_j^T (M128 N64 K=d, K-major smem operands),
+//              O += P_j V_j (M128 N=d K=64, P read from TMEM, V an MN-major
+//              smem operand). S_{j+2} goes into S_j's buffer after P_j V_j;
+//              the MMAs of one thread complete in issue order, so that
+//              reuse needs no extra wait.
+// TMEM columns of slot s (base 256 s): S buffers at +0 and +64, O at +128.
 // Every mbarrier wait is bounded (about 2 s); on expiry the kernel records
 // a timeout in the status word, drains its own copies and MMAs (again with a
 // bound), frees TMEM and returns.
@@ -49,21 +46,13 @@ namespace spark {
 namespace tc {
 
 constexpr int ROWS = 128;
-constexpr int KEYS = 128;                // keys (or summaries) per tile
+constexpr int KEYS = 64;                 // keys (or summaries) per tile = one block
 constexpr int SLOTS = 2;
+constexpr int STAGES = 2;                // K and V ring depth per slot
 constexpr int THREADS = 384;
-// Register split (setmaxnreg, per warpgroup): the block is launched with
-// LAUNCH_REGS per thread; the producer/MMA warpgroup gives registers back so
-// that each softmax thread can hold a whole 128-column S row.
-// 2*128*SOFTMAX_REGS + 128*OTHER_REGS equals THREADS*LAUNCH_REGS, so every
-// increase is covered by the decrease.
-constexpr int LAUNCH_REGS = 168;
-constexpr int SOFTMAX_REGS = 192;
-constexpr int OTHER_REGS = 120;
-static_assert(2 * 128 * SOFTMAX_REGS + 128 * OTHER_REGS == THREADS * LAUNCH_REGS, "register split must balance");
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t S_COL = 0;            // S (and P) of slot s at S_COL + 128 s
-constexpr uint32_t O_COL = 256;          // O of slot s at O_COL + 128 s
+constexpr uint32_t SLOT_COLS = 256;      // TMEM columns per slot
+constexpr uint32_t O_OFF = 128;          // O within a slot's columns
 constexpr float LAZY_RESCALE = 8.0f;     // log2 units
 constexpr unsigned long long WAIT_NS = 2000000000ull;
 constexpr int MASK_WORDS = SPARK_MAX_BLOCKS / 32;
@@ -72,14 +61,14 @@ template <int D>
 struct Layout {
   static constexpr int KATOMS = D / 64;                // 128-byte swizzle atoms along the head dim
   static constexpr int Q_ATOM = ROWS * 128;            // 128 rows x 128 B
-  static constexpr int KV_ATOM = KEYS * 128;           // 128 rows x 128 B
+  static constexpr int KV_ATOM = KEYS * 128;           // 64 rows x 128 B
   static constexpr int Q_BYTES = Q_ATOM * KATOMS;
   static constexpr int KV_TILE = KV_ATOM * KATOMS;
-  // per slot: Q, K, V
-  static constexpr int SLOT_BYTES = Q_BYTES + 2 * KV_TILE;
+  // per slot: Q, STAGES K tiles, STAGES V tiles
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = Q_BYTES;
-  static constexpr int OFF_V = Q_BYTES + KV_TILE;
+  static constexpr int OFF_V = Q_BYTES + STAGES * KV_TILE;
+  static constexpr int SLOT_BYTES = Q_BYTES + 2 * STAGES * KV_TILE;
   static constexpr int BYTES = SLOTS * SLOT_BYTES;
   static constexpr int SMEM = BYTES + 1024;            // slack for 1024-byte alignment
   static constexpr uint32_t IDESC_S = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(KEYS >> 3) << 17) |
@@ -257,14 +246,14 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
                const int32_t* __restrict__ perm, const int32_t* __restrict__ sel, int N, int nb,
                int nb_pad, int ksel, uint16_t* __restrict__ out, float* __restrict__ lse, int* status) {
   using L = Layout<D>;
+  constexpr int NBAR = 16;                             // barriers per slot
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t selm[SLOTS][2][MASK_WORDS];
   __shared__ uint32_t unionm[SLOTS][MASK_WORDS];
-  // per slot: q_full, k_full, k_empty, v_full, v_empty, s_full, p_full; then drain
-  __shared__ __align__(8) uint64_t bars[7 * SLOTS + 1];
+  __shared__ __align__(8) uint64_t bars[NBAR * SLOTS];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int count_sh[THREADS / 32][SLOTS];
-  __shared__ int abort_sh, mma_used_sh;
+  __shared__ int abort_sh, mma_used_sh[SLOTS];
   __shared__ int issued_sh[SLOTS][2], consumed_sh[SLOTS][2], q_seen_sh[SLOTS];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -273,36 +262,35 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
   const int nwords = (nb + 31) >> 5;
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t bar0 = smem_u32(&bars[0]);
-  auto q_full = [&](int s) { return bar0 + 8u * (7 * s + 0); };
-  auto k_full = [&](int s) { return bar0 + 8u * (7 * s + 1); };
-  auto k_empty = [&](int s) { return bar0 + 8u * (7 * s + 2); };
-  auto v_full = [&](int s) { return bar0 + 8u * (7 * s + 3); };
-  auto v_empty = [&](int s) { return bar0 + 8u * (7 * s + 4); };
-  auto s_full = [&](int s) { return bar0 + 8u * (7 * s + 5); };
-  auto p_full = [&](int s) { return bar0 + 8u * (7 * s + 6); };
-  const uint32_t drain = bar0 + 8u * (7 * SLOTS);
+  // barrier b of slot s; rings take the stage / buffer index i
+  auto bar = [&](int s, int b) { return bar0 + 8u * (uint32_t)(NBAR * s + b); };
+  auto q_full = [&](int s) { return bar(s, 0); };
+  auto k_full = [&](int s, int i) { return bar(s, 1 + i); };
+  auto k_empty = [&](int s, int i) { return bar(s, 3 + i); };
+  auto v_full = [&](int s, int i) { return bar(s, 5 + i); };
+  auto v_empty = [&](int s, int i) { return bar(s, 7 + i); };
+  auto s_full = [&](int s, int i) { return bar(s, 9 + i); };
+  auto p_full = [&](int s, int i) { return bar(s, 11 + i); };
+  // o_done(s, j & 1) completes with P_j V_j. Two barriers, because when S_j
+  // has completed only P_{j-2} V_{j-2} is known to be complete, and a parity
+  // wait must never run two phases behind its barrier.
+  auto o_done = [&](int s, int i) { return bar(s, 13 + i); };
+  auto drain = [&](int s) { return bar(s, 15); };
   auto sQ = [&](int s) { return base + (uint32_t)(s * L::SLOT_BYTES + L::OFF_Q); };
-  auto sK = [&](int s) { return base + (uint32_t)(s * L::SLOT_BYTES + L::OFF_K); };
-  auto sV = [&](int s) { return base + (uint32_t)(s * L::SLOT_BYTES + L::OFF_V); };
+  auto sK = [&](int s, int i) { return base + (uint32_t)(s * L::SLOT_BYTES + L::OFF_K + i * L::KV_TILE); };
+  auto sV = [&](int s, int i) { return base + (uint32_t)(s * L::SLOT_BYTES + L::OFF_V + i * L::KV_TILE); };
 
   // ---- prologue: selection masks of the four query blocks, per-slot unions
   for (int i = tid; i < SLOTS * 2 * MASK_WORDS; i += THREADS) (&selm[0][0][0])[i] = 0u;
   if (tid == 0) {
     abort_sh = 0;
-    mma_used_sh = 0;
     for (int s = 0; s < SLOTS; ++s) {
+      mma_used_sh[s] = 0;
       q_seen_sh[s] = 0;
       issued_sh[s][0] = issued_sh[s][1] = 0;
       consumed_sh[s][0] = consumed_sh[s][1] = 0;
-      mbar_init(q_full(s), 1);
-      mbar_init(k_full(s), 1);
-      mbar_init(k_empty(s), 1);
-      mbar_init(v_full(s), 1);
-      mbar_init(v_empty(s), 1);
-      mbar_init(s_full(s), 1);
-      mbar_init(p_full(s), ROWS);
+      for (int b = 0; b < NBAR; ++b) mbar_init(bar(s, b), (b == 11 || b == 12) ? ROWS : 1);
     }
-    mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 10) {
@@ -351,14 +339,13 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
   for (int s = 0; s < SLOTS; ++s) {
     int U = 0;
     for (int w = 0; w < THREADS / 32; ++w) U += count_sh[w][s];
-    TE[s] = (U + 1) >> 1;                                // exact tiles (two union blocks each)
-    T[s] = (SLOTS * blockIdx.x + s < npairs) ? TE[s] + TS : 0;
+    TE[s] = U;                                           // exact tiles: one union block each
+    T[s] = (SLOTS * blockIdx.x + s < npairs) ? U + TS : 0;
   }
   const uint32_t tmem = tmem_base_sh;
   constexpr int NONE = 1 << 30;
 
   if (warp < 8) {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(SOFTMAX_REGS));
     // ------------------------------------------------ softmax of slot warp / 4, one thread per row
     const int s = warp >> 2;
     const int Ts = T[s], TEs = TE[s];
@@ -369,85 +356,71 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
       const bool row_valid = qh == 0 || a0 + 1 < nb;     // uniform per warp
       const uint32_t* mymask = selm[s][qh];
       const uint32_t* um = unionm[s];
-      const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-      const uint32_t sc = tmem + lane_base + S_COL + 128u * (uint32_t)s;
-      const uint32_t oc = tmem + lane_base + O_COL + 128u * (uint32_t)s;
+      const uint32_t tbase = tmem + ((uint32_t)((warp & 3) * 32) << 16) + SLOT_COLS * (uint32_t)s;
+      const uint32_t oc = tbase + O_OFF;
       const float sl2 = (1.0f / sqrtf((float)D)) * 1.4426950408889634f;
       const uint64_t sc2 = f2(sl2, sl2);
       float m_ref = -INFINITY, l = 0.f;
       int cur = next_block(um, 0, nwords);
       bool ok = true;
       for (int j = 0; j < Ts; ++j) {
-        // the tile's blocks (or summary range) and this row's masks, before the wait
+        const uint32_t sc = tbase + 64u * (uint32_t)(j & 1);   // this tile's S (and P) columns
+        // the tile's block (or summary range) and this row's mask, before the wait
         const bool comp = j >= TEs;
-        bool t0 = false, t1 = false;
-        uint32_t ex[4] = {~0u, ~0u, ~0u, ~0u};
+        bool take;
+        uint32_t ex0 = ~0u, ex1 = ~0u;
         int c0 = 0;
         if (!comp) {
-          const int b0 = cur;
-          const int b1 = next_block(um, b0 + 1, nwords);
-          cur = b1 < NONE ? next_block(um, b1 + 1, nwords) : NONE;
-          t0 = row_valid && ((mymask[b0 >> 5] >> (b0 & 31)) & 1u);
-          t1 = row_valid && b1 < NONE && ((mymask[b1 >> 5] >> (b1 & 31)) & 1u);
+          const int b = cur;
+          cur = next_block(um, b + 1, nwords);
+          take = row_valid && ((mymask[b >> 5] >> (b & 31)) & 1u);
         } else {
           c0 = (j - TEs) * KEYS;
+          take = row_valid;
           if (row_valid) {
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              const int lo = c0 + 32 * w;
-              uint32_t e = (lo >> 5) < nwords ? mymask[lo >> 5] : ~0u;
-              if (lo + 32 > nb) e |= lo >= nb ? ~0u : (~0u << (nb - lo));
-              ex[w] = e;
-            }
+            ex0 = (c0 >> 5) < nwords ? mymask[c0 >> 5] : ~0u;
+            ex1 = (c0 >> 5) + 1 < nwords ? mymask[(c0 >> 5) + 1] : ~0u;
+            if (c0 + 32 > nb) ex0 |= c0 >= nb ? ~0u : (~0u << (nb - c0));
+            if (c0 + 64 > nb) ex1 |= c0 + 32 >= nb ? ~0u : (~0u << (nb - c0 - 32));
           }
         }
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full(s), j & 1, status));
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full(s, j & 1), (j >> 1) & 1, status));
         fence_after();
-        const bool ld0 = ok && (comp || t0), ld1 = ok && (comp || t1);   // uniform per warp
-        uint32_t sa[64], sb[64];                         // columns 0..63 / 64..127 of S_j
-        if (ld0) {
-          tmem_ld32p(sc, sa);
-          tmem_ld32p(sc + 32u, sa + 32);
+        take = take && ok;                               // uniform per warp
+        uint32_t sv[64];
+        if (take) {
+          tmem_ld32p(sc, sv);
+          tmem_ld32p(sc + 32u, sv + 32);
+          tmem_ld_wait();
         }
-        if (ld1) {
-          tmem_ld32p(sc + 64u, sb);
-          tmem_ld32p(sc + 96u, sb + 32);
-        }
-        if (ld0 || ld1) tmem_ld_wait();
         float mt = -INFINITY;
-        const float* brow = beta + (size_t)bh * nb_pad + c0;   // summary tiles only
-        if (!comp) {
-          float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-          if (ld0) {
+        if (take) {
+          if (!comp) {
+            float mc[8];
 #pragma unroll
-            for (int c = 0; c < 64; c += 8)
+            for (int i = 0; i < 8; ++i) mc[i] = fmaxf(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]));
 #pragma unroll
-              for (int i = 0; i < 4; ++i)
-                mc[i] = max3(mc[i], __uint_as_float(sa[c + 2 * i]), __uint_as_float(sa[c + 2 * i + 1]));
-          }
-          if (ld1) {
+            for (int c = 16; c < 64; c += 16)
 #pragma unroll
-            for (int c = 0; c < 64; c += 8)
+              for (int i = 0; i < 8; ++i)
+                mc[i] = max3(mc[i], __uint_as_float(sv[c + 2 * i]), __uint_as_float(sv[c + 2 * i + 1]));
+            mt = fmaxf(fmaxf(max3(mc[0], mc[1], mc[2]), max3(mc[3], mc[4], mc[5])), fmaxf(mc[6], mc[7])) * sl2;
+          } else {
+            // x = s / sqrt(d) + beta (log2 units), -inf where the row selected the block
+            const float* brow = beta + (size_t)bh * nb_pad + c0;
 #pragma unroll
-              for (int i = 0; i < 4; ++i)
-                mc[i] = max3(mc[i], __uint_as_float(sb[c + 2 * i]), __uint_as_float(sb[c + 2 * i + 1]));
-          }
-          mt = fmaxf(max3(mc[0], mc[1], mc[2]), mc[3]) * sl2;
-        } else if (ok) {
-          // x = s / sqrt(d) + beta (log2 units), -inf where the row selected the block
+            for (int c4 = 0; c4 < 16; ++c4) {
+              const float4 bb = __ldg(reinterpret_cast<const float4*>(brow) + c4);
+              const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
-          for (int c4 = 0; c4 < 32; ++c4) {
-            const float4 bb = __ldg(reinterpret_cast<const float4*>(brow) + c4);
-            const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = 4 * c4 + e;
-              uint32_t& sv = c < 64 ? sa[c] : sb[c - 64];
-              const float x = ((ex[c >> 5] >> (c & 31)) & 1u)
-                                  ? -INFINITY
-                                  : fmaf(__uint_as_float(sv), sl2, bv[e] * 1.4426950408889634f);
-              sv = __float_as_uint(x);
-              mt = fmaxf(mt, x);
+              for (int e = 0; e < 4; ++e) {
+                const int c = 4 * c4 + e;
+                const uint32_t w = c < 32 ? ex0 : ex1;
+                const float x = ((w >> (c & 31)) & 1u) ? -INFINITY
+                                                       : fmaf(__uint_as_float(sv[c]), sl2, bv[e] * 1.4426950408889634f);
+                sv[c] = __float_as_uint(x);
+                mt = fmaxf(mt, x);
+              }
             }
           }
         }
@@ -464,55 +437,54 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
           }
         }
         if (ok && __any_sync(0xffffffffu, resc)) {
-          // O is idle here: S_j completing means P_{j-1} V_{j-1} has completed
+          // O in place, once P_{j-1} V_{j-1} has landed (P_j V_j needs P_j: not issued yet)
+          if (j > 0) ok = __all_sync(0xffffffffu, mbar_wait(o_done(s, (j - 1) & 1), (uint32_t)((j - 1) >> 1) & 1u, status));
+          fence_after();
+          if (ok) {
 #pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[32];
-            tmem_ld32p(oc + 32u * cc, o);
-            tmem_ld_wait();
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t o[32];
+              tmem_ld32p(oc + 32u * cc, o);
+              tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
-            tmem_st32p(oc + 32u * cc, o);
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
+              tmem_st32p(oc + 32u * cc, o);
+            }
           }
         }
-        // P_j over the first 64 columns of the S buffer, one 64-key half at a time
+        // P_j (bf16 pairs) over the first 32 columns of the tile's S buffer
+        uint32_t pw[32];
         float rs = 0.f;
-        const bool live = comp ? (m_new != -INFINITY && ok) : true;
-        const uint64_t mul2 = comp ? f2(1.f, 1.f) : sc2, nm2 = f2(-m_new, -m_new);
-        auto make_p = [&](const uint32_t(&sv)[64], int hh, bool take) {
-          uint32_t pw[32];
-          if (take) {
-            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+        if (take && m_new != -INFINITY) {
+          const uint64_t mul2 = comp ? f2(1.f, 1.f) : sc2, nm2 = f2(-m_new, -m_new);
+          uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-            for (int c = 0; c < 64; c += 2) {
-              float u0, u1;
-              unf2(ffma2(f2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), mul2, nm2), u0, u1);
-              const float p0 = ex2(u0), p1 = ex2(u1);
-              acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], f2(p0, p1));
-              pw[c >> 1] = cvt_bf2(p0, p1);
-            }
-            float r0, r1, r2, r3;
-            unf2(fadd2(acc[0], acc[1]), r0, r1);
-            unf2(fadd2(acc[2], acc[3]), r2, r3);
-            rs += (r0 + r2) + (r1 + r3);
-          } else {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) pw[c] = 0u;
+          for (int c = 0; c < 64; c += 2) {
+            float u0, u1;
+            unf2(ffma2(f2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), mul2, nm2), u0, u1);
+            const float p0 = ex2(u0), p1 = ex2(u1);
+            acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], f2(p0, p1));
+            pw[c >> 1] = cvt_bf2(p0, p1);
           }
-          if (ok) tmem_st32p(sc + 32u * hh, pw);
-        };
-        make_p(sa, 0, comp ? live : ld0);     // uniform per warp
-        make_p(sb, 1, comp ? live : ld1);
+          float r0, r1, r2, r3;
+          unf2(fadd2(acc[0], acc[1]), r0, r1);
+          unf2(fadd2(acc[2], acc[3]), r2, r3);
+          rs = (r0 + r2) + (r1 + r3);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) pw[c] = 0u;
+        }
         l = l * corr + rs;
         m_ref = m_new;
         if (ok) {
+          tmem_st32p(sc, pw);
           tmem_st_wait();
           fence_before();
-          mbar_arrive(p_full(s));
+          mbar_arrive(p_full(s, j & 1));
         }
       }
       // ---- epilogue: O / l -> out[perm[row]]
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full(s), Ts & 1, status));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done(s, (Ts - 1) & 1), (uint32_t)((Ts - 1) >> 1) & 1u, status));
       if (!ok) atomicExch(&abort_sh, 1);
       fence_after();
       ok = __all_sync(0xffffffffu, ok && !(*(volatile int*)&abort_sh));
@@ -544,9 +516,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
         if (lse != nullptr && dst_ok) lse[(size_t)bh * N + orig] = (m_ref + log2f(l)) * 0.6931471805599453f;
       }
     }
-  } else {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(OTHER_REGS));
-  if (warp == 8 || warp == 9) {
+  } else if (warp == 8 || warp == 9) {
     // ------------------------------------------------ TMA producer of slot warp - 8
     const int s = warp - 8;
     if (lane == 0 && T[s] > 0) {
@@ -559,127 +529,106 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
       int cur = next_block(um, 0, nwords);
       int ik = 0, iv = 0;
       for (int j = 0; j < T[s]; ++j) {
+        const int st = j % STAGES;
+        const uint32_t ph = (uint32_t)((j / STAGES) - 1) & 1u;   // phase of the previous use of the stage
         const CUtensorMap *mk, *mv;
-        int row0, row1;
+        int row;
         if (j < TE[s]) {
-          const int b0 = cur;
-          int b1 = next_block(um, b0 + 1, nwords);
-          cur = b1 < NONE ? next_block(um, b1 + 1, nwords) : NONE;
-          if (b1 >= NONE) b1 = b0;                     // odd count: the second half repeats, masked
-          row0 = bh * N + b0 * BLK;
-          row1 = bh * N + b1 * BLK;
+          row = bh * N + cur * BLK;
+          cur = next_block(um, cur + 1, nwords);
           mk = &maps.k;
           mv = &maps.v;
         } else {
-          row0 = bh * nb_pad + (j - TE[s]) * KEYS;
-          row1 = row0 + BLK;
+          row = bh * nb_pad + (j - TE[s]) * KEYS;
           mk = &maps.kt;
           mv = &maps.vt;
         }
-        // K_j once S_{j-1} has read the buffer
-        if (j > 0 && !mbar_wait(k_empty(s), (j - 1) & 1, status)) {
+        // K_j once S_{j-STAGES} has read the stage
+        if (j >= STAGES && !mbar_wait(k_empty(s, st), ph, status)) {
           atomicExch(&abort_sh, 1);
           break;
         }
         if (*(volatile int*)&abort_sh) break;
-        mbar_arrive_tx(k_full(s), L::KV_TILE);
+        mbar_arrive_tx(k_full(s, st), L::KV_TILE);
 #pragma unroll
-        for (int a = 0; a < L::KATOMS; ++a) {
-          tma_load_2d(sK(s) + a * L::KV_ATOM, mk, 64 * a, row0, k_full(s));
-          tma_load_2d(sK(s) + a * L::KV_ATOM + BLK * 128, mk, 64 * a, row1, k_full(s));
-        }
+        for (int a = 0; a < L::KATOMS; ++a) tma_load_2d(sK(s, st) + a * L::KV_ATOM, mk, 64 * a, row, k_full(s, st));
         ik = j + 1;
-        // V_j once P_{j-1} V_{j-1} has read the buffer
-        if (j > 0 && !mbar_wait(v_empty(s), (j - 1) & 1, status)) {
+        // V_j once P_{j-STAGES} V_{j-STAGES} has read the stage
+        if (j >= STAGES && !mbar_wait(v_empty(s, st), ph, status)) {
           atomicExch(&abort_sh, 1);
           break;
         }
         if (*(volatile int*)&abort_sh) break;
-        mbar_arrive_tx(v_full(s), L::KV_TILE);
+        mbar_arrive_tx(v_full(s, st), L::KV_TILE);
 #pragma unroll
-        for (int a = 0; a < L::KATOMS; ++a) {
-          tma_load_2d(sV(s) + a * L::KV_ATOM, mv, 64 * a, row0, v_full(s));
-          tma_load_2d(sV(s) + a * L::KV_ATOM + BLK * 128, mv, 64 * a, row1, v_full(s));
-        }
+        for (int a = 0; a < L::KATOMS; ++a) tma_load_2d(sV(s, st) + a * L::KV_ATOM, mv, 64 * a, row, v_full(s, st));
         iv = j + 1;
       }
       issued_sh[s][0] = ik;
       issued_sh[s][1] = iv;
     }
-  } else if (warp == 10) {
-    // ------------------------------------------------ MMA issuer, both slots
-    if (lane == 0) {
+  } else {
+    // ------------------------------------------------ MMA issuer of slot warp - 10
+    const int s = warp - 10;
+    if (lane == 0 && T[s] > 0) {
+      const int Ts = T[s];
       bool ok = true;
-      int jp[SLOTS] = {0, 0};                          // next P V product per slot
-      int kc[SLOTS] = {0, 0}, vc[SLOTS] = {0, 0};      // K / V arrivals observed
-      auto issue_s = [&](int s) {
-        const uint32_t d = tmem + S_COL + 128u * (uint32_t)s;
-        const uint64_t dq = sdesc(sQ(s), 16, 1024), dk = sdesc(sK(s), 16, 1024);
+      int kc = 0, vc = 0;                                // K / V arrivals observed
+      const uint32_t sbase = tmem + SLOT_COLS * (uint32_t)s;
+      const uint32_t od = sbase + O_OFF;
+      const uint64_t dq = sdesc(sQ(s), 16, 1024);
+      // S_j = Q K_j^T into S buffer j & 1
+      auto issue_s = [&](int j) -> bool {
+        const int st = j % STAGES;
+        if (!mbar_wait(k_full(s, st), (uint32_t)(j / STAGES) & 1u, status)) return false;
+        kc = j + 1;
+        fence_after();
+        const uint64_t dk = sdesc(sK(s, st), 16, 1024);
+        const uint32_t d = sbase + 64u * (uint32_t)(j & 1);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t qo = (uint64_t)(((ks >> 2) * L::Q_ATOM + (ks & 3) * 32) >> 4);
           const uint64_t ko = (uint64_t)(((ks >> 2) * L::KV_ATOM + (ks & 3) * 32) >> 4);
           mma_f16(d, dq + qo, dk + ko, L::IDESC_S, ks > 0 ? 1u : 0u);
         }
-        mma_commit(k_empty(s));
+        mma_commit(k_empty(s, st));
+        mma_commit(s_full(s, j & 1));
+        return true;
       };
-      for (int s = 0; s < SLOTS && ok; ++s) {
-        if (T[s] == 0) continue;
-        if (!mbar_wait(q_full(s), 0, status)) { ok = false; break; }
-        q_seen_sh[s] = 1;
-        if (!mbar_wait(k_full(s), 0, status)) { ok = false; break; }
-        kc[s] = 1;
-        fence_after();
-        issue_s(s);
-        mma_commit(s_full(s));
-        mma_used_sh = 1;
+      ok = mbar_wait(q_full(s), 0, status);
+      if (ok) q_seen_sh[s] = 1;
+      if (ok) {
+        mma_used_sh[s] = 1;
+        ok = issue_s(0);
       }
-      unsigned long long t_last = globaltimer();
-      while (ok && (jp[0] < T[0] || jp[1] < T[1])) {
-        bool progressed = false;
-        for (int s = 0; s < SLOTS && ok; ++s) {
-          const int j = jp[s];
-          if (j >= T[s] || !mbar_probe(p_full(s), j & 1)) continue;
-          if (!mbar_wait(v_full(s), j & 1, status)) { ok = false; break; }
-          vc[s] = j + 1;
-          fence_after();
-          const uint64_t dv = sdesc(sV(s), L::KV_ATOM, 1024);
-          const uint32_t pa = tmem + S_COL + 128u * (uint32_t)s;
-          const uint32_t od = tmem + O_COL + 128u * (uint32_t)s;
+      if (ok && Ts > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < Ts; ++j) {
+        const int st = j % STAGES;
+        if (!mbar_wait(p_full(s, j & 1), (uint32_t)(j >> 1) & 1u, status)) { ok = false; break; }
+        if (!mbar_wait(v_full(s, st), (uint32_t)(j / STAGES) & 1u, status)) { ok = false; break; }
+        vc = j + 1;
+        fence_after();
+        const uint64_t dv = sdesc(sV(s, st), L::KV_ATOM, 1024);
+        const uint32_t pa = sbase + 64u * (uint32_t)(j & 1);
 #pragma unroll
-          for (int kk = 0; kk < KEYS / 16; ++kk)
-            mma_ts(od, pa + 8u * kk, dv + (uint64_t)((kk * 2048) >> 4), L::IDESC_O, (kk > 0 || j > 0) ? 1u : 0u);
-          mma_commit(v_empty(s));
-          if (j + 1 < T[s]) {
-            if (!mbar_wait(k_full(s), (j + 1) & 1, status)) { ok = false; break; }
-            kc[s] = j + 2;
-            fence_after();
-            issue_s(s);
-          }
-          // S_{j+1} ready, or (after the last tile) O complete
-          mma_commit(s_full(s));
-          jp[s] = j + 1;
-          progressed = true;
-        }
-        if (progressed) {
-          t_last = globaltimer();
-        } else if (globaltimer() - t_last > WAIT_NS) {
-          set_status(status, STATUS_TIMEOUT);
-          ok = false;
-        }
+        for (int kk = 0; kk < KEYS / 16; ++kk)
+          mma_ts(od, pa + 8u * kk, dv + (uint64_t)((kk * 2048) >> 4), L::IDESC_O, (kk > 0 || j > 0) ? 1u : 0u);
+        mma_commit(v_empty(s, st));
+        mma_commit(o_done(s, j & 1));
+        // S buffer j & 1 is free again once P_j V_j has read P_j (issue order)
+        if (j + 2 < Ts && !issue_s(j + 2)) { ok = false; break; }
       }
       // the last arrivals must land before this CTA's shared memory is released
-      for (int s = 0; s < SLOTS && ok; ++s) {
-        if (T[s] == 0) continue;
-        ok = mbar_wait(v_empty(s), (T[s] - 1) & 1, status) && mbar_wait(k_empty(s), (T[s] - 1) & 1, status);
+      for (int jj = Ts - 2; ok && jj < Ts; ++jj) {
+        if (jj < 0) continue;
+        const uint32_t ph = (uint32_t)(jj / STAGES) & 1u;
+        ok = mbar_wait(k_empty(s, jj % STAGES), ph, status) && mbar_wait(v_empty(s, jj % STAGES), ph, status);
       }
+      if (ok) ok = mbar_wait(o_done(s, (Ts - 1) & 1), (uint32_t)((Ts - 1) >> 1) & 1u, status);
       if (!ok) atomicExch(&abort_sh, 1);
-      for (int s = 0; s < SLOTS; ++s) {
-        consumed_sh[s][0] = kc[s];
-        consumed_sh[s][1] = vc[s];
-      }
+      consumed_sh[s][0] = kc;
+      consumed_sh[s][1] = vc;
     }
-  }
   }
 
   // ---- teardown: drain own copies / MMAs (bounded), free TMEM
@@ -691,12 +640,15 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
       // copies issued but never observed by the MMA thread
       const int s = warp - 8;
       if (T[s] > 0 && !q_seen_sh[s]) mbar_wait(q_full(s), 0, status);
-      for (int j = consumed_sh[s][0]; j < issued_sh[s][0]; ++j) mbar_wait(k_full(s), j & 1, status);
-      for (int j = consumed_sh[s][1]; j < issued_sh[s][1]; ++j) mbar_wait(v_full(s), j & 1, status);
+      for (int j = consumed_sh[s][0]; j < issued_sh[s][0]; ++j)
+        mbar_wait(k_full(s, j % STAGES), (uint32_t)(j / STAGES) & 1u, status);
+      for (int j = consumed_sh[s][1]; j < issued_sh[s][1]; ++j)
+        mbar_wait(v_full(s, j % STAGES), (uint32_t)(j / STAGES) & 1u, status);
     }
-    if (warp == 10 && lane == 0 && mma_used_sh) {
-      mma_commit(drain);
-      mbar_wait(drain, 0, status);
+    if ((warp == 10 || warp == 11) && lane == 0 && mma_used_sh[warp - 10]) {
+      // one more commit: its arrival means every MMA of this thread has completed
+      mma_commit(drain(warp - 10));
+      mbar_wait(drain(warp - 10), 0, status);
     }
     fence_before();
     __syncthreads();
@@ -751,14 +703,6 @@ static cudaError_t run(const Plan& pl, const int32_t* perm, const int32_t* sel, 
       !make_map(&maps.vt, ws_at<void>(ws, pl.off_vt), srows, D, 64))
     return cudaErrorInvalidValue;
   auto kern = attn_tc_kernel<D>;
-  // the register split is only sound with exactly LAUNCH_REGS per thread at launch
-  static int regs_ok = -1;
-  if (regs_ok < 0) {
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
-    regs_ok = fa.numRegs == LAUNCH_REGS ? 1 : 0;
-  }
-  if (!regs_ok) return cudaErrorInvalidDeviceFunction;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
   if (e != cudaSuccess) return e;
   const int npairs = (pl.nb + 1) / 2;

@@ -34,6 +34,8 @@ struct Plan {
   size_t off_Qp = 0, off_Kp = 0, off_Vp = 0;
   size_t off_qm = 0, off_km = 0;
   size_t off_kt = 0, off_vt = 0, off_beta = 0;
+  size_t off_scores = 0;           // block-score matrices of score_heads heads (float64 [nb][nb] each)
+  int score_heads = 1;
   size_t total = 0;
   // extra device room used by spark_forward_host
   size_t off_hq = 0, off_hk = 0, off_hv = 0, off_hout = 0, off_hlse = 0;

@@ -8,11 +8,11 @@
 //   x_j = qbar . k_j / sqrt(d), w = softmax(x), k~ = sum w k, v~ = sum w v,
 //   beta = ln sum e^x - qbar . k~ / sqrt(d) (k~ as stored in bf16), or the
 //   mean-pooling ablation (mean k, mean v, beta = ln 64).
-// select: one CTA per R query blocks of a head. Block scores
-//   s_ab = Qbar_a . Kbar_b / sqrt(d) in float64 ("Spark-H3" news post: the
-//   exact branch computes the top-ranked key/value blocks), then per row a
-//   warp-level radix select of the Ksel largest, ties to the lower b, written
-//   in ascending b order.
+// score + topk: block scores s_ab = Qbar_a . Kbar_b / sqrt(d) in float64
+//   ("Spark-H3" news post: the exact branch computes the top-ranked
+//   key/value blocks) for a chunk of heads at a time, then per row a
+//   warp-level radix select of the Ksel largest, ties to the lower b,
+//   written in ascending b order.
 #include <math.h>
 
 #include "common.cuh"
@@ -135,104 +135,166 @@ blockstats_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k
 }
 
 // ------------------------------------------------------------------ selection
+// score_kernel: the block-score matrix of one chunk of heads,
+//   sc[h][a][b] = (Qbar_a . Kbar_b) / sqrt(d) in float64, as a register-tiled
+//   GEMM: a CTA computes a 128 x 128 tile, each thread an 8 x 8 sub-tile
+//   (rows and columns in pairs 32 apart),
+//   with the d dimension staged through shared memory 8 at a time.
+constexpr int SC_TILE = 128, SC_KSTEP = 8;
+
 template <int D>
 __global__ void __launch_bounds__(256)
-select_kernel(const double* __restrict__ qm, const double* __restrict__ km, int nb, int ksel,
-              int R, int32_t* __restrict__ sel) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  constexpr int KC = 64;          // key blocks staged per chunk
-  constexpr int KS = D + 1;       // padded row stride (doubles)
-  double* sc = reinterpret_cast<double*>(smem_raw);            // [R][nb]
-  double* qs = sc + (size_t)R * nb;                             // [R][D]
-  double* kc = qs + (size_t)R * D;                              // [KC][KS]
-  __shared__ int hist[8][256];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.y, a0 = blockIdx.x * R;
-  const int rows = min(R, nb - a0);
-  const double scale = 1.0 / sqrt((double)D);
-
-  for (int e = tid; e < rows * D; e += blockDim.x) qs[e] = qm[((size_t)bh * nb + a0) * D + e];
-  for (int c0 = 0; c0 < nb; c0 += KC) {
-    const int nk = min(KC, nb - c0);
-    __syncthreads();
-    for (int e = tid; e < nk * D; e += blockDim.x)
-      kc[(e / D) * KS + e % D] = km[((size_t)bh * nb + c0) * D + e];
-    __syncthreads();
-    for (int e = tid; e < rows * KC; e += blockDim.x) {
-      const int a = e / KC, bl = e % KC;
-      if (bl < nk) {
-        double s = 0.0;
-#pragma unroll 8
-        for (int j = 0; j < D; ++j) s = fma(qs[a * D + j], kc[bl * KS + j], s);
-        sc[(size_t)a * nb + c0 + bl] = s * scale;
+score_kernel(const double* __restrict__ qm, const double* __restrict__ km, int nb, int h0,
+             double* __restrict__ sc) {
+  __shared__ __align__(16) double qs[2][SC_KSTEP][SC_TILE];   // [k][a]
+  __shared__ __align__(16) double ks[2][SC_KSTEP][SC_TILE];   // [k][b]
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int b0 = blockIdx.x * SC_TILE, a0 = blockIdx.y * SC_TILE, h = blockIdx.z;
+  const size_t bh = (size_t)(h0 + h);
+  const double* Q = qm + bh * nb * D;
+  const double* K = km + bh * nb * D;
+  // loader: thread -> (row r = tid / 2, 4 consecutive k of the 8) for Q and K
+  const int lr = tid >> 1, lk = (tid & 1) * 4;
+  auto load = [&](int buf, int kc) {
+    const int ra = a0 + lr, rb = b0 + lr;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      qs[buf][lk + e][lr] = ra < nb ? Q[(size_t)ra * D + kc + lk + e] : 0.0;
+      ks[buf][lk + e][lr] = rb < nb ? K[(size_t)rb * D + kc + lk + e] : 0.0;
+    }
+  };
+  double acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+  load(0, 0);
+  __syncthreads();
+  for (int kc = 0; kc < D; kc += SC_KSTEP) {
+    const int buf = (kc / SC_KSTEP) & 1;
+    if (kc + SC_KSTEP < D) load(buf ^ 1, kc + SC_KSTEP);
+#pragma unroll
+    for (int kk = 0; kk < SC_KSTEP; ++kk) {
+      // rows ty*2 + 32*ii + {0,1}, columns tx*2 + 32*jj + {0,1}: for each ii / jj
+      // the 16 lanes of a half-warp read consecutive double2 (no bank conflicts)
+      double qa[8], kb[8];
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii) {
+        const double2 t = *reinterpret_cast<const double2*>(&qs[buf][kk][ty * 2 + 32 * ii]);
+        qa[2 * ii] = t.x;
+        qa[2 * ii + 1] = t.y;
+        const double2 u = *reinterpret_cast<const double2*>(&ks[buf][kk][tx * 2 + 32 * ii]);
+        kb[2 * ii] = u.x;
+        kb[2 * ii + 1] = u.y;
       }
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fma(qa[i], kb[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  const double scale = 1.0 / sqrt((double)D);
+  double* out = sc + (size_t)h * nb * nb;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int a = a0 + ty * 2 + 32 * (i >> 1) + (i & 1);
+    if (a >= nb) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int b = b0 + tx * 2 + 32 * (j >> 1) + (j & 1);
+      if (b < nb) out[(size_t)a * nb + b] = acc[i][j] * scale;
     }
   }
-  __syncthreads();
+}
 
-  // per row: the ksel largest scores, ties to the lower block index
-  int* h = hist[warp];
-  for (int a = warp; a < rows; a += 8) {
-    const double* srow = sc + (size_t)a * nb;
-    auto key = [&](int bb) -> uint64_t { return ordered_key(-srow[bb]); };
-    uint64_t prefix = 0, mask = 0;
-    int rank = ksel;
-    for (int shift = 56; shift >= 0; shift -= 8) {
-      for (int i = lane; i < 256; i += 32) h[i] = 0;
-      __syncwarp();
-      for (int bb = lane; bb < nb; bb += 32) {
-        const uint64_t kk = key(bb);
-        if ((kk & mask) == prefix) atomicAdd(&h[(kk >> shift) & 255], 1);
-      }
-      __syncwarp();
-      int loc[8], s = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) { loc[j] = h[lane * 8 + j]; s += loc[j]; }
-      int incl = s;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-      }
-      const int excl = incl - s;
-      int bucket = 0, newrank = 0;
-      const bool mine = (excl < rank && rank <= incl);
-      if (mine) {
-        int c = excl;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (c < rank && rank <= c + loc[j]) { bucket = lane * 8 + j; newrank = rank - c; }
-          c += loc[j];
-        }
-      }
-      const unsigned owner = __ballot_sync(0xffffffffu, mine);
-      const int src = __ffs(owner) - 1;
-      bucket = __shfl_sync(0xffffffffu, bucket, src);
-      newrank = __shfl_sync(0xffffffffu, newrank, src);
-      prefix |= ((uint64_t)bucket) << shift;
-      mask |= ((uint64_t)255) << shift;
-      rank = newrank;
-      __syncwarp();
+// topk_kernel: one warp per query block a of the chunk: the ksel largest
+//   scores of row a, ties to the lower block index, written in ascending
+//   block order. Radix select over the ordered keys of -score, 8 bits per
+//   pass from the top, stopping as soon as the target key is isolated.
+__global__ void __launch_bounds__(256)
+topk_kernel(const double* __restrict__ sc, int nb, int ksel, int h0, int heads, int32_t* __restrict__ sel) {
+  __shared__ int hist[8][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long row = (long)blockIdx.x * 8 + warp;     // (head in chunk, query block)
+  if (row >= (long)heads * nb) return;
+  const int h = (int)(row / nb), a = (int)(row % nb);
+  const double* srow = sc + ((size_t)h * nb + a) * nb;
+  int* hs = hist[warp];
+  auto key = [&](int bb) -> uint64_t { return ordered_key(-srow[bb]); };
+  uint64_t prefix = 0, mask = 0;
+  int rank = ksel;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int i = lane; i < 256; i += 32) hs[i] = 0;
+    __syncwarp();
+    for (int bb = lane; bb < nb; bb += 32) {
+      const uint64_t kk = key(bb);
+      if ((kk & mask) == prefix) atomicAdd(&hs[(kk >> shift) & 255], 1);
     }
-    const uint64_t kstar = prefix;
-    // members with key < kstar, plus the first `rank` members with key == kstar
-    int out = 0, ties = 0;
-    int32_t* dst = sel + ((size_t)bh * nb + a0 + a) * ksel;
-    for (int c0 = 0; c0 < nb; c0 += 32) {
-      const int bb = c0 + lane;
-      uint64_t kk = ~0ull;
-      if (bb < nb) kk = key(bb);
-      const bool less = bb < nb && kk < kstar;
-      const bool eq = bb < nb && kk == kstar;
-      const unsigned em = __ballot_sync(0xffffffffu, eq);
-      const int eq_before = ties + __popc(em & ((1u << lane) - 1u));
-      const bool take = less || (eq && eq_before < rank);
-      const unsigned tm = __ballot_sync(0xffffffffu, take);
-      const int at = out + __popc(tm & ((1u << lane) - 1u));
-      if (take && at < ksel) dst[at] = bb;
-      out += __popc(tm);
-      ties += __popc(em);
+    __syncwarp();
+    int loc[8], s = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) { loc[j] = hs[lane * 8 + j]; s += loc[j]; }
+    int incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
     }
+    const int excl = incl - s;
+    int bucket = 0, newrank = 0, bcount = 0;
+    const bool mine = (excl < rank && rank <= incl);
+    if (mine) {
+      int c = excl;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (c < rank && rank <= c + loc[j]) { bucket = lane * 8 + j; newrank = rank - c; bcount = loc[j]; }
+        c += loc[j];
+      }
+    }
+    const unsigned owner = __ballot_sync(0xffffffffu, mine);
+    const int src = __ffs(owner) - 1;
+    bucket = __shfl_sync(0xffffffffu, bucket, src);
+    newrank = __shfl_sync(0xffffffffu, newrank, src);
+    bcount = __shfl_sync(0xffffffffu, bcount, src);
+    prefix |= ((uint64_t)bucket) << shift;
+    mask |= ((uint64_t)255) << shift;
+    rank = newrank;
+    __syncwarp();
+    if (bcount == 1) break;    // a single key has this prefix: it is the target
+  }
+  // the target key: the unique key with this prefix, or (all 64 bits fixed) the prefix itself
+  uint64_t kstar = prefix;
+  if (mask != ~0ull) {
+    uint64_t mine = ~0ull;
+    for (int bb = lane; bb < nb; bb += 32) {
+      const uint64_t kk = key(bb);
+      if ((kk & mask) == prefix) mine = kk;
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      const uint64_t other = __shfl_xor_sync(0xffffffffu, mine, o);
+      mine = other < mine ? other : mine;
+    }
+    kstar = mine;
+    rank = 1;
+  }
+  // members with key < kstar, plus the first `rank` members with key == kstar
+  int out = 0, ties = 0;
+  int32_t* dst = sel + ((size_t)(h0 + h) * nb + a) * ksel;
+  for (int c0 = 0; c0 < nb; c0 += 32) {
+    const int bb = c0 + lane;
+    uint64_t kk = ~0ull;
+    if (bb < nb) kk = key(bb);
+    const bool less = bb < nb && kk < kstar;
+    const bool eq = bb < nb && kk == kstar;
+    const unsigned em = __ballot_sync(0xffffffffu, eq);
+    const int eq_before = ties + __popc(em & ((1u << lane) - 1u));
+    const bool take = less || (eq && eq_before < rank);
+    const unsigned tm = __ballot_sync(0xffffffffu, take);
+    const int at = out + __popc(tm & ((1u << lane) - 1u));
+    if (take && at < ksel) dst[at] = bb;
+    out += __popc(tm);
+    ties += __popc(em);
   }
 }
 
@@ -251,13 +313,14 @@ static cudaError_t run_select(const Plan& pl, const uint16_t* q, const uint16_t*
   blockstats_kernel<D><<<dim3(pl.nb_pad, pl.BH), 256, 0, s>>>(q, k, v, perm, qmean, pl.N, pl.nb,
                                                               pl.nb_pad, summary, Qp, Kp, Vp, qm, km,
                                                               kt, vt, beta, status);
-  const size_t fixed = sizeof(double) * (64 * (D + 1));
-  int R = (int)std::min<size_t>(8, (190000 - fixed) / (sizeof(double) * ((size_t)pl.nb + D)));
-  if (R < 1) R = 1;
-  const size_t smem = sizeof(double) * ((size_t)R * pl.nb + (size_t)R * D) + fixed;
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  select_kernel<D><<<dim3((pl.nb + R - 1) / R, pl.BH), 256, smem, s>>>(qm, km, pl.nb, pl.ksel, R, sel);
+  double* sc = ws_at<double>(ws, pl.off_scores);
+  const int tiles = (pl.nb + SC_TILE - 1) / SC_TILE;
+  for (int h0 = 0; h0 < pl.BH; h0 += pl.score_heads) {
+    const int heads = std::min(pl.score_heads, pl.BH - h0);
+    score_kernel<D><<<dim3(tiles, tiles, heads), 256, 0, s>>>(qm, km, pl.nb, h0, sc);
+    const long rows = (long)heads * pl.nb;
+    topk_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(sc, pl.nb, pl.ksel, h0, heads, sel);
+  }
   return cudaGetLastError();
 }
 

@@ -123,6 +123,13 @@ bool make_plan(const spark_params* p, Plan* pl) {
   P.off_kt = take(BH * nbp * d * 2);
   P.off_vt = take(BH * nbp * d * 2);
   P.off_beta = take(BH * nbp * 4);
+  {
+    // float64 block-score matrices, a chunk of heads at a time (at most
+    // 1 GiB, at least one head)
+    const size_t per_head = nb * nb * 8;
+    P.score_heads = (int)std::min<size_t>(BH, std::max<size_t>(1, ((size_t)1 << 30) / per_head));
+    P.off_scores = take((size_t)P.score_heads * per_head);
+  }
   P.total = o;
   P.off_hq = take(BH * N * d * 2);
   P.off_hk = take(BH * N * d * 2);
@@ -164,11 +171,13 @@ size_t spark_workspace_size(const spark_params* p) {
 int32_t spark_forward_launches(const spark_params* p) {
   Plan pl;
   if (!make_plan(p, &pl)) return -1;
-  // moments 2; reblock: whiten, normalise, tree, init, split levels, subtree, leaves; select 2; attention 1
+  // moments 2; reblock: whiten, normalise, tree, init, split levels, subtree, leaves;
+  // select: block statistics, then scores + top-K per chunk of heads; attention 1
   int split_launches = 0;
   for (int lv = 0; lv < pl.sub_level; ++lv) split_launches += pl.level_chunks[lv] > 0 ? 4 : 1;
   const int reblock = 4 + split_launches + (pl.sub_level < pl.nlevels ? 1 : 0) + 1;
-  return 2 + reblock + 2 + 1;
+  const int select = 1 + 2 * ((pl.BH + pl.score_heads - 1) / pl.score_heads);
+  return 2 + reblock + select + 1;
 }
 
 size_t spark_host_workspace_size(const spark_params* p) {

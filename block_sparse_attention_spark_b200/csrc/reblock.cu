@@ -29,6 +29,7 @@ namespace spark {
 
 constexpr double REG_EPS = 1e-6;   // relative diagonal jitter before the Cholesky factor
 constexpr int POWER_ITERS = 16;
+constexpr int NORM_EVERY = 4;      // power-iteration steps between rescalings of v
 
 // ------------------------------------------------------------------ whitening factor
 template <int D>
@@ -251,7 +252,10 @@ __device__ uint64_t radix_select_u64(int n, int rank, int nbits, GetKey getkey, 
 // rg*RPT.. and columns cg*CPT.. of S in registers and its own copy of v on
 // those columns; z goes through a padded, double-buffered shared array (one
 // slot of padding per column group: conflict-free reads) and |z|^2 through
-// per-warp partials, so a step needs one barrier. Writes v to vs.
+// per-warp partials, so a step needs one barrier. v is rescaled to unit
+// length every NORM_EVERY steps and after the last one (the direction after
+// POWER_ITERS steps is the same as with a rescale at every step). Writes v
+// to vs.
 template <int D>
 __device__ void power_iterate(double* acc64, double* vs) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -270,8 +274,12 @@ __device__ void power_iterate(double* acc64, double* vs) {
   auto zpad = [](int c) { return c + c / CPT; };
   bool zero_dir = false;
   double* nparts = zb + 2 * ZP;               // [2][8] per-warp partial |z|^2
+  // v <- S v, scaled to unit length every NORM_EVERY steps and at the end:
+  // scaling does not change the direction, and with |S| <= 1 (a covariance
+  // of unit vectors) NORM_EVERY unscaled steps stay far from underflow
   for (int iter = 0; iter < POWER_ITERS; ++iter) {
     double* z = zb + (iter & 1) * ZP;
+    const bool norm_step = (iter % NORM_EVERY) == NORM_EVERY - 1 || iter == POWER_ITERS - 1;
     double sq = 0.0;
     double zr[RPT];
 #pragma unroll
@@ -289,17 +297,22 @@ __device__ void power_iterate(double* acc64, double* vs) {
       if (cg == 0) z[zpad(rg * RPT + i)] = zr[i];
       sq = fma(zr[i], zr[i], sq);
     }
-    // lanes 0, 8, 16, 24 of each warp hold the warp's four row groups
-    sq += __shfl_xor_sync(0xffffffffu, sq, 8);
-    sq += __shfl_xor_sync(0xffffffffu, sq, 16);
-    if (lane == 0) nparts[(iter & 1) * 8 + warp] = sq;
+    if (norm_step) {
+      // lanes 0, 8, 16, 24 of each warp hold the warp's four row groups
+      sq += __shfl_xor_sync(0xffffffffu, sq, 8);
+      sq += __shfl_xor_sync(0xffffffffu, sq, 16);
+      if (lane == 0) nparts[(iter & 1) * 8 + warp] = sq;
+    }
     __syncthreads();
-    double nn = 0.0;
+    double inv = 1.0;
+    if (norm_step) {
+      double pw[8];
 #pragma unroll
-    for (int w = 0; w < 8; ++w) nn += nparts[(iter & 1) * 8 + w];
-    const double nrm = sqrt(nn);
-    if (nrm == 0.0) { zero_dir = true; break; }   // uniform: every thread saw the same partials
-    const double inv = 1.0 / nrm;
+      for (int w = 0; w < 8; ++w) pw[w] = nparts[(iter & 1) * 8 + w];
+      const double nn = ((pw[0] + pw[1]) + (pw[2] + pw[3])) + ((pw[4] + pw[5]) + (pw[6] + pw[7]));
+      if (nn == 0.0) { zero_dir = true; break; }   // uniform: every thread saw the same partials
+      inv = rsqrt(nn);
+    }
 #pragma unroll
     for (int j = 0; j < CPT; ++j) vloc[j] = z[zpad(cg * CPT + j)] * inv;
   }
@@ -879,7 +892,8 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
   for (int j = 0; j < G::NT * 2; ++j) vl[j] = 1.0 / sqrt((double)D);
   bool zero_dir = false;
   for (int iter = 0; iter < POWER_ITERS; ++iter) {
-    double* z = zp + (iter & 1) * 2 * D;        // [wn][row]
+    double* z = zp + (iter & 1) * 2 * D;        // [wn][row]: the two column halves' partial sums
+    const bool norm_step = (iter % NORM_EVERY) == NORM_EVERY - 1 || iter == POWER_ITERS - 1;
     double zr[G::MT][2];
 #pragma unroll
     for (int mt = 0; mt < G::MT; ++mt) { zr[mt][0] = 0.0; zr[mt][1] = 0.0; }
@@ -904,27 +918,20 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
         for (int h = 0; h < 2; ++h) z[wn * D + m0 + mt * 16 + (lane >> 2) + 8 * h] = zr[mt][h];
     }
     __syncthreads();
-    // |z|^2 from the warps of column half 0 (each row once)
-    double sq = 0.0;
-    if (wn == 0 && (lane & 3) == 0) {
+    double inv = 1.0;
+    if (norm_step) {
+      // every warp forms |z|^2 itself, in the same order: no second barrier
+      double sq = 0.0;
 #pragma unroll
-      for (int mt = 0; mt < G::MT; ++mt)
+      for (int k = 0; k < D / 32; ++k) {
+        const double zz = z[lane + 32 * k] + z[D + lane + 32 * k];
+        sq = fma(zz, zz, sq);
+      }
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int row = m0 + mt * 16 + (lane >> 2) + 8 * h;
-          const double zz = z[row] + z[D + row];
-          sq = fma(zz, zz, sq);
-        }
+      for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      if (sq == 0.0) { zero_dir = true; break; }
+      inv = rsqrt(sq);
     }
-    sq += __shfl_xor_sync(0xffffffffu, sq, 4);
-    sq += __shfl_xor_sync(0xffffffffu, sq, 8);
-    sq += __shfl_xor_sync(0xffffffffu, sq, 16);
-    if (wn == 0 && lane == 0) npart[(iter & 1) * 4 + wm] = sq;
-    __syncthreads();
-    const double nrm = sqrt((npart[(iter & 1) * 4 + 0] + npart[(iter & 1) * 4 + 1]) +
-                            (npart[(iter & 1) * 4 + 2] + npart[(iter & 1) * 4 + 3]));
-    if (nrm == 0.0) { zero_dir = true; break; }
-    const double inv = 1.0 / nrm;
 #pragma unroll
     for (int nt = 0; nt < G::NT; ++nt)
 #pragma unroll

@@ -76,11 +76,11 @@ bool make_plan(const spark_params* p, Plan* pl) {
     P.sub_level = P.nlevels;
     for (int lv = 0; lv < P.nlevels; ++lv)
       if (P.level_maxg[lv] <= 9) { P.sub_level = lv; break; }
-    // few large groups (fewer than two waves of CTAs) are spread over chunks of 32 tiles
+    // groups of two or more 32-tile chunks are spread over one CTA per chunk
     P.level_chunks.assign(P.nlevels, 0);
     for (int lv = 0; lv < P.sub_level; ++lv) {
       const int ch = (P.level_maxg[lv] + 31) / 32;
-      if ((long)P.level_count[lv] * P.BH < 296 && ch >= 2) P.level_chunks[lv] = ch;
+      if (ch >= 2) P.level_chunks[lv] = ch;
     }
   }
   {

@@ -200,7 +200,7 @@ __device__ __forceinline__ int block_excl_scan_256(int flag, int* warp_tot, int&
 // uint64 (digits from bit 56 down). All 256 threads must call it.
 template <class GetKey>
 __device__ uint64_t radix_select_u64(int n, int rank, int nbits, GetKey getkey, int* hist,
-                                     int* sh_sel) {
+                                     int* sh_sel, unsigned long long* sh_key) {
   uint64_t prefix = 0, mask = 0;
   const int tid = threadIdx.x;
   for (int shift = nbits - 8; shift >= 0; shift -= 8) {
@@ -232,7 +232,7 @@ __device__ uint64_t radix_select_u64(int n, int rank, int nbits, GetKey getkey, 
         int c = excl;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          if (c < rank && rank <= c + loc[j]) { sh_sel[0] = tid * 8 + j; sh_sel[1] = rank - c; }
+          if (c < rank && rank <= c + loc[j]) { sh_sel[0] = tid * 8 + j; sh_sel[1] = rank - c; sh_sel[2] = loc[j]; }
           c += loc[j];
         }
       }
@@ -241,7 +241,19 @@ __device__ uint64_t radix_select_u64(int n, int rank, int nbits, GetKey getkey, 
     prefix |= ((uint64_t)sh_sel[0]) << shift;
     mask |= ((uint64_t)255) << shift;
     rank = sh_sel[1];
+    const int in_bucket = sh_sel[2];
     __syncthreads();
+    if (in_bucket == 1 && shift > 0) {
+      // a single key carries this prefix: it is the answer
+      for (int i = tid; i < n; i += blockDim.x) {
+        const uint64_t k = getkey(i);
+        if ((k & mask) == prefix) *sh_key = k;
+      }
+      __syncthreads();
+      const uint64_t r = *sh_key;
+      __syncthreads();
+      return r;
+    }
   }
   return prefix;
 }
@@ -330,16 +342,14 @@ __device__ void power_iterate(double* acc64, double* vs) {
 
 // The cut of one group: the key of rank nL among the (sgn * p, index) keys
 // (block radix select on the ordered float64 projection, then index ties),
-// then a stable partition written over the group's index slice: the nL
-// smallest keys left, the rest right. pv/pi: the group's projections and
-// token indices (global scratch), ids: the group's index slice (output).
-__device__ void cut_and_partition(int n, int nL, double sgn, const double* pv, const int32_t* pi,
-                                  int32_t* ids, int* hist, int* sh_sel, int* warp_tot, int* red_i,
-                                  int* status) {
+// then a stable partition: the nL smallest keys to positions 0..nL-1, the
+// rest after them. pkey(i) / pid(i): ordered key and token index of member
+// i; put(dst, i) moves member i to position dst.
+template <class KeyF, class IdF, class PutF>
+__device__ void cut_partition(int n, int nL, KeyF pkey, IdF pid, PutF put, int* hist, int* sh_sel,
+                              unsigned long long* sh_key, int* warp_tot, int* red_i, int* status) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // ---- phase 5: the cut - key of rank nL among (sgn * p) keys, then index ties
-  auto pkey = [&](int i) -> uint64_t { return ordered_key(sgn * pv[i]); };
-  const uint64_t kstar = radix_select_u64(n, nL, 64, pkey, hist, sh_sel);
+  const uint64_t kstar = radix_select_u64(n, nL, 64, pkey, hist, sh_sel, sh_key);
   int c_less = 0, c_eq = 0;
   for (int i = tid; i < n; i += blockDim.x) {
     const uint64_t k = pkey(i);
@@ -365,33 +375,39 @@ __device__ void cut_and_partition(int n, int nL, double sgn, const double* pv, c
   int32_t istar = 0x7fffffff;
   if (need < ties) {   // several tokens share the cut value: lowest indices go left
     auto ikey = [&](int i) -> uint64_t {
-      return (pkey(i) == kstar) ? (uint64_t)(uint32_t)pi[i] : 0xffffffffull;
+      return (pkey(i) == kstar) ? (uint64_t)(uint32_t)pid(i) : 0xffffffffull;
     };
-    istar = (int32_t)radix_select_u64(n, need, 32, ikey, hist, sh_sel);
+    istar = (int32_t)radix_select_u64(n, need, 32, ikey, hist, sh_sel, sh_key);
   }
-
-  // ---- phase 6: stable partition, written in place over the group's indices
   int left_done = 0, right_done = 0;
   for (int base = 0; base < n; base += blockDim.x) {
     const int i = base + tid;
     int goleft = 0;
-    int32_t id = 0;
     if (i < n) {
       const uint64_t k = pkey(i);
-      id = pi[i];
-      goleft = (k < kstar) || (k == kstar && id <= istar);
+      goleft = (k < kstar) || (k == kstar && pid(i) <= istar);
     }
     int tot;
     const int lpos = block_excl_scan_256(goleft, warp_tot, tot);
     if (i < n) {
       const int dst = goleft ? left_done + lpos : nL + right_done + (tid - lpos);
       const bool in_side = goleft ? (dst < nL) : (dst < n);
-      if (in_side) ids[dst] = id;
+      if (in_side) put(dst, i);
       else set_status(status, STATUS_BAD_INPUT);
     }
     left_done += tot;
     right_done += min((int)blockDim.x, n - base) - tot;
   }
+}
+
+// The cut over a group's projections in global scratch (pv, pi), written
+// over the group's index slice ids.
+__device__ void cut_and_partition(int n, int nL, double sgn, const double* pv, const int32_t* pi,
+                                  int32_t* ids, int* hist, int* sh_sel, unsigned long long* sh_key,
+                                  int* warp_tot, int* red_i, int* status) {
+  cut_partition(
+      n, nL, [&](int i) -> uint64_t { return ordered_key(sgn * pv[i]); }, [&](int i) { return pi[i]; },
+      [&](int dst, int i) { ids[dst] = pi[i]; }, hist, sh_sel, sh_key, warp_tot, red_i, status);
 }
 
 // ------------------------------------------------------------------ one split level
@@ -419,7 +435,8 @@ split_level_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restr
   __shared__ double red_d[8];
   __shared__ int red_i[8];
   __shared__ int hist[256];
-  __shared__ int sh_sel[2];
+  __shared__ int sh_sel[3];
+  __shared__ unsigned long long sh_key;
   __shared__ int warp_tot[8];
   __shared__ double sh_scalar;
 
@@ -566,7 +583,7 @@ split_level_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restr
   __syncthreads();
   const double sgn = sh_scalar;
 
-  cut_and_partition(n, nL, sgn, pv, pi, ids, hist, sh_sel, warp_tot, red_i, status);
+  cut_and_partition(n, nL, sgn, pv, pi, ids, hist, sh_sel, &sh_key, warp_tot, red_i, status);
 }
 
 // ------------------------------------------------------------------ large groups over many CTAs
@@ -661,10 +678,24 @@ big_solve_kernel(const int2* __restrict__ nodes, int nnodes, int chunks, const d
     mus[tid] = t * invn;
   }
   __syncthreads();
-  for (int e = tid; e < D * D; e += blockDim.x) {
-    double t = 0.0;
-    for (int c = 0; c < used; ++c) t += src[(size_t)c * (D * D + D) + e];
-    Smat[e] = t * invn - mus[e / D] * mus[e % D];
+  // 8 elements per thread at a time, so that their loads are in flight together
+  for (int e0 = tid; e0 < D * D; e0 += 8 * blockDim.x) {
+    double t[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) t[u] = 0.0;
+    for (int c = 0; c < used; ++c) {
+      const double* pc = src + (size_t)c * (D * D + D);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int e = e0 + u * blockDim.x;
+        if (e < D * D) t[u] += pc[e];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = e0 + u * blockDim.x;
+      if (e < D * D) Smat[e] = t[u] * invn - mus[e / D] * mus[e % D];
+    }
   }
   __syncthreads();
   power_iterate<D>(Smat, vs);
@@ -769,7 +800,8 @@ big_select_kernel(int N, const int2* __restrict__ nodes, int nnodes, int chunks,
                   int32_t* __restrict__ idx, const double* __restrict__ pval, const int32_t* __restrict__ pidx,
                   int* status) {
   __shared__ int hist[256];
-  __shared__ int sh_sel[2];
+  __shared__ int sh_sel[3];
+  __shared__ unsigned long long sh_key;
   __shared__ int warp_tot[8];
   __shared__ int red_i[8];
   __shared__ double sh_sgn;
@@ -789,7 +821,8 @@ big_select_kernel(int N, const int2* __restrict__ nodes, int nnodes, int chunks,
   }
   __syncthreads();
   const size_t gpos = (size_t)bh * N + (size_t)node.x * BLK;
-  cut_and_partition(n, nL, sh_sgn, pval + gpos, pidx + gpos, idx + gpos, hist, sh_sel, warp_tot, red_i, status);
+  cut_and_partition(n, nL, sh_sgn, pval + gpos, pidx + gpos, idx + gpos, hist, sh_sel, &sh_key, warp_tot,
+                    red_i, status);
 }
 
 // ------------------------------------------------------------------ whole small subtrees
@@ -810,22 +843,18 @@ struct SubSmem {
   static constexpr size_t off_rows = 0;
   static constexpr size_t off_pv = off_rows + sizeof(uint16_t) * TMAX * RS;
   static constexpr size_t off_ids = off_pv + sizeof(double) * TMAX;
-  static constexpr int SORTN = 1024;                     // power of two >= TMAX
-  static_assert(SORTN >= TMAX, "sort buffer must hold a whole subtree");
   static constexpr size_t off_loc = off_ids + sizeof(int32_t) * TMAX;
-  static constexpr size_t off_skey = (off_loc + sizeof(uint16_t) * TMAX + 15) & ~(size_t)15;
-  static constexpr size_t off_sid = off_skey + sizeof(uint64_t) * SORTN;
-  static constexpr size_t off_stok = off_sid + sizeof(int32_t) * SORTN;
-  static constexpr size_t off_zp = (off_stok + sizeof(uint16_t) * SORTN + 15) & ~(size_t)15;
+  static constexpr size_t off_stok = off_loc + sizeof(uint16_t) * TMAX;   // partition target
+  static constexpr size_t off_zp = (off_stok + sizeof(uint16_t) * TMAX + 15) & ~(size_t)15;
   static constexpr size_t zp_bytes = sizeof(double) * 2 * 2 * D > sizeof(int32_t) * TMAX ? sizeof(double) * 2 * 2 * D : sizeof(int32_t) * TMAX;
   static constexpr size_t bytes = off_zp + (zp_bytes > sizeof(double) * 256 ? zp_bytes : sizeof(double) * 256);
 };
 
 template <int D>
 __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* ids, uint16_t* loc,
-                              uint64_t* skey, int32_t* sid, uint16_t* stok, double* zp, double* mus,
-                              double* vs, double* npart, double* red_d, int* red_i, double* sh_sgn, int s0,
-                              int nn) {
+                              uint16_t* stok, double* zp, double* mus, double* vs, double* red_d, int* red_i,
+                              double* sh_sgn, int* hist, int* sh_sel, unsigned long long* sh_key,
+                              int* warp_tot, int* status, int s0, int nn) {
   using G = Gram<D>;
   using SM = SubSmem<D>;
   constexpr int RS = SM::RS;
@@ -1004,40 +1033,14 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
   }
   __syncthreads();
   const double sgn = *sh_sgn;
-  // ascending order of (sgn * p, index): bitonic sort of the node's keys
-  int P2 = 64;
-  while (P2 < nn) P2 <<= 1;
-  for (int t = tid; t < P2; t += blockDim.x) {
-    if (t < nn) {
-      skey[t] = ordered_key(sgn * pv[t]);
-      sid[t] = ids[lo[t]];
-      stok[t] = lo[t];
-    } else {
-      skey[t] = ~0ull;
-      sid[t] = 0x7fffffff;
-      stok[t] = 0;
-    }
-  }
+  // the cut: the nL smallest (sgn * p, index) keys become the left child's
+  // slice, the rest the right child's (order inside a child is irrelevant:
+  // it is cut again, and leaves are sorted by index at the end)
+  const int nL = BLK * ((nn / BLK) / 2);
+  cut_partition(
+      nn, nL, [&](int t) -> uint64_t { return ordered_key(sgn * pv[t]); }, [&](int t) { return ids[lo[t]]; },
+      [&](int dst, int t) { stok[dst] = lo[t]; }, hist, sh_sel, sh_key, warp_tot, red_i, status);
   __syncthreads();
-  for (int kk = 2; kk <= P2; kk <<= 1) {
-    for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-      for (int i = tid; i < P2; i += blockDim.x) {
-        const int ixj = i ^ jj;
-        if (ixj > i) {
-          const uint64_t ka = skey[i], kb = skey[ixj];
-          const int32_t ia = sid[i], ib = sid[ixj];
-          const bool a_gt = (ka > kb) || (ka == kb && ia > ib);
-          if (a_gt == ((i & kk) == 0)) {
-            skey[i] = kb; skey[ixj] = ka;
-            sid[i] = ib; sid[ixj] = ia;
-            const uint16_t ta = stok[i];
-            stok[i] = stok[ixj]; stok[ixj] = ta;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
   for (int t = tid; t < nn; t += blockDim.x) loc[s0 + t] = stok[t];
   __syncthreads();
 }
@@ -1052,12 +1055,11 @@ subtree_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restrict_
   double* pv = reinterpret_cast<double*>(smem_raw + SM::off_pv);
   int32_t* ids = reinterpret_cast<int32_t*>(smem_raw + SM::off_ids);
   uint16_t* loc = reinterpret_cast<uint16_t*>(smem_raw + SM::off_loc);
-  uint64_t* skey = reinterpret_cast<uint64_t*>(smem_raw + SM::off_skey);
-  int32_t* sid = reinterpret_cast<int32_t*>(smem_raw + SM::off_sid);
   uint16_t* stok = reinterpret_cast<uint16_t*>(smem_raw + SM::off_stok);
   double* zp = reinterpret_cast<double*>(smem_raw + SM::off_zp);
-  __shared__ double mus[D], vs[D], npart[8], red_d[16];
-  __shared__ int red_i[8];
+  __shared__ double mus[D], vs[D], red_d[16];
+  __shared__ int red_i[8], hist[256], sh_sel[3], warp_tot[8];
+  __shared__ unsigned long long sh_key;
   __shared__ double sh_sgn;
   __shared__ int2 lvl[2][SUB_BLOCKS];
   __shared__ int lvl_n[2];
@@ -1092,8 +1094,8 @@ subtree_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restrict_
     for (int i = 0; i < cnt; ++i) {
       const int2 nd = lvl[cur][i];
       if (nd.y >= 2)
-        subtree_split<D>(rows, pv, ids, loc, skey, sid, stok, zp, mus, vs, npart, red_d, red_i, &sh_sgn,
-                         nd.x * BLK, nd.y * BLK);
+        subtree_split<D>(rows, pv, ids, loc, stok, zp, mus, vs, red_d, red_i, &sh_sgn, hist, sh_sel, &sh_key,
+                         warp_tot, status, nd.x * BLK, nd.y * BLK);
     }
     if (tid == 0) {
       int m = 0;

@@ -12,7 +12,8 @@
 //
 // Kernels, in launch order:
 //   whiten_prep  : one CTA per head - regularise M, float64 Cholesky -> L (f32)
-//   normalize    : one thread per token - u = L^T x (f32), u_hat = bf16(u/|u|)
+//   normalize    : persistent CTAs over 128-token tiles - U = X L on the tensor
+//                  cores (L as three bf16 terms), u_hat = bf16(u/|u|)
 //   tree_build   : node table (first block, g) per level; depends on nb only
 //   init_idx     : identity token order
 //   split_level  : one CTA per (node, head) per level - Gram of the group
@@ -82,72 +83,142 @@ whiten_prep_kernel(const double* __restrict__ M, float* __restrict__ Lout, int* 
 // Output dims [Q*D/4, (Q+1)*D/4) of u = L^T x; L is lower triangular, so
 // only inputs i >= Q*D/4 contribute. The inner loop is fully unrolled so the
 // token's x stays in registers.
-template <int D, int Q>
-__device__ __forceinline__ void normalize_quarter(const uint32_t (&xr)[D / 2], const float* Ls, float* us,
-                                                  int tid, double& nrm2) {
-  for (int j4 = Q * (D / 16); j4 < (Q + 1) * (D / 16); ++j4) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-    for (int i = Q * (D / 4); i < D; ++i) {
-      const float4 l = *reinterpret_cast<const float4*>(Ls + i * D + 4 * j4);
-      const float xi = (i & 1) ? bf_hi(xr[i >> 1]) : bf_lo(xr[i >> 1]);
-      a0 = fmaf(l.x, xi, a0); a1 = fmaf(l.y, xi, a1);
-      a2 = fmaf(l.z, xi, a2); a3 = fmaf(l.w, xi, a3);
-    }
-    us[(4 * j4 + 0) * 256 + tid] = a0; us[(4 * j4 + 1) * 256 + tid] = a1;
-    us[(4 * j4 + 2) * 256 + tid] = a2; us[(4 * j4 + 3) * 256 + tid] = a3;
-    nrm2 += (double)a0 * a0 + (double)a1 * a1 + (double)a2 * a2 + (double)a3 * a3;
-  }
-}
-
 // ------------------------------------------------------------------ normalised whitened tokens
-// u_j = sum_{i >= j} L[i][j] x_i, u_hat = bf16(u / |u|). Thread = token.
+// u_j = sum_{i >= j} L[i][j] x_i, u_hat = bf16(u / |u|), as the tile product
+// U = X L on the tensor cores (mma.sync m16n8k16, float32 accumulation).
+// x is exact in bf16; L (float32) is split into three bf16 terms that sum to
+// it to within 2^-24 relative, so the product is as accurate as a float32
+// evaluation. Blocks of L above the diagonal are zero and skipped. The norm
+// and the final scaling are float64, the rounding to bf16 is correct
+// rounding of the float64 quotient.
+//
+// Persistent CTAs walk a contiguous range of (head, 128-token tile) items;
+// the three L terms of the current head sit transposed in shared memory
+// (row j = column j of L, for conflict-free ldmatrix B fragments), the X
+// tiles are double-buffered with cp.async. Warp w owns tokens 16w..16w+15
+// of a tile and all D outputs, and writes its bf16 rows back through its
+// own rows of the tile buffer for coalesced stores.
 template <int D>
-__global__ void __launch_bounds__(256)
-normalize_kernel(const uint16_t* __restrict__ X, const float* __restrict__ Lall, int N,
+struct NormSmem {
+  static constexpr int TOK = 128;                      // tokens per tile
+  static constexpr int RS = D + 8;                     // padded row (elements)
+  static constexpr size_t l_bytes = sizeof(uint16_t) * 3 * D * RS;
+  static constexpr size_t x_bytes = sizeof(uint16_t) * TOK * RS;
+  static constexpr size_t bytes = l_bytes + 2 * x_bytes;
+};
+
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+normalize_kernel(const uint16_t* __restrict__ X, const float* __restrict__ Lall, int N, int BH,
                  uint16_t* __restrict__ uhat) {
+  using SM = NormSmem<D>;
+  constexpr int TOK = SM::TOK, RS = SM::RS, NT = D / 8;
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  float* Ls = reinterpret_cast<float*>(smem_raw);       // [D][D]
-  float* us = Ls + D * D;                                // [D][256]
-  const int tid = threadIdx.x, bh = blockIdx.y;
-  const float* L = Lall + (size_t)bh * D * D;
-  for (int e = tid * 4; e < D * D; e += blockDim.x * 4)
-    *reinterpret_cast<float4*>(Ls + e) = *reinterpret_cast<const float4*>(L + e);
-  const long tok = (long)blockIdx.x * blockDim.x + tid;
-  uint32_t xr[D / 2];
-  if (tok < N) {
-    const uint4* src = reinterpret_cast<const uint4*>(X + ((size_t)bh * N + tok) * D);
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-      uint4 w = src[c];
-      xr[4 * c + 0] = w.x; xr[4 * c + 1] = w.y; xr[4 * c + 2] = w.z; xr[4 * c + 3] = w.w;
+  uint16_t* Lt = reinterpret_cast<uint16_t*>(smem_raw);                 // [3][D][RS]
+  uint16_t* Xs = reinterpret_cast<uint16_t*>(smem_raw + SM::l_bytes);   // [2][TOK][RS]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tpb = (N + TOK - 1) / TOK;
+  const long items = (long)BH * tpb;
+  const long per = (items + gridDim.x - 1) / gridDim.x;
+  const long it0 = (long)blockIdx.x * per, it1 = min(items, it0 + per);
+  if (it0 >= it1) return;
+
+  auto load_x = [&](long it, int buf) {
+    const int bh = (int)(it / tpb), t0 = (int)(it % tpb) * TOK;
+    uint16_t* dst = Xs + (size_t)buf * TOK * RS;
+    for (int c = tid; c < TOK * (D / 8); c += 256) {
+      const int r = c / (D / 8), ch = c % (D / 8);
+      if (t0 + r < N) cp_async16(dst + r * RS + ch * 8, X + ((size_t)bh * N + t0 + r) * D + ch * 8);
+      else *reinterpret_cast<uint4*>(dst + r * RS + ch * 8) = make_uint4(0u, 0u, 0u, 0u);
     }
-  } else {
-#pragma unroll
-    for (int c = 0; c < D / 2; ++c) xr[c] = 0u;
-  }
-  __syncthreads();
-  double nrm2 = 0.0;
-  normalize_quarter<D, 0>(xr, Ls, us, tid, nrm2);
-  normalize_quarter<D, 1>(xr, Ls, us, tid, nrm2);
-  normalize_quarter<D, 2>(xr, Ls, us, tid, nrm2);
-  normalize_quarter<D, 3>(xr, Ls, us, tid, nrm2);
-  if (tok >= N) return;
-  const double nrm = sqrt(nrm2);
-  const double inv = nrm > 0.0 ? 1.0 / nrm : 0.0;
-  uint4* dst = reinterpret_cast<uint4*>(uhat + ((size_t)bh * N + tok) * D);
-#pragma unroll 4
-  for (int c = 0; c < D / 8; ++c) {
-    uint32_t w[4];
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const int j = 8 * c + 2 * h;
-      const uint16_t lo = __bfloat16_as_ushort(__double2bfloat16((double)us[j * 256 + tid] * inv));
-      const uint16_t hi = __bfloat16_as_ushort(__double2bfloat16((double)us[(j + 1) * 256 + tid] * inv));
-      w[h] = (uint32_t)lo | ((uint32_t)hi << 16);
+  };
+  int cur_bh = -1;
+  load_x(it0, 0);
+  cp_async_commit();
+  for (long it = it0; it < it1; ++it) {
+    const int buf = (int)((it - it0) & 1);
+    const int bh = (int)(it / tpb), t0 = (int)(it % tpb) * TOK;
+    __syncthreads();                                   // every warp is done with the buffer refilled next
+    if (bh != cur_bh) {
+      // three bf16 terms of L, transposed: Lt[term][j][i] = term of L[i][j]
+      const float* L = Lall + (size_t)bh * D * D;
+      for (int e = tid; e < D * D; e += 256) {
+        const int i = e / D, j = e % D;
+        const float l = L[e];
+        const __nv_bfloat16 h1 = __float2bfloat16_rn(l);
+        const float r1 = l - __bfloat162float(h1);
+        const __nv_bfloat16 h2 = __float2bfloat16_rn(r1);
+        const float r2 = r1 - __bfloat162float(h2);
+        const __nv_bfloat16 h3 = __float2bfloat16_rn(r2);
+        Lt[(0 * D + j) * RS + i] = __bfloat16_as_ushort(h1);
+        Lt[(1 * D + j) * RS + i] = __bfloat16_as_ushort(h2);
+        Lt[(2 * D + j) * RS + i] = __bfloat16_as_ushort(h3);
+      }
+      cur_bh = bh;
     }
-    dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    if (it + 1 < it1) load_x(it + 1, buf ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+
+    uint16_t* xs = Xs + (size_t)buf * TOK * RS + (size_t)warp * 16 * RS;   // this warp's 16 rows
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      uint32_t a[4];
+      ldsm_x4(a[0], a[1], a[2], a[3], xs + (lane & 15) * RS + ks * 16 + (lane >> 4) * 8);
+#pragma unroll
+      for (int np = 0; np < NT / 2; ++np) {
+        if (16 * ks + 15 < 16 * np) continue;          // L[i][j] = 0 for i < j: both n-tiles zero
+#pragma unroll
+        for (int term = 0; term < 3; ++term) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(b0, b1, b2, b3,
+                  Lt + (size_t)(term * D + 16 * np + (lane >> 4) * 8 + (lane & 7)) * RS + ks * 16 +
+                      ((lane >> 3) & 1) * 8);
+          mma_bf16(acc[2 * np], a, b0, b1);
+          mma_bf16(acc[2 * np + 1], a, b2, b3);
+        }
+      }
+    }
+    // rows r0 = lane / 4 and r0 + 8 of this warp's 16; columns 8 nt + 2 (lane % 4) + {0, 1}
+    double n0 = 0.0, n1 = 0.0;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      n0 += (double)acc[nt][0] * acc[nt][0] + (double)acc[nt][1] * acc[nt][1];
+      n1 += (double)acc[nt][2] * acc[nt][2] + (double)acc[nt][3] * acc[nt][3];
+    }
+    n0 += __shfl_xor_sync(0xffffffffu, n0, 1);
+    n0 += __shfl_xor_sync(0xffffffffu, n0, 2);
+    n1 += __shfl_xor_sync(0xffffffffu, n1, 1);
+    n1 += __shfl_xor_sync(0xffffffffu, n1, 2);
+    const double i0 = n0 > 0.0 ? 1.0 / sqrt(n0) : 0.0, i1 = n1 > 0.0 ? 1.0 / sqrt(n1) : 0.0;
+    __syncwarp();
+    const int r0 = lane >> 2, c0 = 2 * (lane & 3);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const uint32_t w0 = (uint32_t)__bfloat16_as_ushort(__double2bfloat16((double)acc[nt][0] * i0)) |
+                          ((uint32_t)__bfloat16_as_ushort(__double2bfloat16((double)acc[nt][1] * i0)) << 16);
+      const uint32_t w1 = (uint32_t)__bfloat16_as_ushort(__double2bfloat16((double)acc[nt][2] * i1)) |
+                          ((uint32_t)__bfloat16_as_ushort(__double2bfloat16((double)acc[nt][3] * i1)) << 16);
+      *reinterpret_cast<uint32_t*>(xs + r0 * RS + 8 * nt + c0) = w0;
+      *reinterpret_cast<uint32_t*>(xs + (r0 + 8) * RS + 8 * nt + c0) = w1;
+    }
+    __syncwarp();
+    // this warp's 16 rows, 16-byte chunks
+    for (int c = lane; c < 16 * (D / 8); c += 32) {
+      const int r = c / (D / 8), ch = c % (D / 8);
+      const int tok = t0 + warp * 16 + r;
+      if (tok < N)
+        *reinterpret_cast<uint4*>(uhat + ((size_t)bh * N + tok) * D + ch * 8) =
+            *reinterpret_cast<const uint4*>(xs + r * RS + ch * 8);
+    }
   }
+  cp_async_wait<0>();
 }
 
 // ------------------------------------------------------------------ tree table
@@ -1165,10 +1236,17 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
   if (e != cudaSuccess) return e;
   whiten_prep_kernel<D><<<pl.BH, 256, smem_w, s>>>(M, L, status);
 
-  const size_t smem_n = sizeof(float) * (D * D + D * 256);
+  const size_t smem_n = NormSmem<D>::bytes;
   e = cudaFuncSetAttribute(normalize_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_n);
   if (e != cudaSuccess) return e;
-  normalize_kernel<D><<<dim3((pl.N + 255) / 256, pl.BH), 256, smem_n, s>>>(x, L, pl.N, uhat);
+  {
+    int sms = 148;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long items = (long)pl.BH * ((pl.N + NormSmem<D>::TOK - 1) / NormSmem<D>::TOK);
+    const int grid = (int)std::min<long>(items, sms);
+    normalize_kernel<D><<<grid, 256, smem_n, s>>>(x, L, pl.N, pl.BH, uhat);
+  }
 
   tree_build_kernel<<<1, 1, 0, s>>>(pl.nb, nodes);
   const long total = (long)pl.BH * pl.N;

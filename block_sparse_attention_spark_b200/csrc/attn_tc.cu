@@ -343,7 +343,6 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
     T[s] = (SLOTS * blockIdx.x + s < npairs) ? U + TS : 0;
   }
   const uint32_t tmem = tmem_base_sh;
-  constexpr int NONE = 1 << 30;
 
   if (warp < 8) {
     // ------------------------------------------------ softmax of slot warp / 4, one thread per row

@@ -23,13 +23,16 @@ struct Plan {
   std::vector<int> level_maxg;    // largest group (in blocks) at each level
   int moment_splits = 1;
   int sub_level = 0;              // first level whose nodes are split by the in-shared-memory subtree kernel
-  std::vector<int> level_chunks;  // > 0: the level's groups are spread over this many chunk CTAs each
+  std::vector<int> level_chunks;  // chunk CTAs per group at each level above the subtree level
+  std::vector<int> level_derive;  // 1: right children's Gram sums derived from the parent level's
+  std::vector<int> level_store;   // 1: the level's Gram sums are kept for the next level
   // byte offsets into the workspace
   size_t off_MQ = 0, off_MK = 0, off_qmean = 0;
   size_t off_mpart = 0;
   size_t off_L = 0, off_uhat = 0, off_idx = 0, off_pval = 0, off_pidx = 0;
   size_t off_nodes = 0;
   size_t off_bigpart = 0, off_biginfo = 0, off_bigcand = 0;
+  size_t off_gstore[2] = {0, 0};   // Gram sums of consecutive levels (float64 [D*D + D] per group)
   size_t off_perm = 0, off_sel = 0;
   size_t off_Qp = 0, off_Kp = 0, off_Vp = 0;
   size_t off_qm = 0, off_km = 0;

@@ -16,10 +16,14 @@
 //                  cores (L as three bf16 terms), u_hat = bf16(u/|u|)
 //   tree_build   : node table (first block, g) per level; depends on nb only
 //   init_idx     : identity token order
-//   split_level  : one CTA per (node, head) per level - Gram of the group
-//                  (mma.sync, float64 flush), covariance, float64 power
-//                  iteration in registers, float64 projections, orientation,
-//                  radix select of the cut, stable in-place partition
+//   big_gram / big_solve / big_project / big_select, per level above the
+//                  subtree level - chunked Gram sums of the groups (mma.sync,
+//                  float64 flush; right halves derived from the parent level),
+//                  covariance and float64 power iteration in registers,
+//                  float64 projections, orientation, radix select of the cut,
+//                  stable partition of the group's index slice
+//   subtree      : one CTA per group of at most SUB_BLOCKS blocks - all
+//                  remaining splits of its subtree in shared memory
 //   leaf_sort    : ascending original index inside every 64-token leaf -> perm
 #include <math.h>
 
@@ -491,185 +495,21 @@ struct SplitSmem {
   static constexpr size_t bytes = acc_bytes + tile_bytes;
 };
 
-template <int D>
-__global__ void __launch_bounds__(256, 1)
-split_level_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restrict__ nodes,
-                   int32_t* __restrict__ idx, double* __restrict__ pval, int32_t* __restrict__ pidx,
-                   int* status) {
-  using G = Gram<D>;
-  using SM = SplitSmem<D>;
-  constexpr int STAGES = SM::STAGES;
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  double* acc64 = reinterpret_cast<double*>(smem_raw);
-  uint16_t* tiles = reinterpret_cast<uint16_t*>(smem_raw + SM::acc_bytes);
-  __shared__ double mus[D], vs[D], zs[D];
-  __shared__ double red_d[8];
-  __shared__ int red_i[8];
-  __shared__ int hist[256];
-  __shared__ int sh_sel[3];
-  __shared__ unsigned long long sh_key;
-  __shared__ int warp_tot[8];
-  __shared__ double sh_scalar;
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int2 node = nodes[blockIdx.x];
-  const int bh = blockIdx.y;
-  const int n = node.y * BLK, pos0 = node.x * BLK, nL = BLK * (node.y / 2);
-  const int ntiles = node.y;
-  const uint16_t* X = uhat + (size_t)bh * N * D;
-  int32_t* ids = idx + (size_t)bh * N + pos0;
-  double* pv = pval + (size_t)bh * N + pos0;
-  int32_t* pi = pidx + (size_t)bh * N + pos0;
-
-  // ---- phase 1: Gram matrix and column sums of the group
-  for (int j = tid; j < G::ACC * G::THREADS; j += G::THREADS) acc64[j] = 0.0;
-  float acc[G::ACC];
-#pragma unroll
-  for (int j = 0; j < G::ACC; ++j) acc[j] = 0.f;
-  double csum = 0.0;
-#pragma unroll
-  for (int s = 0; s < STAGES - 1; ++s) {
-    if (s < ntiles) G::load_tile(tiles + s * G::TILE, X, ids + s * BLK, 0, tid);
-    cp_async_commit();
-  }
-  for (int it = 0; it < ntiles; ++it) {
-    cp_async_wait<STAGES - 2>();
-    __syncthreads();
-    const int nxt = it + STAGES - 1;
-    if (nxt < ntiles) G::load_tile(tiles + (nxt % STAGES) * G::TILE, X, ids + nxt * BLK, 0, tid);
-    cp_async_commit();
-    const uint16_t* sm = tiles + (it % STAGES) * G::TILE;
-    G::tile_mma(sm, acc, warp, lane);
-    {
-      // column sums: thread covers column tid % D over rows (tid / D) + k * (256 / D)
-      constexpr int RSTEP = 256 / D;
-      float c4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int r = tid / D, k = 0; r < BLK; r += RSTEP, ++k) c4[k & 3] += bf2f(sm[r * G::RS + (tid % D)]);
-      csum += (double)((c4[0] + c4[1]) + (c4[2] + c4[3]));
-    }
-    if ((it + 1) % G::FLUSH == 0 || it == ntiles - 1) G::flush(acc, acc64, tid);
-  }
-  cp_async_wait<0>();
-  const double invn = 1.0 / (double)n;
-  {
-    double* cs = reinterpret_cast<double*>(tiles);   // tiles are drained: reuse for the column reduction
-    __syncthreads();                                  // every warp is done with the last tile
-    cs[tid] = csum;
-    __syncthreads();
-    if (tid < D) {
-      double t = 0.0;
-      for (int k = 0; k < 256 / D; ++k) t += cs[tid + k * D];
-      mus[tid] = t * invn;
-    }
-  }
-  __syncthreads();
-
-  // ---- phase 2: S = G/n - mu mu^T, written over the accumulators as a D x D matrix
-  {
-    double g[G::ACC];
-#pragma unroll
-    for (int j = 0; j < G::ACC; ++j) g[j] = acc64[j * G::THREADS + tid];
-    __syncthreads();
-#pragma unroll
-    for (int j = 0; j < G::ACC; ++j) {
-      int row, col;
-      G::coord(j, warp, lane, row, col);
-      acc64[row * D + col] = g[j] * invn - mus[row] * mus[col];
-    }
-  }
-  __syncthreads();
-
-  power_iterate<D>(acc64, vs);
-
-  // ---- phase 4: projections p_i = v . u_i - v . mu (float64); best |p|, lowest index
-  double best_abs = -1.0, best_p = 0.0;
-  int best_id = 0x7fffffff;
-  {
-    constexpr int QD = D / 4;
-    const int tok = tid >> 2, qd = tid & 3;
-    double vr[QD];
-#pragma unroll
-    for (int j = 0; j < QD; ++j) vr[j] = vs[qd * QD + j];
-    double vmu = 0.0;
-#pragma unroll 8
-    for (int j = 0; j < D; ++j) vmu = fma(vs[j], mus[j], vmu);
-#pragma unroll
-    for (int s = 0; s < STAGES - 1; ++s) {
-      if (s < ntiles) G::load_tile(tiles + s * G::TILE, X, ids + s * BLK, 0, tid);
-      cp_async_commit();
-    }
-    for (int it = 0; it < ntiles; ++it) {
-      cp_async_wait<STAGES - 2>();
-      __syncthreads();
-      const int nxt = it + STAGES - 1;
-      if (nxt < ntiles) G::load_tile(tiles + (nxt % STAGES) * G::TILE, X, ids + nxt * BLK, 0, tid);
-      cp_async_commit();
-      const uint16_t* sm = tiles + (it % STAGES) * G::TILE;
-      const uint4* rr = reinterpret_cast<const uint4*>(sm + tok * G::RS + qd * QD);
-      double s4[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll
-      for (int c = 0; c < QD / 8; ++c) {
-        const uint4 w = rr[c];
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          s4[e] = fma(vr[8 * c + 2 * e], (double)bf_lo(ws[e]), s4[e]);
-          s4[e] = fma(vr[8 * c + 2 * e + 1], (double)bf_hi(ws[e]), s4[e]);
-        }
-      }
-      double s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      s += __shfl_xor_sync(0xffffffffu, s, 2);
-      s -= vmu;
-      if (qd == 0) {
-        const int pos = it * BLK + tok;
-        const int id = ids[pos];
-        pv[pos] = s;
-        pi[pos] = id;
-        const double a = fabs(s);
-        if (a > best_abs || (a == best_abs && id < best_id)) { best_abs = a; best_p = s; best_id = id; }
-      }
-    }
-    cp_async_wait<0>();
-  }
-  // block argmax of (|p|, -index)
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const double oa = __shfl_xor_sync(0xffffffffu, best_abs, o);
-    const double op = __shfl_xor_sync(0xffffffffu, best_p, o);
-    const int oi = __shfl_xor_sync(0xffffffffu, best_id, o);
-    if (oa > best_abs || (oa == best_abs && oi < best_id)) { best_abs = oa; best_p = op; best_id = oi; }
-  }
-  if (lane == 0) { red_d[warp] = best_p; red_i[warp] = best_id; zs[warp] = best_abs; }
-  __syncthreads();
-  if (tid == 0) {
-    double ba = zs[0], bp = red_d[0];
-    int bi = red_i[0];
-    for (int w = 1; w < 8; ++w) {
-      if (zs[w] > ba || (zs[w] == ba && red_i[w] < bi)) { ba = zs[w]; bp = red_d[w]; bi = red_i[w]; }
-    }
-    sh_scalar = (bp < 0.0) ? -1.0 : 1.0;
-  }
-  __syncthreads();
-  const double sgn = sh_scalar;
-
-  cut_and_partition(n, nL, sgn, pv, pi, ids, hist, sh_sel, &sh_key, warp_tot, red_i, status);
-}
-
 // ------------------------------------------------------------------ large groups over many CTAs
-// For the top levels (few, large groups) one group is spread over a grid of
-// chunk CTAs: partial Gram matrices (float64 sums of float32 tile sums), one
-// CTA per group to reduce them and run the power iteration, chunk CTAs for
-// the projections (with each chunk's best |p| candidate), and one CTA per
-// group for orientation, cut and partition. Same arithmetic as
-// split_level_kernel, so both paths give the same split.
+// Every level above the subtree level spreads a group over a grid of chunk
+// CTAs (32 tiles each): partial Gram matrices (float64 sums of float32 tile
+// sums), one CTA per group to reduce them and run the power iteration,
+// chunk CTAs for the projections (with each chunk's best |p| candidate), and
+// one CTA per group for orientation, cut and partition. When a level's
+// groups are the two halves of each group one level up, only left halves
+// get chunk Gram partials: a right half's Gram sum is its parent's (kept
+// from the level above) minus its sibling's.
 constexpr int BIG_CHUNK_TILES = 32;
 
 template <int D>
 __global__ void __launch_bounds__(256, 1)
 big_gram_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restrict__ nodes, int nnodes,
-                int chunks, const int32_t* __restrict__ idx, double* __restrict__ part) {
+                int chunks, int kstep, const int32_t* __restrict__ idx, double* __restrict__ part) {
   using G = Gram<D>;
   using SM = SplitSmem<D>;
   constexpr int STAGES = SM::STAGES;
@@ -677,7 +517,7 @@ big_gram_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restrict
   double* acc64 = reinterpret_cast<double*>(smem_raw);
   uint16_t* tiles = reinterpret_cast<uint16_t*>(smem_raw + SM::acc_bytes);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int c = blockIdx.x, k = blockIdx.y, bh = blockIdx.z;
+  const int c = blockIdx.x, k = blockIdx.y * kstep, bh = blockIdx.z;
   const int2 node = nodes[k];
   const int t0 = c * BIG_CHUNK_TILES, t1 = min(node.y, t0 + BIG_CHUNK_TILES);
   const int ntiles = max(0, t1 - t0);
@@ -733,19 +573,30 @@ big_gram_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restrict
 template <int D>
 __global__ void __launch_bounds__(256, 1)
 big_solve_kernel(const int2* __restrict__ nodes, int nnodes, int chunks, const double* __restrict__ part,
-                 double* __restrict__ info) {
+                 double* __restrict__ info, int derive, const double* __restrict__ gpar, int npar,
+                 double* __restrict__ gout) {
+  // The group's Gram sum G = sum u u^T and column sums: from its own chunk
+  // partials, or (derive) a right child's as its parent's minus its left
+  // sibling's, the parent's having been stored one level up. Stored again
+  // (gout) when the next level derives from this one.
   extern __shared__ __align__(128) unsigned char smem_raw[];
   double* Smat = reinterpret_cast<double*>(smem_raw);      // D x D
   __shared__ double mus[D], vs[D];
   const int tid = threadIdx.x, k = blockIdx.x, bh = blockIdx.y;
   const int2 node = nodes[k];
   const int n = node.y * BLK;
-  const int used = (node.y + BIG_CHUNK_TILES - 1) / BIG_CHUNK_TILES;
-  const double* src = part + (size_t)(bh * nnodes + k) * chunks * (size_t)(D * D + D);
+  const int ks = derive ? (k & ~1) : k;                    // node whose partials exist
+  const bool right = derive && (k & 1);
+  const int used = (nodes[ks].y + BIG_CHUNK_TILES - 1) / BIG_CHUNK_TILES;
+  const double* src = part + (size_t)(bh * nnodes + ks) * chunks * (size_t)(D * D + D);
+  const double* par = right ? gpar + (size_t)(bh * npar + (k >> 1)) * (size_t)(D * D + D) : nullptr;
+  double* gsave = gout ? gout + (size_t)(bh * nnodes + k) * (size_t)(D * D + D) : nullptr;
   const double invn = 1.0 / (double)n;
   if (tid < D) {
     double t = 0.0;
     for (int c = 0; c < used; ++c) t += src[(size_t)c * (D * D + D) + D * D + tid];
+    if (right) t = par[D * D + tid] - t;
+    if (gsave) gsave[D * D + tid] = t;
     mus[tid] = t * invn;
   }
   __syncthreads();
@@ -765,7 +616,11 @@ big_solve_kernel(const int2* __restrict__ nodes, int nnodes, int chunks, const d
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int e = e0 + u * blockDim.x;
-      if (e < D * D) Smat[e] = t[u] * invn - mus[e / D] * mus[e % D];
+      if (e < D * D) {
+        const double g = right ? par[e] - t[u] : t[u];
+        if (gsave) gsave[e] = g;
+        Smat[e] = g * invn - mus[e / D] * mus[e % D];
+      }
     }
   }
   __syncthreads();
@@ -900,7 +755,7 @@ big_select_kernel(int N, const int2* __restrict__ nodes, int nnodes, int chunks,
 // One CTA per node of at most SUB_BLOCKS blocks at the first level where all
 // nodes are that small: the node's normalised whitened rows are staged in
 // shared memory once and every remaining split of its subtree is done
-// on-chip (same split rule as split_level_kernel): Gram by mma.sync with
+// on-chip (same split rule as the chunked levels): Gram by mma.sync with
 // per-lane gathered ldmatrix rows, float64 covariance and power iteration in
 // the MMA fragment layout, float64 projections, orientation, and the cut by
 // exact ranks of (projection, index) - the node's slice of the local order
@@ -1253,8 +1108,6 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
   init_idx_kernel<<<(int)std::min<long>((total + 255) / 256, 4096), 256, 0, s>>>(idx, pl.N, total);
 
   const size_t smem_s = SplitSmem<D>::bytes;
-  e = cudaFuncSetAttribute(split_level_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s);
-  if (e != cudaSuccess) return e;
   const size_t smem_t = SubSmem<D>::bytes;
   e = cudaFuncSetAttribute(subtree_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_t);
   if (e != cudaSuccess) return e;
@@ -1269,24 +1122,26 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
   double* bpart = ws_at<double>(ws, pl.off_bigpart);
   double* binfo = ws_at<double>(ws, pl.off_biginfo);
   double* bcand = ws_at<double>(ws, pl.off_bigcand);
+  double* gstore[2] = {ws_at<double>(ws, pl.off_gstore[0]), ws_at<double>(ws, pl.off_gstore[1])};
   for (int lv = 0; lv < pl.nlevels; ++lv) {
-    if (pl.level_chunks[lv] > 0) {   // few large groups: spread each over chunk CTAs
-      const int cnt = pl.level_count[lv], ch = pl.level_chunks[lv];
-      const int2* nd = nodes + pl.level_off[lv];
-      big_gram_kernel<D><<<dim3(ch, cnt, pl.BH), 256, smem_s, s>>>(uhat, pl.N, nd, cnt, ch, idx, bpart);
-      big_solve_kernel<D><<<dim3(cnt, pl.BH), 256, smem_solve, s>>>(nd, cnt, ch, bpart, binfo);
-      big_project_kernel<D><<<dim3(ch, cnt, pl.BH), 256, smem_proj, s>>>(uhat, pl.N, nd, cnt, ch, idx, binfo, pval,
-                                                                        pidx, bcand);
-      big_select_kernel<<<dim3(cnt, pl.BH), 256, 0, s>>>(pl.N, nd, cnt, ch, bcand, idx, pval, pidx, status);
-      continue;
-    }
     if (pl.level_maxg[lv] <= SUB_BLOCKS) {   // this level and everything below it, in shared memory
       subtree_kernel<D><<<dim3(pl.level_count[lv], pl.BH), 256, smem_t, s>>>(uhat, pl.N, nodes + pl.level_off[lv],
                                                                             idx, status);
       break;
     }
-    split_level_kernel<D><<<dim3(pl.level_count[lv], pl.BH), 256, smem_s, s>>>(
-        uhat, pl.N, nodes + pl.level_off[lv], idx, pval, pidx, status);
+    // each group spread over chunk CTAs; a right child's Gram derived from its parent's
+    const int cnt = pl.level_count[lv], ch = pl.level_chunks[lv];
+    const int2* nd = nodes + pl.level_off[lv];
+    const int derive = pl.level_derive[lv];
+    const int kstep = derive ? 2 : 1;
+    double* gpar = derive ? gstore[(lv - 1) & 1] : nullptr;
+    double* gout = pl.level_store[lv] ? gstore[lv & 1] : nullptr;
+    big_gram_kernel<D><<<dim3(ch, cnt / kstep, pl.BH), 256, smem_s, s>>>(uhat, pl.N, nd, cnt, ch, kstep, idx, bpart);
+    big_solve_kernel<D><<<dim3(cnt, pl.BH), 256, smem_solve, s>>>(nd, cnt, ch, bpart, binfo, derive, gpar,
+                                                                   derive ? pl.level_count[lv - 1] : 0, gout);
+    big_project_kernel<D><<<dim3(ch, cnt, pl.BH), 256, smem_proj, s>>>(uhat, pl.N, nd, cnt, ch, idx, binfo, pval,
+                                                                      pidx, bcand);
+    big_select_kernel<<<dim3(cnt, pl.BH), 256, 0, s>>>(pl.N, nd, cnt, ch, bcand, idx, pval, pidx, status);
   }
   const long nbt = (long)pl.BH * pl.nb;
   leaf_sort_kernel<<<(int)((nbt + 7) / 8), 256, 0, s>>>(idx, perm, nbt);

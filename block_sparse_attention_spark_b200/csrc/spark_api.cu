@@ -76,11 +76,19 @@ bool make_plan(const spark_params* p, Plan* pl) {
     P.sub_level = P.nlevels;
     for (int lv = 0; lv < P.nlevels; ++lv)
       if (P.level_maxg[lv] <= 9) { P.sub_level = lv; break; }
-    // groups of two or more 32-tile chunks are spread over one CTA per chunk
+    // every level above the subtree level: groups spread over one CTA per
+    // 32-tile chunk; when a level's groups are exactly the children of the
+    // previous level's (two per parent), only left children's Gram sums are
+    // computed and right children's are derived from their parents'
     P.level_chunks.assign(P.nlevels, 0);
+    P.level_derive.assign(P.nlevels, 0);
+    P.level_store.assign(P.nlevels, 0);
     for (int lv = 0; lv < P.sub_level; ++lv) {
-      const int ch = (P.level_maxg[lv] + 31) / 32;
-      if (ch >= 2) P.level_chunks[lv] = ch;
+      P.level_chunks[lv] = std::max(1, (P.level_maxg[lv] + 31) / 32);
+      if (lv > 0 && P.level_count[lv] == 2 * P.level_count[lv - 1]) {
+        P.level_derive[lv] = 1;
+        P.level_store[lv - 1] = 1;
+      }
     }
   }
   {
@@ -112,6 +120,11 @@ bool make_plan(const spark_params* p, Plan* pl) {
     P.off_bigpart = take(std::max<size_t>(part, 8));
     P.off_biginfo = take(std::max<size_t>(info, 8));
     P.off_bigcand = take(std::max<size_t>(cand, 8));
+    size_t gs = 8;
+    for (int lv = 0; lv < P.nlevels; ++lv)
+      if (P.level_store[lv]) gs = std::max(gs, (size_t)P.BH * P.level_count[lv] * (d * d + d) * 8);
+    P.off_gstore[0] = take(gs);
+    P.off_gstore[1] = take(gs);
   }
   P.off_perm = take(BH * N * 4);
   P.off_sel = take(BH * nb * (size_t)P.ksel * 4);
@@ -174,7 +187,7 @@ int32_t spark_forward_launches(const spark_params* p) {
   // moments 2; reblock: whiten, normalise, tree, init, split levels, subtree, leaves;
   // select: block statistics, then scores + top-K per chunk of heads; attention 1
   int split_launches = 0;
-  for (int lv = 0; lv < pl.sub_level; ++lv) split_launches += pl.level_chunks[lv] > 0 ? 4 : 1;
+  for (int lv = 0; lv < pl.sub_level; ++lv) split_launches += 4;
   const int reblock = 4 + split_launches + (pl.sub_level < pl.nlevels ? 1 : 0) + 1;
   const int select = 1 + 2 * ((pl.BH + pl.score_heads - 1) / pl.score_heads);
   return 2 + reblock + select + 1;

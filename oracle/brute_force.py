@@ -18,7 +18,7 @@ import math
 import numpy as np
 
 
-def forward(q, k, v, perm, ksel, summary="reweight"):
+def forward(q, k, v, perm, ksel, summary="reweight", tail="query"):
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -61,7 +61,10 @@ def forward(q, k, v, perm, ksel, summary="reweight"):
     exact_mask = chosen[blk][:, blk]              # [N, N]: key j's block is kept for query i
     comp_mask = ~chosen[blk]                      # [N, nb]: block b is summarised for query i
     L_exact = np.where(exact_mask, q @ k.T * c, -np.inf)
-    L_comp = np.where(comp_mask, q @ kt.T * c + beta[None, :], -np.inf)
+    # compressed logits with each query's own q, or (tail granularity "block")
+    # with the mean query of the permuted block it sits in
+    qc = q if tail == "query" else Qm[blk]
+    L_comp = np.where(comp_mask, qc @ kt.T * c + beta[None, :], -np.inf)
     m = np.maximum(L_exact.max(axis=1), L_comp.max(axis=1))
     E = np.exp(L_exact - m[:, None])
     C = np.exp(L_comp - m[:, None])

@@ -278,7 +278,7 @@ def select(qm, km, ksel):
 # --------------------------------------------------------------------------
 # a5-a7. exact branch, compressed branch, merge
 
-def attention(q, k, v, perm, sel, kt, vt, beta, rows=None):
+def attention(q, k, v, perm, sel, kt, vt, beta, rows=None, tail="query", qm=None):
     """a5-a7, R11: each query i in permuted block a attends exactly to every
     key of its selected blocks ([P1] exact branch) and, with its own real q_i
     ([P2] "keeps a real Q per query and downsamples only K/V"), to the summary
@@ -286,6 +286,12 @@ def attention(q, k, v, perm, sel, kt, vt, beta, rows=None):
     branches are one softmax: o_i = (sum_exact e^s v_j + sum_comp e^l v~_b) /
     (sum_exact e^s + sum_comp e^l), i.e. the log-sum-exp merge of the two
     partial softmaxes. The row is written at the token's original index.
+
+    tail="block" is the coarser tail granularity ([P2] Inputs,
+    tail_granularity; reading R15): the compressed logits of every query in
+    block a use the block's mean query Qbar_a (block_means of q, the same
+    means the selection scores use) instead of the query itself; the exact
+    branch keeps the real q_i. qm: those block means (computed if None).
 
     rows: optional iterable of query blocks to evaluate (default all).
     Returns out [N, d] (rows of skipped blocks are NaN) and lse [N] (natural
@@ -296,6 +302,10 @@ def attention(q, k, v, perm, sel, kt, vt, beta, rows=None):
     N, d = q.shape
     nb = N // BLOCK
     scale = 1.0 / math.sqrt(d)
+    if tail not in ("query", "block"):
+        raise ValueError(tail)
+    if tail == "block" and qm is None:
+        qm = block_means(q, perm)
     out = np.full((N, d), np.nan)
     lse = np.full(N, np.nan)
     blocks = range(nb) if rows is None else rows
@@ -306,7 +316,11 @@ def attention(q, k, v, perm, sel, kt, vt, beta, rows=None):
         chosen[sel[a]] = True
         krows = np.concatenate([perm[b * BLOCK:(b + 1) * BLOCK] for b in sel[a]])
         s_exact = Qa @ k[krows].T * scale
-        s_comp = Qa @ kt[~chosen].T * scale + beta[~chosen]
+        if tail == "query":
+            s_comp = Qa @ kt[~chosen].T * scale + beta[~chosen]
+        else:
+            s_comp = np.broadcast_to(np.asarray(qm[a], dtype=np.float64) @ kt[~chosen].T * scale + beta[~chosen],
+                                     (BLOCK, int((~chosen).sum())))
         m = np.maximum(s_exact.max(axis=1),
                        s_comp.max(axis=1) if s_comp.shape[1] else -np.inf)
         e_exact = np.exp(s_exact - m[:, None])
@@ -332,7 +346,7 @@ def dense_attention(q, k, v):
 # whole forward pass of one head
 
 def forward_head(q, k, v, ratio=0.2, topk_blocks=0, layout="q_reuse_k",
-                 summary="reweight", perm=None, rows=None):
+                 summary="reweight", perm=None, rows=None, tail="query"):
     """Every intermediate of the forward pass for one (batch item, head).
 
     layout: "q_reuse_k" partitions the queries under M_K and reuses that
@@ -355,7 +369,7 @@ def forward_head(q, k, v, ratio=0.2, topk_blocks=0, layout="q_reuse_k",
     qm, km = block_means(q, perm), block_means(k, perm)
     sel = select(qm, km, ksel)
     kt, vt, beta = summaries(k, v, perm, qbar, summary)
-    out, lse = attention(q, k, v, perm, sel, kt, vt, beta, rows=rows)
+    out, lse = attention(q, k, v, perm, sel, kt, vt, beta, rows=rows, tail=tail, qm=qm)
     return {"MQ": MQ, "MK": MK, "qbar": qbar, "perm": perm, "ksel": ksel,
             "qm": qm, "km": km, "sel": sel, "kt": kt, "vt": vt, "beta": beta,
             "out": out, "lse": lse}

@@ -44,9 +44,16 @@ def _select_lowest(qm, km, ksel):
     return _orig["select"](-qm, km, ksel)
 
 
-def _attention_unscaled(q, k, v, perm, sel, kt, vt, beta, rows=None):
+def _attention_unscaled(q, k, v, perm, sel, kt, vt, beta, rows=None, **kw):
     s = math.sqrt(q.shape[1])
-    return _orig["attention"](q * s, k, v, perm, sel, kt, vt, beta, rows)
+    return _orig["attention"](q * s, k, v, perm, sel, kt, vt, beta, rows, **kw)
+
+
+def _block_tail_from_head_anchor(q, k, v, perm, sel, kt, vt, beta, rows=None, tail="query", qm=None):
+    # block tail built from the head's mean query instead of each block's
+    if tail == "block":
+        qm = np.repeat(np.asarray(q, dtype=np.float64).mean(axis=0)[None, :], len(q) // 64, axis=0)
+    return _orig["attention"](q, k, v, perm, sel, kt, vt, beta, rows, tail=tail, qm=qm)
 
 
 def _truncating_round(x):
@@ -74,6 +81,8 @@ MUTANTS = [
     ("split_direction", _uncentered_direction, [pins.test_split_direction_is_top_eigenvector]),
     ("select", _select_lowest, [pins.test_select_against_full_sort]),
     ("attention", _attention_unscaled, [pins.test_density_one_is_dense_attention]),
+    ("attention", _block_tail_from_head_anchor,
+     [lambda: pins.test_block_tail_matches_brute_force(256, 8, 0.25, "reweight")]),
     ("round_bf16", _truncating_round, [pins.test_round_bf16_matches_bit_rounding]),
     ("split_group", _split_ceil_left, [pins.test_split_group_orientation_and_capacity]),
 ]

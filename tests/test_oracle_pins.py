@@ -426,6 +426,44 @@ def test_oracle_matches_brute_force(N, d, ratio, summary):
     assert np.allclose(res["lse"], bf["lse"], rtol=1e-12, atol=1e-12)
 
 
+@pytest.mark.parametrize("N,d,ratio,summary", [(128, 8, 0.5, "reweight"), (256, 8, 0.25, "reweight"),
+                                               (256, 4, 0.5, "meanpool")])
+def test_block_tail_matches_brute_force(N, d, ratio, summary):
+    """Tail granularity "block" (compressed logits from the block's mean
+    query) against the loop-free brute-force statement."""
+    q, k, v = rand_qkv(N, d, seed=3 * N + d, scale=1.3)
+    res = so.forward_head(q, k, v, ratio=ratio, summary=summary, tail="block")
+    bf = brute_force.forward(q, k, v, res["perm"], res["ksel"], summary, tail="block")
+    assert np.allclose(res["out"], bf["out"], rtol=1e-12, atol=1e-12)
+    assert np.allclose(res["lse"], bf["lse"], rtol=1e-12, atol=1e-12)
+    ref = so.forward_head(q, k, v, ratio=ratio, summary=summary, tail="query")
+    assert not np.allclose(res["out"], ref["out"], rtol=1e-6, atol=1e-6)   # the two tails differ
+
+
+def test_block_tail_equals_query_tail_for_uniform_blocks():
+    """When every query of a permuted block equals the block's mean query,
+    the two tail granularities are the same computation."""
+    r = np.random.default_rng(11)
+    N, d = 256, 8
+    base = bf16(r.standard_normal((N // 64, d)))
+    q = np.repeat(base, 64, axis=0)                    # identical queries per positional block
+    k = bf16(r.standard_normal((N, d)))
+    v = bf16(r.standard_normal((N, d)))
+    perm = np.arange(N)
+    a = so.forward_head(q, k, v, ratio=0.25, layout="given", perm=perm, tail="block")
+    b = so.forward_head(q, k, v, ratio=0.25, layout="given", perm=perm, tail="query")
+    assert np.allclose(a["out"], b["out"], rtol=1e-13, atol=1e-13)
+    assert np.allclose(a["lse"], b["lse"], rtol=1e-13, atol=1e-13)
+
+
+def test_block_tail_density_one_is_dense():
+    """At density 1.0 there are no compressed terms: both tails are dense."""
+    q, k, v = rand_qkv(256, 8, seed=5)
+    res = so.forward_head(q, k, v, ratio=1.0, tail="block")
+    ref, _ = so.dense_attention(q, k, v)
+    assert np.allclose(res["out"], ref, rtol=1e-12, atol=1e-12)
+
+
 # ------------------------------------------------------------------ statistics
 
 def test_mass_recall_is_100_at_density_one():

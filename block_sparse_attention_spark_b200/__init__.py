@@ -14,13 +14,14 @@ import os
 __all__ = ["SparkError", "Params", "lib", "params", "num_selected", "workspace_size",
            "host_workspace_size", "workspace_region", "alloc_workspace", "moments", "reblock",
            "positional_perm", "select", "attn_fwd", "forward", "forward_host", "get_status",
-           "LAYOUTS", "SUMMARIES", "WS"]
+           "LAYOUTS", "SUMMARIES", "TAILS", "WS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libspark.so")
 
 LAYOUTS = {"q_reuse_k": 0, "k_reuse_q": 1}
 SUMMARIES = {"reweight": 0, "meanpool": 1}
+TAILS = {"query": 0, "block": 1}
 WS = {"MQ": 0, "MK": 1, "QMEAN": 2, "PERM": 3, "SEL": 4, "QM": 5, "KM": 6, "KT": 7, "VT": 8,
       "BETA": 9, "UHAT": 10}
 STATUS = {0: "SPARK_OK", 1: "SPARK_ERR_INVALID_ARG", 2: "SPARK_ERR_UNSUPPORTED",
@@ -94,9 +95,9 @@ def _check(code: int, where: str):
 
 
 def params(B, H, N, d, topk_ratio=0.2, topk_blocks=0, layout="q_reuse_k",
-           summary="reweight") -> Params:
+           summary="reweight", tail="query") -> Params:
     return Params(B, H, N, d, float(topk_ratio), int(topk_blocks), LAYOUTS[layout],
-                  SUMMARIES[summary], 0)
+                  SUMMARIES[summary], TAILS[tail])
 
 
 def validate(p: Params) -> int:

@@ -242,7 +242,7 @@ struct Maps {
 
 template <int D>
 __global__ void __launch_bounds__(THREADS, 1)
-attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta,
+attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta, const float* __restrict__ ttab,
                const int32_t* __restrict__ perm, const int32_t* __restrict__ sel, int N, int nb,
                int nb_pad, int ksel, uint16_t* __restrict__ out, float* __restrict__ lse, int* status) {
   using L = Layout<D>;
@@ -405,8 +405,10 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
                 mc[i] = max3(mc[i], __uint_as_float(sv[c + 2 * i]), __uint_as_float(sv[c + 2 * i + 1]));
             mt = fmaxf(fmaxf(max3(mc[0], mc[1], mc[2]), max3(mc[3], mc[4], mc[5])), fmaxf(mc[6], mc[7])) * sl2;
           } else {
-            // x = s / sqrt(d) + beta (log2 units), -inf where the row selected the block
-            const float* brow = beta + (size_t)bh * nb_pad + c0;
+            // x = s / sqrt(d) + beta (log2 units), -inf where the row selected the block;
+            // block tail granularity: the query block's precomputed logit row instead
+            const float* brow = ttab ? ttab + ((size_t)bh * nb + a0 + qh) * nb_pad + c0
+                                     : beta + (size_t)bh * nb_pad + c0;
 #pragma unroll
             for (int c4 = 0; c4 < 16; ++c4) {
               const float4 bb = __ldg(reinterpret_cast<const float4*>(brow) + c4);
@@ -415,8 +417,8 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
               for (int e = 0; e < 4; ++e) {
                 const int c = 4 * c4 + e;
                 const uint32_t w = c < 32 ? ex0 : ex1;
-                const float x = ((w >> (c & 31)) & 1u) ? -INFINITY
-                                                       : fmaf(__uint_as_float(sv[c]), sl2, bv[e] * 1.4426950408889634f);
+                const float xs = ttab ? bv[e] : fmaf(__uint_as_float(sv[c]), sl2, bv[e] * 1.4426950408889634f);
+                const float x = ((w >> (c & 31)) & 1u) ? -INFINITY : xs;
                 sv[c] = __float_as_uint(x);
                 mt = fmaxf(mt, x);
               }
@@ -705,7 +707,8 @@ static cudaError_t run(const Plan& pl, const int32_t* perm, const int32_t* sel, 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
   if (e != cudaSuccess) return e;
   const int npairs = (pl.nb + 1) / 2;
-  kern<<<dim3((npairs + SLOTS - 1) / SLOTS, pl.BH), THREADS, Lay::SMEM, s>>>(maps, ws_at<float>(ws, pl.off_beta), perm, sel,
+  const float* ttab = pl.tail == SPARK_TAIL_BLOCK ? ws_at<float>(ws, pl.off_tail) : nullptr;
+  kern<<<dim3((npairs + SLOTS - 1) / SLOTS, pl.BH), THREADS, Lay::SMEM, s>>>(maps, ws_at<float>(ws, pl.off_beta), ttab, perm, sel,
                                                                  pl.N, pl.nb, pl.nb_pad, pl.ksel, out, lse, status);
   return cudaGetLastError();
 }

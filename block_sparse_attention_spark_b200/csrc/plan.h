@@ -17,6 +17,7 @@ constexpr int MOMENT_SPLITS_MAX = 64;
 
 struct Plan {
   int B = 0, H = 0, N = 0, d = 0, BH = 0, nb = 0, ksel = 0, nb_pad = 0;
+  int tail = 0;                   // SPARK_TAIL_*
   int nlevels = 0;
   std::vector<int> level_count;   // nodes that split at each level
   std::vector<int> level_off;     // offset of each level in the node table
@@ -38,6 +39,7 @@ struct Plan {
   size_t off_qm = 0, off_km = 0;
   size_t off_kt = 0, off_vt = 0, off_beta = 0;
   size_t off_scores = 0;           // block-score matrices of score_heads heads (float64 [nb][nb] each)
+  size_t off_tail = 0;             // block-tail compressed logits (float32 [BH][nb][nb_pad], log2 units)
   int score_heads = 1;
   size_t total = 0;
   // extra device room used by spark_forward_host

@@ -298,6 +298,52 @@ topk_kernel(const double* __restrict__ sc, int nb, int ksel, int h0, int heads, 
   }
 }
 
+// tail_logits_kernel: the compressed-branch logits of the block tail
+//   granularity, x_ab = (Qbar_a . k~_b / sqrt(d) + beta_b) * log2(e), for 8
+//   query blocks a per CTA and every summary b (log2 units, as the attention
+//   kernel works in; columns nb .. nb_pad-1 are -inf). float32 dot products of
+//   the float64 block means (rounded to float32) and the bf16 summaries.
+constexpr int TAIL_ROWS = 8;
+
+template <int D>
+__global__ void __launch_bounds__(256)
+tail_logits_kernel(const double* __restrict__ qm, const uint16_t* __restrict__ kt, const float* __restrict__ beta,
+                   int nb, int nb_pad, float* __restrict__ tab) {
+  __shared__ float qa[TAIL_ROWS][D];
+  const int tid = threadIdx.x, a0 = blockIdx.x * TAIL_ROWS, bh = blockIdx.y;
+  for (int e = tid; e < TAIL_ROWS * D; e += blockDim.x) {
+    const int r = e / D, j = e % D;
+    qa[r][j] = a0 + r < nb ? (float)qm[((size_t)bh * nb + a0 + r) * D + j] : 0.f;
+  }
+  __syncthreads();
+  const float scale = 1.0f / sqrtf((float)D), log2e = 1.4426950408889634f;
+  for (int b = tid; b < nb_pad; b += blockDim.x) {
+    float acc[TAIL_ROWS];
+#pragma unroll
+    for (int r = 0; r < TAIL_ROWS; ++r) acc[r] = 0.f;
+    if (b < nb) {
+      const uint4* row = reinterpret_cast<const uint4*>(kt + ((size_t)bh * nb_pad + b) * D);
+#pragma unroll 4
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 w = row[c];
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float lo = bf_lo(ws[e]), hi = bf_hi(ws[e]);
+#pragma unroll
+          for (int r = 0; r < TAIL_ROWS; ++r) acc[r] = fmaf(qa[r][8 * c + 2 * e + 1], hi, fmaf(qa[r][8 * c + 2 * e], lo, acc[r]));
+        }
+      }
+    }
+    const float bb = b < nb ? beta[(size_t)bh * nb_pad + b] : 0.f;
+#pragma unroll
+    for (int r = 0; r < TAIL_ROWS; ++r) {
+      if (a0 + r >= nb) break;
+      tab[((size_t)bh * nb + a0 + r) * nb_pad + b] = b < nb ? (acc[r] * scale + bb) * log2e : -INFINITY;
+    }
+  }
+}
+
 template <int D>
 static cudaError_t run_select(const Plan& pl, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                               const int32_t* perm, const double* qmean, int32_t* sel, int summary,
@@ -313,6 +359,9 @@ static cudaError_t run_select(const Plan& pl, const uint16_t* q, const uint16_t*
   blockstats_kernel<D><<<dim3(pl.nb_pad, pl.BH), 256, 0, s>>>(q, k, v, perm, qmean, pl.N, pl.nb,
                                                               pl.nb_pad, summary, Qp, Kp, Vp, qm, km,
                                                               kt, vt, beta, status);
+  if (pl.tail == SPARK_TAIL_BLOCK)
+    tail_logits_kernel<D><<<dim3((pl.nb + TAIL_ROWS - 1) / TAIL_ROWS, pl.BH), 256, 0, s>>>(
+        qm, kt, beta, pl.nb, pl.nb_pad, ws_at<float>(ws, pl.off_tail));
   double* sc = ws_at<double>(ws, pl.off_scores);
   const int tiles = (pl.nb + SC_TILE - 1) / SC_TILE;
   for (int h0 = 0; h0 < pl.BH; h0 += pl.score_heads) {

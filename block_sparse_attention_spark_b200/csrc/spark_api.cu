@@ -32,7 +32,7 @@ static spark_status validate(const spark_params* p) {
   if (p->topk_blocks < 0) return SPARK_ERR_INVALID_ARG;
   if (p->layout != SPARK_LAYOUT_Q_REUSE_K && p->layout != SPARK_LAYOUT_K_REUSE_Q) return SPARK_ERR_INVALID_ARG;
   if (p->summary != SPARK_SUMMARY_REWEIGHT && p->summary != SPARK_SUMMARY_MEANPOOL) return SPARK_ERR_INVALID_ARG;
-  if (p->tail != SPARK_TAIL_QUERY) return SPARK_ERR_INVALID_ARG;
+  if (p->tail != SPARK_TAIL_QUERY && p->tail != SPARK_TAIL_BLOCK) return SPARK_ERR_INVALID_ARG;
   if (p->N % SPARK_BLOCK != 0) return SPARK_ERR_UNSUPPORTED;
   if (p->d != 64 && p->d != 128) return SPARK_ERR_UNSUPPORTED;
   const long nb = p->N / SPARK_BLOCK;
@@ -50,6 +50,7 @@ bool make_plan(const spark_params* p, Plan* pl) {
   P = Plan();
   P.B = p->B; P.H = p->H; P.N = p->N; P.d = p->d;
   P.BH = p->B * p->H;
+  P.tail = p->tail;
   P.nb = p->N / SPARK_BLOCK;
   P.ksel = num_selected_impl(P.nb, p->topk_ratio, p->topk_blocks);
   P.nb_pad = (P.nb + 2 * SPARK_BLOCK - 1) / (2 * SPARK_BLOCK) * (2 * SPARK_BLOCK);   // summary tiles of 128
@@ -136,6 +137,7 @@ bool make_plan(const spark_params* p, Plan* pl) {
   P.off_kt = take(BH * nbp * d * 2);
   P.off_vt = take(BH * nbp * d * 2);
   P.off_beta = take(BH * nbp * 4);
+  P.off_tail = P.tail == SPARK_TAIL_BLOCK ? take(BH * nb * nbp * 4) : 0;
   {
     // float64 block-score matrices, a chunk of heads at a time (at most
     // 1 GiB, at least one head)
@@ -189,7 +191,7 @@ int32_t spark_forward_launches(const spark_params* p) {
   int split_launches = 0;
   for (int lv = 0; lv < pl.sub_level; ++lv) split_launches += 4;
   const int reblock = 4 + split_launches + (pl.sub_level < pl.nlevels ? 1 : 0) + 1;
-  const int select = 1 + 2 * ((pl.BH + pl.score_heads - 1) / pl.score_heads);
+  const int select = 1 + 2 * ((pl.BH + pl.score_heads - 1) / pl.score_heads) + (pl.tail == SPARK_TAIL_BLOCK ? 1 : 0);
   return 2 + reblock + select + 1;
 }
 

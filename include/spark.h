@@ -75,9 +75,13 @@ enum {
   SPARK_SUMMARY_MEANPOOL = 1   /* ablation: mean k, mean v, beta = ln 64 */
 };
 
-/* tail granularity ([P2]: a real Q per query, only K/V downsampled). */
+/* tail granularity of the compressed branch ([P2] Inputs: tail_granularity;
+ * "What it's doing under the hood": a real Q per query, only K/V downsampled). */
 enum {
-  SPARK_TAIL_QUERY = 0         /* each query attends to the summaries with its own q */
+  SPARK_TAIL_QUERY = 0,        /* each query scores the summaries with its own q */
+  SPARK_TAIL_BLOCK = 1         /* every query of a block scores them with the block's mean
+                                  query (the exact block means the selection uses); the
+                                  exact branch keeps each query's own q */
 };
 
 typedef struct {

@@ -75,8 +75,11 @@ def test_bad_enums_rejected():
     p.summary = 3
     assert spark.validate(p) == 1
     p = P()
-    p.tail = 1
+    p.tail = 2
     assert spark.validate(p) == 1
+    p = P()
+    p.tail = 1                      # SPARK_TAIL_BLOCK is a valid granularity
+    assert spark.validate(p) == 0
     p = P(topk_blocks=-2)
     assert spark.validate(p) == 1
 

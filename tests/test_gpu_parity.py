@@ -27,11 +27,11 @@ def bf16_to_f64(t):
 
 
 def run_stages(w, ratio=None, layout="q_reuse_k", summary="reweight", topk_blocks=0, qkv=None,
-               perm=None):
+               perm=None, tail="query"):
     import torch
     q, k, v = qkv if qkv is not None else make_inputs(w)
     B, H, N, d = q.shape
-    p = spark.params(B, H, N, d, ratio if ratio is not None else w.ratio, topk_blocks, layout, summary)
+    p = spark.params(B, H, N, d, ratio if ratio is not None else w.ratio, topk_blocks, layout, summary, tail)
     ws = spark.alloc_workspace(p)
     qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
     MQ, MK, qmean = spark.moments(p, qd, kd, ws)
@@ -54,7 +54,7 @@ def run_stages(w, ratio=None, layout="q_reuse_k", summary="reweight", topk_block
 
 
 def check_head(r, b, h, layout="q_reuse_k", summary="reweight", rows=None, check_perm=True,
-               report=None):
+               report=None, tail="query"):
     q = bf16_bits_to_f64(r["q"][b, h])
     k = bf16_bits_to_f64(r["k"][b, h])
     v = bf16_bits_to_f64(r["v"][b, h])
@@ -104,7 +104,7 @@ def check_head(r, b, h, layout="q_reuse_k", summary="reweight", rows=None, check
     if report is not None:
         report.append(("sel", b, h, st["rows"], st["mismatched"], st["certified"]))
     # a5-a7 outputs, given the CUDA permutation and selection
-    ref, ref_lse = so.attention(q, k, v, perm, sel, kt, vt, beta, rows=rows)
+    ref, ref_lse = so.attention(q, k, v, perm, sel, kt, vt, beta, rows=rows, tail=tail, qm=qm)
     mask = ~np.isnan(ref[:, 0])
     e = parity.out_errors(r["out"][b, h][mask], ref[mask])
     assert e["max_rel_to_bound"] <= 1.0, e
@@ -159,6 +159,17 @@ def test_layouts_and_summaries(layout, summary):
     r = run_stages(w, layout=layout, summary=summary)
     for h in range(2):
         check_head(r, 0, h, layout=layout, summary=summary)
+
+
+@pytest.mark.parametrize("summary", ["reweight", "meanpool"])
+def test_block_tail_granularity(summary):
+    """SPARK_TAIL_BLOCK: compressed logits from the block's mean query. An odd
+    block count leaves the last query-block pair half empty."""
+    w = tiny_workload("tail", 2, (3, 8, 40), 128, 0.3, seed_index=700)
+    assert w.nb % 2 == 1
+    r = run_stages(w, summary=summary, tail="block")
+    for h in range(2):
+        check_head(r, 0, h, summary=summary, tail="block")
 
 
 def test_topk_blocks_and_batch():

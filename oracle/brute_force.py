@@ -18,7 +18,7 @@ import math
 import numpy as np
 
 
-def forward(q, k, v, perm, ksel, summary="reweight", tail="query"):
+def forward(q, k, v, perm, ksel, summary="reweight", tail="query", perm_k=None):
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -26,14 +26,18 @@ def forward(q, k, v, perm, ksel, summary="reweight", tail="query"):
     nb = N // 64
     c = 1.0 / math.sqrt(d)
 
-    # one-hot block membership of every original token
-    blk = np.empty(N, dtype=np.int64)
-    blk[np.asarray(perm)] = np.arange(N) // 64
-    onehot = (blk[:, None] == np.arange(nb)[None, :]).astype(np.float64)  # [N, nb]
+    # one-hot block membership of every original token, for queries and (when
+    # keys are partitioned on their own) for keys
+    def membership(pm):
+        b = np.empty(N, dtype=np.int64)
+        b[np.asarray(pm)] = np.arange(N) // 64
+        return b, (b[:, None] == np.arange(nb)[None, :]).astype(np.float64)   # [N], [N, nb]
+    blk, onehot = membership(perm)
+    kblk, konehot = membership(perm if perm_k is None else perm_k)
 
     # block means and block scores
     Qm = onehot.T @ q / 64.0
-    Km = onehot.T @ k / 64.0
+    Km = konehot.T @ k / 64.0
     s = Qm @ Km.T * c
     # rank of each key block within its row: strictly better scores, or equal
     # scores at a lower block index, come first
@@ -46,19 +50,19 @@ def forward(q, k, v, perm, ksel, summary="reweight", tail="query"):
     qbar = q.mean(axis=0)
     if summary == "meanpool":
         kt = Km.copy()
-        vt = onehot.T @ v / 64.0
+        vt = konehot.T @ v / 64.0
         beta = np.full(nb, math.log(64.0))
     else:
         x = k @ qbar * c                          # anchor logits [N]
-        xmax = np.where(onehot > 0, x[:, None], -np.inf).max(axis=0)   # [nb]
-        ex = np.exp(x - xmax[blk])
-        Z = onehot.T @ ex
-        kt = (onehot.T @ (ex[:, None] * k)) / Z[:, None]
-        vt = (onehot.T @ (ex[:, None] * v)) / Z[:, None]
+        xmax = np.where(konehot > 0, x[:, None], -np.inf).max(axis=0)   # [nb]
+        ex = np.exp(x - xmax[kblk])
+        Z = konehot.T @ ex
+        kt = (konehot.T @ (ex[:, None] * k)) / Z[:, None]
+        vt = (konehot.T @ (ex[:, None] * v)) / Z[:, None]
         beta = xmax + np.log(Z) - kt @ qbar * c
 
     # per-pair rules
-    exact_mask = chosen[blk][:, blk]              # [N, N]: key j's block is kept for query i
+    exact_mask = chosen[blk][:, kblk]             # [N, N]: key j's block is kept for query i
     comp_mask = ~chosen[blk]                      # [N, nb]: block b is summarised for query i
     L_exact = np.where(exact_mask, q @ k.T * c, -np.inf)
     # compressed logits with each query's own q, or (tail granularity "block")

@@ -278,7 +278,7 @@ def select(qm, km, ksel):
 # --------------------------------------------------------------------------
 # a5-a7. exact branch, compressed branch, merge
 
-def attention(q, k, v, perm, sel, kt, vt, beta, rows=None, tail="query", qm=None):
+def attention(q, k, v, perm, sel, kt, vt, beta, rows=None, tail="query", qm=None, perm_k=None):
     """a5-a7, R11: each query i in permuted block a attends exactly to every
     key of its selected blocks ([P1] exact branch) and, with its own real q_i
     ([P2] "keeps a real Q per query and downsamples only K/V"), to the summary
@@ -293,6 +293,10 @@ def attention(q, k, v, perm, sel, kt, vt, beta, rows=None, tail="query", qm=None
     means the selection scores use) instead of the query itself; the exact
     branch keeps the real q_i. qm: those block means (computed if None).
 
+    perm_k: the key (and value) permutation when keys are partitioned apart
+    from the queries (layout "separate"; default: perm for both). Query block
+    a is perm's block a; key block b is perm_k's block b.
+
     rows: optional iterable of query blocks to evaluate (default all).
     Returns out [N, d] (rows of skipped blocks are NaN) and lse [N] (natural
     log of the softmax denominator)."""
@@ -304,6 +308,8 @@ def attention(q, k, v, perm, sel, kt, vt, beta, rows=None, tail="query", qm=None
     scale = 1.0 / math.sqrt(d)
     if tail not in ("query", "block"):
         raise ValueError(tail)
+    if perm_k is None:
+        perm_k = perm
     if tail == "block" and qm is None:
         qm = block_means(q, perm)
     out = np.full((N, d), np.nan)
@@ -314,7 +320,7 @@ def attention(q, k, v, perm, sel, kt, vt, beta, rows=None, tail="query", qm=None
         Qa = q[qrow]
         chosen = np.zeros(nb, dtype=bool)
         chosen[sel[a]] = True
-        krows = np.concatenate([perm[b * BLOCK:(b + 1) * BLOCK] for b in sel[a]])
+        krows = np.concatenate([perm_k[b * BLOCK:(b + 1) * BLOCK] for b in sel[a]])
         s_exact = Qa @ k[krows].T * scale
         if tail == "query":
             s_comp = Qa @ kt[~chosen].T * scale + beta[~chosen]
@@ -346,12 +352,15 @@ def dense_attention(q, k, v):
 # whole forward pass of one head
 
 def forward_head(q, k, v, ratio=0.2, topk_blocks=0, layout="q_reuse_k",
-                 summary="reweight", perm=None, rows=None, tail="query"):
+                 summary="reweight", perm=None, rows=None, tail="query", perm_k=None):
     """Every intermediate of the forward pass for one (batch item, head).
 
     layout: "q_reuse_k" partitions the queries under M_K and reuses that
     partition for K and V (R5, [P1] workflows pin reblock_layout=q_reuse_k);
-    "k_reuse_q" is the mirror (keys under M_Q); "given" uses perm as is."""
+    "k_reuse_q" is the mirror (keys under M_Q); "separate" partitions the
+    queries under M_K and the keys (with their values) under M_Q, each on its
+    own ([P2] under the hood: queries grouped under E[kk^T], keys under
+    E[qq^T]; reading R16); "given" uses perm as is (perm_k too, if given)."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -362,15 +371,18 @@ def forward_head(q, k, v, ratio=0.2, topk_blocks=0, layout="q_reuse_k",
         perm = reblock(q, MK)
     elif layout == "k_reuse_q":
         perm = reblock(k, MQ)
+    elif layout == "separate":
+        perm, perm_k = reblock(q, MK), reblock(k, MQ)
     elif layout != "given":
         raise ValueError(layout)
     perm = np.asarray(perm)
+    perm_k = perm if perm_k is None else np.asarray(perm_k)
     ksel = num_selected(nb, ratio, topk_blocks)
-    qm, km = block_means(q, perm), block_means(k, perm)
+    qm, km = block_means(q, perm), block_means(k, perm_k)
     sel = select(qm, km, ksel)
-    kt, vt, beta = summaries(k, v, perm, qbar, summary)
-    out, lse = attention(q, k, v, perm, sel, kt, vt, beta, rows=rows, tail=tail, qm=qm)
-    return {"MQ": MQ, "MK": MK, "qbar": qbar, "perm": perm, "ksel": ksel,
+    kt, vt, beta = summaries(k, v, perm_k, qbar, summary)
+    out, lse = attention(q, k, v, perm, sel, kt, vt, beta, rows=rows, tail=tail, qm=qm, perm_k=perm_k)
+    return {"MQ": MQ, "MK": MK, "qbar": qbar, "perm": perm, "perm_k": perm_k, "ksel": ksel,
             "qm": qm, "km": km, "sel": sel, "kt": kt, "vt": vt, "beta": beta,
             "out": out, "lse": lse}
 

@@ -49,11 +49,16 @@ def _attention_unscaled(q, k, v, perm, sel, kt, vt, beta, rows=None, **kw):
     return _orig["attention"](q * s, k, v, perm, sel, kt, vt, beta, rows, **kw)
 
 
-def _block_tail_from_head_anchor(q, k, v, perm, sel, kt, vt, beta, rows=None, tail="query", qm=None):
+def _block_tail_from_head_anchor(q, k, v, perm, sel, kt, vt, beta, rows=None, tail="query", qm=None, **kw):
     # block tail built from the head's mean query instead of each block's
     if tail == "block":
         qm = np.repeat(np.asarray(q, dtype=np.float64).mean(axis=0)[None, :], len(q) // 64, axis=0)
-    return _orig["attention"](q, k, v, perm, sel, kt, vt, beta, rows, tail=tail, qm=qm)
+    return _orig["attention"](q, k, v, perm, sel, kt, vt, beta, rows, tail=tail, qm=qm, **kw)
+
+
+def _keys_through_query_perm(q, k, v, perm, sel, kt, vt, beta, rows=None, perm_k=None, **kw):
+    # separate layout: key blocks looked up through the query permutation
+    return _orig["attention"](q, k, v, perm, sel, kt, vt, beta, rows, perm_k=perm, **kw)
 
 
 def _truncating_round(x):
@@ -83,6 +88,8 @@ MUTANTS = [
     ("attention", _attention_unscaled, [pins.test_density_one_is_dense_attention]),
     ("attention", _block_tail_from_head_anchor,
      [lambda: pins.test_block_tail_matches_brute_force(256, 8, 0.25, "reweight")]),
+    ("attention", _keys_through_query_perm,
+     [lambda: pins.test_separate_layout_matches_brute_force(256, 8, 0.25, "reweight")]),
     ("round_bf16", _truncating_round, [pins.test_round_bf16_matches_bit_rounding]),
     ("split_group", _split_ceil_left, [pins.test_split_group_orientation_and_capacity]),
 ]

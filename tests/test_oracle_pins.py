@@ -464,6 +464,42 @@ def test_block_tail_density_one_is_dense():
     assert np.allclose(res["out"], ref, rtol=1e-12, atol=1e-12)
 
 
+@pytest.mark.parametrize("N,d,ratio,summary", [(128, 8, 0.5, "reweight"), (256, 8, 0.25, "reweight"),
+                                               (256, 4, 0.5, "meanpool")])
+def test_separate_layout_matches_brute_force(N, d, ratio, summary):
+    """Layout "separate" (queries grouped under M_K, keys under M_Q, each on
+    its own) against the brute force given both permutations."""
+    q, k, v = rand_qkv(N, d, seed=7 * N + d, scale=1.3)
+    res = so.forward_head(q, k, v, ratio=ratio, summary=summary, layout="separate")
+    assert not np.array_equal(res["perm"], res["perm_k"])      # the two partitions differ here
+    bf = brute_force.forward(q, k, v, res["perm"], res["ksel"], summary, perm_k=res["perm_k"])
+    nb = N // 64
+    chosen = np.zeros((nb, nb), dtype=bool)
+    for a in range(nb):
+        chosen[a, res["sel"][a]] = True
+    assert np.array_equal(chosen, bf["chosen"])
+    assert np.allclose(res["kt"], bf["kt"], rtol=1e-12, atol=1e-12)
+    assert np.allclose(res["out"], bf["out"], rtol=1e-12, atol=1e-12)
+    assert np.allclose(res["lse"], bf["lse"], rtol=1e-12, atol=1e-12)
+
+
+def test_separate_layout_is_shared_layout_when_q_equals_k():
+    """With k = q the two moments coincide, so both partitions coincide and
+    the separate layout is the shared one."""
+    q, _, v = rand_qkv(256, 8, seed=9)
+    a = so.forward_head(q, q, v, ratio=0.25, layout="separate")
+    b = so.forward_head(q, q, v, ratio=0.25, layout="q_reuse_k")
+    assert np.array_equal(a["perm"], a["perm_k"]) and np.array_equal(a["perm"], b["perm"])
+    assert np.array_equal(a["out"], b["out"])
+
+
+def test_separate_layout_density_one_is_dense():
+    q, k, v = rand_qkv(256, 8, seed=13)
+    res = so.forward_head(q, k, v, ratio=1.0, layout="separate")
+    ref, _ = so.dense_attention(q, k, v)
+    assert np.allclose(res["out"], ref, rtol=1e-12, atol=1e-12)
+
+
 # ------------------------------------------------------------------ statistics
 
 def test_mass_recall_is_100_at_density_one():

@@ -19,7 +19,7 @@ __all__ = ["SparkError", "Params", "lib", "params", "num_selected", "workspace_s
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libspark.so")
 
-LAYOUTS = {"q_reuse_k": 0, "k_reuse_q": 1}
+LAYOUTS = {"q_reuse_k": 0, "k_reuse_q": 1, "separate": 2}
 SUMMARIES = {"reweight": 0, "meanpool": 1}
 TAILS = {"query": 0, "block": 1}
 WS = {"MQ": 0, "MK": 1, "QMEAN": 2, "PERM": 3, "SEL": 4, "QM": 5, "KM": 6, "KT": 7, "VT": 8,
@@ -204,9 +204,14 @@ def moments_noalloc(p: Params, q, k, MQ, MK, qmean):
     return MQ, MK, qmean
 
 
+def perm_shape(p: Params):
+    """[B, H, N], or [2, B, H, N] (query, then key permutation) for the separate layout."""
+    return (2, p.B, p.H, p.N) if p.layout == LAYOUTS["separate"] else (p.B, p.H, p.N)
+
+
 def reblock(p: Params, q, k, MQ, MK, ws):
     torch = _torch()
-    perm = torch.empty(p.B, p.H, p.N, dtype=torch.int32, device="cuda")
+    perm = torch.empty(perm_shape(p), dtype=torch.int32, device="cuda")
     _check(lib().spark_reblock(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(MQ), _ptr(MK), _ptr(perm),
                                _ptr(ws), ws.numel(), _stream()), "spark_reblock")
     return perm
@@ -215,7 +220,7 @@ def reblock(p: Params, q, k, MQ, MK, ws):
 def positional_perm(p: Params, grid):
     torch = _torch()
     F, Hl, Wl = grid
-    perm = torch.empty(p.B, p.H, p.N, dtype=torch.int32, device="cuda")
+    perm = torch.empty(perm_shape(p), dtype=torch.int32, device="cuda")
     _check(lib().spark_positional_perm(ctypes.byref(p), F, Hl, Wl, _ptr(perm), _stream()),
            "spark_positional_perm")
     return perm

@@ -18,6 +18,8 @@ constexpr int MOMENT_SPLITS_MAX = 64;
 struct Plan {
   int B = 0, H = 0, N = 0, d = 0, BH = 0, nb = 0, ksel = 0, nb_pad = 0;
   int tail = 0;                   // SPARK_TAIL_*
+  int layout = 0;                 // SPARK_LAYOUT_*
+  int nperm = 1;                  // permutations per pass (2 for SPARK_LAYOUT_SEPARATE)
   int nlevels = 0;
   std::vector<int> level_count;   // nodes that split at each level
   std::vector<int> level_off;     // offset of each level in the node table

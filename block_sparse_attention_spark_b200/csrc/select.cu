@@ -24,6 +24,7 @@ template <int D>
 __global__ void __launch_bounds__(256)
 blockstats_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
                   const uint16_t* __restrict__ v, const int32_t* __restrict__ perm,
+                  const int32_t* __restrict__ perm_k,
                   const double* __restrict__ qmean, int N, int nb, int nb_pad, int summary,
                   uint16_t* __restrict__ Qp, uint16_t* __restrict__ Kp, uint16_t* __restrict__ Vp,
                   double* __restrict__ qm, double* __restrict__ km, uint16_t* __restrict__ kt,
@@ -48,16 +49,19 @@ blockstats_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k
     return;
   }
 
-  // gather + permuted copies; q rows go straight to the column sums below
+  // gather + permuted copies (q through the query permutation, k and v
+  // through the key permutation, the same array unless the layout is separate)
   const int32_t* pr = perm + (size_t)bh * N + (size_t)b * BLK;
+  const int32_t* pk = perm_k + (size_t)bh * N + (size_t)b * BLK;
   for (int c = tid; c < BLK * CH; c += blockDim.x) {
     const int r = c / CH, ch = c % CH;
-    int row = pr[r];
+    int row = pr[r], rowk = pk[r];
     if ((unsigned)row >= (unsigned)N) { set_status(status, STATUS_BAD_INPUT); row = 0; }
-    const size_t src = hb + (size_t)row * D + ch * 8;
+    if ((unsigned)rowk >= (unsigned)N) { set_status(status, STATUS_BAD_INPUT); rowk = 0; }
+    const size_t src = hb + (size_t)row * D + ch * 8, srck = hb + (size_t)rowk * D + ch * 8;
     const size_t dst = hb + ((size_t)b * BLK + r) * D + ch * 8;
-    const uint4 kk = *reinterpret_cast<const uint4*>(k + src);
-    const uint4 vv = *reinterpret_cast<const uint4*>(v + src);
+    const uint4 kk = *reinterpret_cast<const uint4*>(k + srck);
+    const uint4 vv = *reinterpret_cast<const uint4*>(v + srck);
     const uint4 qq = *reinterpret_cast<const uint4*>(q + src);
     *reinterpret_cast<uint4*>(Kp + dst) = kk;
     *reinterpret_cast<uint4*>(Vp + dst) = vv;
@@ -356,7 +360,8 @@ static cudaError_t run_select(const Plan& pl, const uint16_t* q, const uint16_t*
   uint16_t* kt = ws_at<uint16_t>(ws, pl.off_kt);
   uint16_t* vt = ws_at<uint16_t>(ws, pl.off_vt);
   float* beta = ws_at<float>(ws, pl.off_beta);
-  blockstats_kernel<D><<<dim3(pl.nb_pad, pl.BH), 256, 0, s>>>(q, k, v, perm, qmean, pl.N, pl.nb,
+  const int32_t* perm_k = perm + (pl.nperm == 2 ? (size_t)pl.BH * pl.N : 0);
+  blockstats_kernel<D><<<dim3(pl.nb_pad, pl.BH), 256, 0, s>>>(q, k, v, perm, perm_k, qmean, pl.N, pl.nb,
                                                               pl.nb_pad, summary, Qp, Kp, Vp, qm, km,
                                                               kt, vt, beta, status);
   if (pl.tail == SPARK_TAIL_BLOCK)

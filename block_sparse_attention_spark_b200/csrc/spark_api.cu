@@ -30,7 +30,9 @@ static spark_status validate(const spark_params* p) {
   if (p == nullptr) return SPARK_ERR_INVALID_ARG;
   if (p->B < 1 || p->H < 1 || p->N < 1 || p->d < 1) return SPARK_ERR_INVALID_ARG;
   if (p->topk_blocks < 0) return SPARK_ERR_INVALID_ARG;
-  if (p->layout != SPARK_LAYOUT_Q_REUSE_K && p->layout != SPARK_LAYOUT_K_REUSE_Q) return SPARK_ERR_INVALID_ARG;
+  if (p->layout != SPARK_LAYOUT_Q_REUSE_K && p->layout != SPARK_LAYOUT_K_REUSE_Q &&
+      p->layout != SPARK_LAYOUT_SEPARATE)
+    return SPARK_ERR_INVALID_ARG;
   if (p->summary != SPARK_SUMMARY_REWEIGHT && p->summary != SPARK_SUMMARY_MEANPOOL) return SPARK_ERR_INVALID_ARG;
   if (p->tail != SPARK_TAIL_QUERY && p->tail != SPARK_TAIL_BLOCK) return SPARK_ERR_INVALID_ARG;
   if (p->N % SPARK_BLOCK != 0) return SPARK_ERR_UNSUPPORTED;
@@ -51,6 +53,8 @@ bool make_plan(const spark_params* p, Plan* pl) {
   P.B = p->B; P.H = p->H; P.N = p->N; P.d = p->d;
   P.BH = p->B * p->H;
   P.tail = p->tail;
+  P.layout = p->layout;
+  P.nperm = p->layout == SPARK_LAYOUT_SEPARATE ? 2 : 1;
   P.nb = p->N / SPARK_BLOCK;
   P.ksel = num_selected_impl(P.nb, p->topk_ratio, p->topk_blocks);
   P.nb_pad = (P.nb + 2 * SPARK_BLOCK - 1) / (2 * SPARK_BLOCK) * (2 * SPARK_BLOCK);   // summary tiles of 128
@@ -127,7 +131,7 @@ bool make_plan(const spark_params* p, Plan* pl) {
     P.off_gstore[0] = take(gs);
     P.off_gstore[1] = take(gs);
   }
-  P.off_perm = take(BH * N * 4);
+  P.off_perm = take((size_t)P.nperm * BH * N * 4);
   P.off_sel = take(BH * nb * (size_t)P.ksel * 4);
   P.off_Qp = take(BH * N * d * 2);
   P.off_Kp = take(BH * N * d * 2);
@@ -190,7 +194,7 @@ int32_t spark_forward_launches(const spark_params* p) {
   // select: block statistics, then scores + top-K per chunk of heads; attention 1
   int split_launches = 0;
   for (int lv = 0; lv < pl.sub_level; ++lv) split_launches += 4;
-  const int reblock = 4 + split_launches + (pl.sub_level < pl.nlevels ? 1 : 0) + 1;
+  const int reblock = pl.nperm * (4 + split_launches + (pl.sub_level < pl.nlevels ? 1 : 0) + 1);
   const int select = 1 + 2 * ((pl.BH + pl.score_heads - 1) / pl.score_heads) + (pl.tail == SPARK_TAIL_BLOCK ? 1 : 0);
   return 2 + reblock + select + 1;
 }
@@ -212,6 +216,16 @@ spark_status spark_moments(const spark_params* p, const void* q, const void* k, 
   return cuda_status(launch_moments(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, ws, stream));
 }
 
+// The partition(s) of the layout: queries under M_K, keys under M_Q, or both
+// (SPARK_LAYOUT_SEPARATE: query permutation first, key permutation after it).
+static cudaError_t reblock_layout(const Plan& pl, const void* q, const void* k, const double* MQ,
+                                  const double* MK, int32_t* perm, void* ws, cudaStream_t s) {
+  if (pl.layout == SPARK_LAYOUT_K_REUSE_Q) return launch_reblock(pl, (const uint16_t*)k, MQ, perm, ws, status_ptr(), s);
+  cudaError_t e = launch_reblock(pl, (const uint16_t*)q, MK, perm, ws, status_ptr(), s);
+  if (e != cudaSuccess || pl.layout != SPARK_LAYOUT_SEPARATE) return e;
+  return launch_reblock(pl, (const uint16_t*)k, MQ, perm + (size_t)pl.BH * pl.N, ws, status_ptr(), s);
+}
+
 spark_status spark_reblock(const spark_params* p, const void* q, const void* k, const double* MQ,
                            const double* MK, int32_t* perm, void* ws, size_t ws_bytes,
                            cudaStream_t stream) {
@@ -222,10 +236,7 @@ spark_status spark_reblock(const spark_params* p, const void* q, const void* k, 
   if (!q || !k || !MQ || !MK || !perm || !aligned16(q) || !aligned16(k)) return SPARK_ERR_INVALID_ARG;
   const spark_status w = check_ws(pl, ws, ws_bytes);
   if (w != SPARK_OK) return w;
-  const bool qside = p->layout == SPARK_LAYOUT_Q_REUSE_K;
-  const uint16_t* x = (const uint16_t*)(qside ? q : k);
-  const double* M = qside ? MK : MQ;
-  return cuda_status(launch_reblock(pl, x, M, perm, ws, status_ptr(), stream));
+  return cuda_status(reblock_layout(pl, q, k, MQ, MK, perm, ws, stream));
 }
 
 spark_status spark_positional_perm(const spark_params* p, int32_t F, int32_t Hl, int32_t Wl,
@@ -237,7 +248,10 @@ spark_status spark_positional_perm(const spark_params* p, int32_t F, int32_t Hl,
   if (F % 2 != 0 || Hl % 8 != 0 || Wl % 4 != 0) return SPARK_ERR_UNSUPPORTED;
   Plan pl;
   make_plan(p, &pl);
-  return cuda_status(launch_positional(pl, F, Hl, Wl, perm, stream));
+  cudaError_t e = launch_positional(pl, F, Hl, Wl, perm, stream);
+  // the separate layout takes the same fixed tiles for its key permutation
+  if (e == cudaSuccess && pl.nperm == 2) e = launch_positional(pl, F, Hl, Wl, perm + (size_t)pl.BH * pl.N, stream);
+  return cuda_status(e);
 }
 
 spark_status spark_select(const spark_params* p, const void* q, const void* k, const void* v,
@@ -285,8 +299,7 @@ spark_status spark_forward(const spark_params* p, const void* q, const void* k, 
   int32_t* sel = sel_out ? sel_out : ws_at<int32_t>(ws, pl.off_sel);
   cudaError_t e = launch_moments(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, ws, stream);
   if (e != cudaSuccess) return SPARK_ERR_CUDA;
-  const bool qside = p->layout == SPARK_LAYOUT_Q_REUSE_K;
-  e = launch_reblock(pl, (const uint16_t*)(qside ? q : k), qside ? MK : MQ, perm, ws, status_ptr(), stream);
+  e = reblock_layout(pl, q, k, MQ, MK, perm, ws, stream);
   if (e != cudaSuccess) return SPARK_ERR_CUDA;
   e = launch_select(pl, (const uint16_t*)q, (const uint16_t*)k, (const uint16_t*)v, perm, qmean, sel,
                     p->summary, ws, status_ptr(), stream);
@@ -331,7 +344,7 @@ size_t spark_workspace_region(const spark_params* p, int32_t region, size_t* byt
     case SPARK_WS_MQ: off = pl.off_MQ; sz = BH * d * d * 8; break;
     case SPARK_WS_MK: off = pl.off_MK; sz = BH * d * d * 8; break;
     case SPARK_WS_QMEAN: off = pl.off_qmean; sz = BH * d * 8; break;
-    case SPARK_WS_PERM: off = pl.off_perm; sz = BH * N * 4; break;
+    case SPARK_WS_PERM: off = pl.off_perm; sz = (size_t)pl.nperm * BH * N * 4; break;
     case SPARK_WS_SEL: off = pl.off_sel; sz = BH * nb * (size_t)pl.ksel * 4; break;
     case SPARK_WS_QM: off = pl.off_qm; sz = BH * nb * d * 8; break;
     case SPARK_WS_KM: off = pl.off_km; sz = BH * nb * d * 8; break;

@@ -24,7 +24,8 @@
  *
  * Conventions shared by every entry point
  *   - Tensors q, k, v, out are [B, H, N, d] bfloat16, contiguous, row-major,
- *     base address 16-byte aligned. perm is [B, H, N] int32; sel is
+ *     base address 16-byte aligned. perm is [B, H, N] int32 ([2, B, H, N]
+ *     for SPARK_LAYOUT_SEPARATE: query permutation, then key permutation); sel is
  *     [B, H, nb, Ksel] int32 with nb = N / 64 and Ksel = spark_num_selected().
  *   - All pointers are DEVICE pointers unless the entry point says "host".
  *     The caller owns all memory; the library allocates and frees nothing.
@@ -66,7 +67,11 @@ typedef enum {
 /* reblock_layout ([P1] Workflows: every shipped workflow pins q_reuse_k). */
 enum {
   SPARK_LAYOUT_Q_REUSE_K = 0,  /* partition the queries under M_K; K and V reuse it */
-  SPARK_LAYOUT_K_REUSE_Q = 1   /* mirror: partition the keys under M_Q; Q reuses it */
+  SPARK_LAYOUT_K_REUSE_Q = 1,  /* mirror: partition the keys under M_Q; Q reuses it */
+  SPARK_LAYOUT_SEPARATE = 2    /* queries under M_K and keys (with their values) under M_Q,
+                                  each on its own ([P2] under the hood: two-sided reblock);
+                                  every perm below then holds 2*B*H*N entries: the query
+                                  permutation [B,H,N] followed by the key permutation */
 };
 
 /* compressed-branch summaries ([P2]: Reweight replaces mean pooling). */
@@ -145,7 +150,7 @@ spark_status spark_moments_noalloc(const spark_params* p, const void* q, const v
 
 /* Step 2 - reblock ([P1] Spark-Reblock bullet; [P2] under the hood):
  * recursive bisection of the partitioned side (queries for q_reuse_k, keys
- * for k_reuse_q) along the top principal direction of its whitened,
+ * for k_reuse_q, both in turn for separate) along the top principal direction of its whitened,
  * normalised vectors (Cholesky factor of the opposite side's moment),
  * split by rank into 64*floor(g/2) and the rest, down to 64-token leaves.
  *   q, k   : [B,H,N,d] bf16 device, read only
@@ -161,7 +166,8 @@ spark_status spark_reblock(const spark_params* p, const void* q, const void* k,
 /* The fixed-tile layout Spark-Reblock replaces ([P1] Spark-Reblock bullet:
  * "fixed spatio-temporal tiles"): 2x8x4 (frame,row,column) tiles of the
  * F x Hl x Wl latent grid in raster order, ascending index inside a tile.
- * Requires F*Hl*Wl == N and F%2 == Hl%8 == Wl%4 == 0. perm as above. */
+ * Requires F*Hl*Wl == N and F%2 == Hl%8 == Wl%4 == 0. perm as above (for
+ * SPARK_LAYOUT_SEPARATE both halves get the same tiles). */
 spark_status spark_positional_perm(const spark_params* p, int32_t F, int32_t Hl, int32_t Wl,
                                    int32_t* perm, cudaStream_t stream);
 
@@ -170,7 +176,9 @@ spark_status spark_positional_perm(const spark_params* p, int32_t F, int32_t Hl,
  * topk_ratio). Block score s_ab = mean(q over block a) . mean(k over block b)
  * / sqrt(d); per query block the Ksel largest, ties to the lower b, written in
  * ascending order. Also leaves in ws the permuted copies of q, k, v and the
- * key/value summaries spark_attn_fwd reads.
+ * key/value summaries spark_attn_fwd reads. With SPARK_LAYOUT_SEPARATE query
+ * blocks follow the query permutation and key blocks (and the k, v copies and
+ * summaries) the key permutation.
  *   perm  : [B,H,N] int32 device (from spark_reblock, spark_positional_perm
  *           or the caller; must be a bijection per head)
  *   qmean : [B,H,d] float64 device (from spark_moments)

@@ -66,8 +66,22 @@ def check_head(r, b, h, layout="q_reuse_k", summary="reweight", rows=None, check
     assert np.abs(r["MQ"][b, h] - MQ).max() <= 1e-6 * np.abs(MQ).max()
     assert np.abs(r["MK"][b, h] - MK).max() <= 1e-6 * np.abs(MK).max()
     assert np.abs(r["qmean"][b, h] - qbar).max() <= 1e-12 * (1 + np.abs(qbar).max())
-    perm = r["perm"][b, h].astype(np.int64)
-    xs, Ms = (q, MK) if layout == "q_reuse_k" else (k, MQ)
+    if layout == "separate":
+        # query permutation (queries under M_K) and key permutation (keys under M_Q)
+        perm, perm_k = r["perm"][0, b, h].astype(np.int64), r["perm"][1, b, h].astype(np.int64)
+        if check_perm:
+            # the workspace's u_hat is the key side's (the second reblock); the
+            # query side is replayed with the oracle's own u_hat
+            st = parity.certify_perm(q, MK, perm)
+            print("perm q", b, h, st)
+            assert st["failures"] == 0, st
+        xs, Ms = k, MQ
+        perm_side = perm_k
+    else:
+        perm = r["perm"][b, h].astype(np.int64)
+        perm_k = perm
+        xs, Ms = (q, MK) if layout == "q_reuse_k" else (k, MQ)
+        perm_side = perm
     if check_perm:
         # normalised whitened tokens: identical up to isolated 1-ulp roundings
         # (float32 whitening: the error is relative to |u|, so an element far
@@ -79,18 +93,19 @@ def check_head(r, b, h, layout="q_reuse_k", summary="reweight", rows=None, check
             ref_ulp = np.ldexp(1.0, np.frexp(np.abs(U[diff]))[1] - 8)
             dev = np.abs(r["uhat"][b, h][diff] - U[diff])
             assert np.all(dev <= np.maximum(ref_ulp, 4e-6)), dev.max()
-        st = parity.certify_perm(xs, Ms, perm, U=r["uhat"][b, h])
+        st = parity.certify_perm(xs, Ms, perm_side, U=r["uhat"][b, h])
         print("perm", b, h, st)
         assert st["failures"] == 0, st
         if report is not None:
             report.append(("perm", b, h, st["nodes"], st["mismatched"], st["certified"], st["worst"]))
     else:
         parity.check_perm_structure(perm, N)
+        parity.check_perm_structure(perm_k, N)
     # a3 block means (exact sums) and summaries, given the CUDA permutation
-    qm, km = so.block_means(q, perm), so.block_means(k, perm)
+    qm, km = so.block_means(q, perm), so.block_means(k, perm_k)
     assert np.abs(r["qm"][b, h] - qm).max() <= 1e-14 * (1 + np.abs(qm).max())
     assert np.abs(r["km"][b, h] - km).max() <= 1e-14 * (1 + np.abs(km).max())
-    kt, vt, beta = so.summaries(k, v, perm, qbar, summary)
+    kt, vt, beta = so.summaries(k, v, perm_k, qbar, summary)
     gk, gv, gb = r["kt"][b, h, :nb], r["vt"][b, h, :nb], r["beta"][b, h, :nb]
     assert np.all(np.abs(gk - kt) <= 2 ** -8 * np.abs(kt) + 1e-6 * np.abs(kt).max())
     assert np.all(np.abs(gv - vt) <= 2 ** -8 * np.abs(vt) + 1e-6 * np.abs(vt).max())
@@ -104,7 +119,7 @@ def check_head(r, b, h, layout="q_reuse_k", summary="reweight", rows=None, check
     if report is not None:
         report.append(("sel", b, h, st["rows"], st["mismatched"], st["certified"]))
     # a5-a7 outputs, given the CUDA permutation and selection
-    ref, ref_lse = so.attention(q, k, v, perm, sel, kt, vt, beta, rows=rows, tail=tail, qm=qm)
+    ref, ref_lse = so.attention(q, k, v, perm, sel, kt, vt, beta, rows=rows, tail=tail, qm=qm, perm_k=perm_k)
     mask = ~np.isnan(ref[:, 0])
     e = parity.out_errors(r["out"][b, h][mask], ref[mask])
     assert e["max_rel_to_bound"] <= 1.0, e
@@ -153,7 +168,7 @@ def test_density_one_is_dense_attention():
 
 
 @pytest.mark.parametrize("summary", ["reweight", "meanpool"])
-@pytest.mark.parametrize("layout", ["q_reuse_k", "k_reuse_q"])
+@pytest.mark.parametrize("layout", ["q_reuse_k", "k_reuse_q", "separate"])
 def test_layouts_and_summaries(layout, summary):
     w = tiny_workload("lay", 2, (2, 16, 64), 64, 0.25, seed_index=400)
     r = run_stages(w, layout=layout, summary=summary)
@@ -170,6 +185,24 @@ def test_block_tail_granularity(summary):
     r = run_stages(w, summary=summary, tail="block")
     for h in range(2):
         check_head(r, 0, h, summary=summary, tail="block")
+
+
+def test_separate_layout_forward_matches_stages():
+    """spark_forward with the separate layout writes both permutations and the
+    same output as the step-by-step calls."""
+    import torch
+    w = tiny_workload("sep", 2, (2, 16, 64), 128, 0.2, seed_index=800)
+    q, k, v = make_inputs(w)
+    r = run_stages(w, layout="separate", qkv=(q, k, v))
+    p = r["p"]
+    ws = spark.alloc_workspace(p)
+    perm = torch.empty(spark.perm_shape(p), dtype=torch.int32, device="cuda")
+    out = spark.forward(p, to_dev(q), to_dev(k), to_dev(v), ws=ws, perm=perm)
+    assert spark.get_status() == 0
+    assert np.array_equal(perm.cpu().numpy(), r["perm"])
+    assert np.array_equal(bf16_to_f64(out), r["out"])
+    for h in range(2):
+        check_head(r, 0, h, layout="separate")
 
 
 def test_topk_blocks_and_batch():

@@ -18,7 +18,7 @@ import math
 import numpy as np
 
 
-def forward(q, k, v, perm, ksel, summary="reweight", tail="query", perm_k=None):
+def forward(q, k, v, perm, ksel, summary="reweight", tail="query", perm_k=None, context=None):
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -69,11 +69,27 @@ def forward(q, k, v, perm, ksel, summary="reweight", tail="query", perm_k=None):
     # with the mean query of the permuted block it sits in
     qc = q if tail == "query" else Qm[blk]
     L_comp = np.where(comp_mask, qc @ kt.T * c + beta[None, :], -np.inf)
+    if context is not None:
+        # joint attention: every context key is an exact term for every video
+        # query; context queries see every key of both segments
+        qc, kc, vc = (np.asarray(x, dtype=np.float64) for x in context)
+        L_exact = np.concatenate([L_exact, q @ kc.T * c], axis=1)
+        v_exact = np.concatenate([v, vc], axis=0)
+    else:
+        v_exact = v
     m = np.maximum(L_exact.max(axis=1), L_comp.max(axis=1))
     E = np.exp(L_exact - m[:, None])
     C = np.exp(L_comp - m[:, None])
     den = E.sum(axis=1) + C.sum(axis=1)
-    out = (E @ v + C @ vt) / den[:, None]
+    out = (E @ v_exact + C @ vt) / den[:, None]
     lse = m + np.log(den)
-    return {"out": out, "lse": lse, "chosen": chosen, "kt": kt, "vt": vt, "beta": beta,
-            "qm": Qm, "km": Km}
+    res = {"out": out, "lse": lse, "chosen": chosen, "kt": kt, "vt": vt, "beta": beta,
+           "qm": Qm, "km": Km}
+    if context is not None:
+        Lc = qc @ np.concatenate([k, kc]).T * c                         # [C, N + C]
+        mc = Lc.max(axis=1)
+        Ec = np.exp(Lc - mc[:, None])
+        denc = Ec.sum(axis=1)
+        res["outc"] = Ec @ np.concatenate([v, vc]) / denc[:, None]
+        res["lsec"] = mc + np.log(denc)
+    return res

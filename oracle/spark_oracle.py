@@ -338,6 +338,68 @@ def attention(q, k, v, perm, sel, kt, vt, beta, rows=None, tail="query", qm=None
     return out, lse
 
 
+def joint_attention(q, k, v, perm, sel, kt, vt, beta, qc, kc, vc, rows=None, tail="query", qm=None,
+                    perm_k=None):
+    """Joint attention with an exact, dense context segment (reading R17;
+    the step either side of the path in the real model: text / audio /
+    conditioning tokens attend jointly with the video tokens). The video
+    tokens go through the method unchanged (moments, partition, selection and
+    summaries from video tokens only); each video query additionally attends
+    exactly to every context key, inside the same softmax as its exact and
+    compressed terms; each context query attends densely to all N video keys
+    and all C context keys.
+
+    qc, kc, vc: [C, d] context tokens. Returns (out [N, d], lse [N], outc
+    [C, d], lsec [C]); rows of skipped video blocks are NaN."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    qc = np.asarray(qc, dtype=np.float64)
+    kc = np.asarray(kc, dtype=np.float64)
+    vc = np.asarray(vc, dtype=np.float64)
+    if perm_k is None:
+        perm_k = perm
+    N, d = q.shape
+    nb = N // BLOCK
+    scale = 1.0 / math.sqrt(d)
+    if tail == "block" and qm is None:
+        qm = block_means(q, perm)
+    out = np.full((N, d), np.nan)
+    lse = np.full(N, np.nan)
+    blocks = range(nb) if rows is None else rows
+    for a in blocks:
+        qrow = perm[a * BLOCK:(a + 1) * BLOCK]
+        Qa = q[qrow]
+        chosen = np.zeros(nb, dtype=bool)
+        chosen[sel[a]] = True
+        krows = np.concatenate([perm_k[b * BLOCK:(b + 1) * BLOCK] for b in sel[a]])
+        s_exact = np.concatenate([Qa @ k[krows].T, Qa @ kc.T], axis=1) * scale
+        vals = np.concatenate([v[krows], vc], axis=0)
+        if tail == "query":
+            s_comp = Qa @ kt[~chosen].T * scale + beta[~chosen]
+        else:
+            s_comp = np.broadcast_to(np.asarray(qm[a], dtype=np.float64) @ kt[~chosen].T * scale + beta[~chosen],
+                                     (BLOCK, int((~chosen).sum())))
+        m = np.maximum(s_exact.max(axis=1), s_comp.max(axis=1) if s_comp.shape[1] else -np.inf)
+        e_exact = np.exp(s_exact - m[:, None])
+        e_comp = np.exp(s_comp - m[:, None])
+        den = e_exact.sum(axis=1) + e_comp.sum(axis=1)
+        out[qrow] = (e_exact @ vals + e_comp @ vt[~chosen]) / den[:, None]
+        lse[qrow] = m + np.log(den)
+    outc, lsec = dense_attention_lse(qc, np.concatenate([k, kc]), np.concatenate([v, vc]))
+    return out, lse, outc, lsec
+
+
+def dense_attention_lse(q, k, v):
+    """Plain softmax attention with its natural-log denominators."""
+    q = np.asarray(q, dtype=np.float64)
+    s = q @ np.asarray(k, dtype=np.float64).T / math.sqrt(q.shape[1])
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    den = e.sum(axis=1, keepdims=True)
+    return e @ np.asarray(v, dtype=np.float64) / den, (m + np.log(den))[:, 0]
+
+
 def dense_attention(q, k, v):
     """Plain softmax attention, the density-1.0 limit of the method."""
     q = np.asarray(q, dtype=np.float64)

@@ -11,7 +11,7 @@ from oracle import spark_oracle as so
 
 _orig = {name: getattr(so, name) for name in
          ("summaries", "whitening_factor", "split_direction", "select", "attention",
-          "split_group", "round_bf16", "block_means")}
+          "split_group", "round_bf16", "block_means", "dense_attention_lse")}
 
 
 def _beta_without_anchor_term(k, v, perm, qbar, mode="reweight"):
@@ -56,6 +56,11 @@ def _block_tail_from_head_anchor(q, k, v, perm, sel, kt, vt, beta, rows=None, ta
     return _orig["attention"](q, k, v, perm, sel, kt, vt, beta, rows, tail=tail, qm=qm, **kw)
 
 
+def _context_rows_without_context_keys(q, k, v):
+    # context queries that only see the video keys (the context segment dropped)
+    return _orig["dense_attention_lse"](q, k[: len(k) - len(k) % 64], v[: len(v) - len(v) % 64])
+
+
 def _keys_through_query_perm(q, k, v, perm, sel, kt, vt, beta, rows=None, perm_k=None, **kw):
     # separate layout: key blocks looked up through the query permutation
     return _orig["attention"](q, k, v, perm, sel, kt, vt, beta, rows, perm_k=perm, **kw)
@@ -88,6 +93,8 @@ MUTANTS = [
     ("attention", _attention_unscaled, [pins.test_density_one_is_dense_attention]),
     ("attention", _block_tail_from_head_anchor,
      [lambda: pins.test_block_tail_matches_brute_force(256, 8, 0.25, "reweight")]),
+    ("dense_attention_lse", _context_rows_without_context_keys,
+     [lambda: pins.test_joint_attention_matches_brute_force(128, 8, 0.5, 7)]),
     ("attention", _keys_through_query_perm,
      [lambda: pins.test_separate_layout_matches_brute_force(256, 8, 0.25, "reweight")]),
     ("round_bf16", _truncating_round, [pins.test_round_bf16_matches_bit_rounding]),

@@ -500,6 +500,59 @@ def test_separate_layout_density_one_is_dense():
     assert np.allclose(res["out"], ref, rtol=1e-12, atol=1e-12)
 
 
+def _context(C, d, seed, scale=1.3):
+    r = np.random.default_rng(seed)
+    return (bf16(r.standard_normal((C, d)) * scale), bf16(r.standard_normal((C, d)) * scale),
+            bf16(r.standard_normal((C, d))))
+
+
+@pytest.mark.parametrize("N,d,ratio,C", [(128, 8, 0.5, 7), (256, 8, 0.25, 64), (256, 4, 0.5, 100)])
+def test_joint_attention_matches_brute_force(N, d, ratio, C):
+    """Joint attention (dense context segment) against the brute force."""
+    q, k, v = rand_qkv(N, d, seed=11 * N + C, scale=1.3)
+    qc, kc, vc = _context(C, d, seed=C)
+    res = so.forward_head(q, k, v, ratio=ratio)
+    out, lse, outc, lsec = so.joint_attention(q, k, v, res["perm"], res["sel"], res["kt"], res["vt"],
+                                              res["beta"], qc, kc, vc)
+    bf = brute_force.forward(q, k, v, res["perm"], res["ksel"], context=(qc, kc, vc))
+    assert np.allclose(out, bf["out"], rtol=1e-12, atol=1e-12)
+    assert np.allclose(lse, bf["lse"], rtol=1e-12, atol=1e-12)
+    assert np.allclose(outc, bf["outc"], rtol=1e-12, atol=1e-12)
+    assert np.allclose(lsec, bf["lsec"], rtol=1e-12, atol=1e-12)
+
+
+def test_joint_attention_density_one_is_dense_joint():
+    """At density 1.0 the whole thing is dense attention over both segments,
+    for video and context queries alike."""
+    q, k, v = rand_qkv(256, 8, seed=21)
+    qc, kc, vc = _context(40, 8, seed=22)
+    res = so.forward_head(q, k, v, ratio=1.0)
+    out, _, outc, _ = so.joint_attention(q, k, v, res["perm"], res["sel"], res["kt"], res["vt"], res["beta"],
+                                         qc, kc, vc)
+    K, V = np.concatenate([k, kc]), np.concatenate([v, vc])
+    ref, _ = so.dense_attention(q, K, V)
+    refc, _ = so.dense_attention(qc, K, V)
+    assert np.allclose(out, ref, rtol=1e-12, atol=1e-12)
+    assert np.allclose(outc, refc, rtol=1e-12, atol=1e-12)
+
+
+def test_joint_attention_lse_merge():
+    """A video row's joint lse is the log-sum-exp merge of its video-only lse
+    and its lse over the context keys alone."""
+    q, k, v = rand_qkv(256, 8, seed=31)
+    qc, kc, vc = _context(33, 8, seed=32)
+    res = so.forward_head(q, k, v, ratio=0.25)
+    out, lse, _, _ = so.joint_attention(q, k, v, res["perm"], res["sel"], res["kt"], res["vt"], res["beta"],
+                                        qc, kc, vc)
+    _, lse_ctx = so.dense_attention_lse(q, kc, vc)
+    merged = np.logaddexp(res["lse"], lse_ctx)
+    assert np.allclose(lse, merged, rtol=1e-12, atol=1e-12)
+    # and the output is the matching convex combination of the two partial outputs
+    o_ctx, _ = so.dense_attention_lse(q, kc, vc)
+    w = np.exp(res["lse"] - lse)[:, None]
+    assert np.allclose(out, w * res["out"] + (1 - w) * o_ctx, rtol=1e-10, atol=1e-12)
+
+
 # ------------------------------------------------------------------ statistics
 
 def test_mass_recall_is_100_at_density_one():

@@ -13,7 +13,8 @@ import os
 
 __all__ = ["SparkError", "Params", "lib", "params", "num_selected", "workspace_size",
            "host_workspace_size", "workspace_region", "alloc_workspace", "moments", "reblock",
-           "positional_perm", "select", "attn_fwd", "forward", "forward_host", "get_status",
+           "positional_perm", "select", "attn_fwd", "attn_fwd_joint", "forward", "forward_joint",
+           "forward_host", "get_status",
            "LAYOUTS", "SUMMARIES", "TAILS", "WS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -67,6 +68,9 @@ _SIGS = {
     "spark_select": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "spark_attn_fwd": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "spark_forward": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "spark_attn_fwd_joint": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "spark_forward_joint": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _sz,
+                                   _vp]),
     "spark_forward_host": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "spark_get_status": (_i32, [_vp]),
     "spark_strerror": (ctypes.c_char_p, [_i32]),
@@ -242,6 +246,42 @@ def attn_fwd(p: Params, perm, sel, ws, return_lse=False):
     _check(lib().spark_attn_fwd(ctypes.byref(p), _ptr(perm), _ptr(sel), _ptr(out), _ptr(lse),
                                 _ptr(ws), ws.numel(), _stream()), "spark_attn_fwd")
     return (out, lse) if return_lse else out
+
+
+def attn_fwd_joint(p: Params, perm, sel, qc, kc, vc, ws, return_lse=False):
+    """Video rows with the context segment, and the context rows (dense).
+    qc, kc, vc: [B, H, C, d] bf16. Returns (out, outc) or (out, outc, lse, lsec)."""
+    torch = _torch()
+    C = qc.shape[2]
+    for t, n in ((qc, "qc"), (kc, "kc"), (vc, "vc")):
+        _need(t, torch.bfloat16, (p.B, p.H, C, p.d), n)
+    out = torch.empty(p.B, p.H, p.N, p.d, dtype=torch.bfloat16, device="cuda")
+    outc = torch.empty(p.B, p.H, C, p.d, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(p.B, p.H, p.N, dtype=torch.float32, device="cuda") if return_lse else None
+    lsec = torch.empty(p.B, p.H, C, dtype=torch.float32, device="cuda") if return_lse else None
+    _check(lib().spark_attn_fwd_joint(ctypes.byref(p), _ptr(perm), _ptr(sel), _ptr(qc), _ptr(kc), _ptr(vc), C,
+                                      _ptr(out), _ptr(lse), _ptr(outc), _ptr(lsec), _ptr(ws), ws.numel(),
+                                      _stream()), "spark_attn_fwd_joint")
+    return (out, outc, lse, lsec) if return_lse else (out, outc)
+
+
+def forward_joint(p: Params, q, k, v, qc, kc, vc, ws=None):
+    """The whole pass with a context segment. Returns (out, outc)."""
+    torch = _torch()
+    C = qc.shape[2]
+    shp = (p.B, p.H, p.N, p.d)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, shp, n)
+    for t, n in ((qc, "qc"), (kc, "kc"), (vc, "vc")):
+        _need(t, torch.bfloat16, (p.B, p.H, C, p.d), n)
+    if ws is None:
+        ws = alloc_workspace(p)
+    out = torch.empty(shp, dtype=torch.bfloat16, device="cuda")
+    outc = torch.empty(p.B, p.H, C, p.d, dtype=torch.bfloat16, device="cuda")
+    _check(lib().spark_forward_joint(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(qc), _ptr(kc), _ptr(vc), C,
+                                     _ptr(out), None, _ptr(outc), None, _ptr(ws), ws.numel(), _stream()),
+           "spark_forward_joint")
+    return out, outc
 
 
 def forward(p: Params, q, k, v, ws=None, out=None, lse=None, perm=None, sel=None):

@@ -238,13 +238,15 @@ __device__ __forceinline__ int next_block(const uint32_t* um, int from, int nwor
 
 struct Maps {
   CUtensorMap q, k, v, kt, vt;
+  CUtensorMap qc, kc, vc;      // context segment (joint attention); copies of q, k, v when absent
 };
 
 template <int D>
 __global__ void __launch_bounds__(THREADS, 1)
 attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta, const float* __restrict__ ttab,
                const int32_t* __restrict__ perm, const int32_t* __restrict__ sel, int N, int nb,
-               int nb_pad, int ksel, uint16_t* __restrict__ out, float* __restrict__ lse, int* status) {
+               int nb_pad, int ksel, uint16_t* __restrict__ out, float* __restrict__ lse, int C, int nvid,
+               uint16_t* __restrict__ outc, float* __restrict__ lsec, int* status) {
   using L = Layout<D>;
   constexpr int NBAR = 16;                             // barriers per slot
   extern __shared__ unsigned char smem_raw[];
@@ -333,26 +335,42 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
     }
   }
   __syncthreads();
-  int TE[SLOTS], T[SLOTS];
+  // Tiles of a unit. Video pairs (blockIdx.x < nvid): the union blocks, then
+  // the summaries, then the context keys (joint attention, C > 0). Context
+  // query chunks (blockIdx.x >= nvid): every video block, then the context keys.
+  const bool ctx_cta = (int)blockIdx.x >= nvid;
+  int TE[SLOTS], T[SLOTS], TX[SLOTS];                  // exact (or dense) tiles, all tiles, first context tile
   const int TS = (nb + KEYS - 1) / KEYS;               // summary tiles
+  const int TC = (C + KEYS - 1) / KEYS;                // context tiles
 #pragma unroll
   for (int s = 0; s < SLOTS; ++s) {
-    int U = 0;
-    for (int w = 0; w < THREADS / 32; ++w) U += count_sh[w][s];
-    TE[s] = U;                                           // exact tiles: one union block each
-    T[s] = (SLOTS * blockIdx.x + s < npairs) ? U + TS : 0;
+    if (!ctx_cta) {
+      int U = 0;
+      for (int w = 0; w < THREADS / 32; ++w) U += count_sh[w][s];
+      TE[s] = U;                                         // exact tiles: one union block each
+      TX[s] = U + TS;
+      T[s] = (SLOTS * blockIdx.x + s < npairs) ? U + TS + TC : 0;
+    } else {
+      const int cc = SLOTS * ((int)blockIdx.x - nvid) + s;
+      TE[s] = nb;
+      TX[s] = nb;
+      T[s] = cc * ROWS < C ? nb + TC : 0;
+    }
   }
   const uint32_t tmem = tmem_base_sh;
 
   if (warp < 8) {
     // ------------------------------------------------ softmax of slot warp / 4, one thread per row
     const int s = warp >> 2;
-    const int Ts = T[s], TEs = TE[s];
+    const int Ts = T[s], TEs = TE[s], TXs = TX[s];
     if (Ts > 0) {
       const int a0 = 2 * (SLOTS * blockIdx.x + s);
+      const int crow0 = (SLOTS * ((int)blockIdx.x - nvid) + s) * ROWS;   // context CTAs
       const int r = (warp & 3) * 32 + lane;              // query row 0..127 of the pair
       const int qh = r >> 6;                             // which of the two query blocks
-      const bool row_valid = qh == 0 || a0 + 1 < nb;     // uniform per warp
+      // uniform per warp (C - crow0 is a multiple of 32 only at whole warps; rows
+      // of a partial warp past C still take part, their results are not written)
+      const bool row_valid = ctx_cta ? (crow0 + (warp & 3) * 32 < C) : (qh == 0 || a0 + 1 < nb);
       const uint32_t* mymask = selm[s][qh];
       const uint32_t* um = unionm[s];
       const uint32_t tbase = tmem + ((uint32_t)((warp & 3) * 32) << 16) + SLOT_COLS * (uint32_t)s;
@@ -360,19 +378,28 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
       const float sl2 = (1.0f / sqrtf((float)D)) * 1.4426950408889634f;
       const uint64_t sc2 = f2(sl2, sl2);
       float m_ref = -INFINITY, l = 0.f;
-      int cur = next_block(um, 0, nwords);
+      int cur = ctx_cta ? 0 : next_block(um, 0, nwords);
       bool ok = true;
       for (int j = 0; j < Ts; ++j) {
         const uint32_t sc = tbase + 64u * (uint32_t)(j & 1);   // this tile's S (and P) columns
-        // the tile's block (or summary range) and this row's mask, before the wait
-        const bool comp = j >= TEs;
+        // the tile's block (or summary range) and this row's mask, before the wait;
+        // kind 0: exact keys, 1: summaries, 2: context keys (per-column masks for 1, 2)
+        const int kind = j < TEs ? 0 : (j < TXs ? 1 : 2);
+        const bool comp = kind != 0;
         bool take;
         uint32_t ex0 = ~0u, ex1 = ~0u;
         int c0 = 0;
-        if (!comp) {
+        if (kind == 0 && ctx_cta) {
+          take = row_valid;                              // dense: every video block
+        } else if (kind == 0) {
           const int b = cur;
           cur = next_block(um, b + 1, nwords);
           take = row_valid && ((mymask[b >> 5] >> (b & 31)) & 1u);
+        } else if (kind == 2) {
+          const int vc = C - (j - TXs) * KEYS;           // valid context keys in this tile (>= 1)
+          take = row_valid;
+          ex0 = vc >= 32 ? 0u : (~0u << vc);
+          ex1 = vc >= 64 ? 0u : (vc <= 32 ? ~0u : (~0u << (vc - 32)));
         } else {
           c0 = (j - TEs) * KEYS;
           take = row_valid;
@@ -406,18 +433,21 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
             mt = fmaxf(fmaxf(max3(mc[0], mc[1], mc[2]), max3(mc[3], mc[4], mc[5])), fmaxf(mc[6], mc[7])) * sl2;
           } else {
             // x = s / sqrt(d) + beta (log2 units), -inf where the row selected the block;
-            // block tail granularity: the query block's precomputed logit row instead
-            const float* brow = ttab ? ttab + ((size_t)bh * nb + a0 + qh) * nb_pad + c0
-                                     : beta + (size_t)bh * nb_pad + c0;
+            // block tail granularity: the query block's precomputed logit row instead;
+            // context keys: s / sqrt(d), -inf past the end of the segment
+            const bool tab = kind == 1 && ttab != nullptr;
+            const float* brow = kind == 2 ? nullptr
+                                : tab    ? ttab + ((size_t)bh * nb + a0 + qh) * nb_pad + c0
+                                         : beta + (size_t)bh * nb_pad + c0;
 #pragma unroll
             for (int c4 = 0; c4 < 16; ++c4) {
-              const float4 bb = __ldg(reinterpret_cast<const float4*>(brow) + c4);
+              const float4 bb = brow ? __ldg(reinterpret_cast<const float4*>(brow) + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
               const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const int c = 4 * c4 + e;
                 const uint32_t w = c < 32 ? ex0 : ex1;
-                const float xs = ttab ? bv[e] : fmaf(__uint_as_float(sv[c]), sl2, bv[e] * 1.4426950408889634f);
+                const float xs = tab ? bv[e] : fmaf(__uint_as_float(sv[c]), sl2, bv[e] * 1.4426950408889634f);
                 const float x = ((w >> (c & 31)) & 1u) ? -INFINITY : xs;
                 sv[c] = __float_as_uint(x);
                 mt = fmaxf(mt, x);
@@ -490,12 +520,21 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
       fence_after();
       ok = __all_sync(0xffffffffu, ok && !(*(volatile int*)&abort_sh));
       if (ok && row_valid) {
-        const int pos = a0 * BLK + r;
-        const int orig = perm[(size_t)bh * N + pos];
-        const bool dst_ok = (unsigned)orig < (unsigned)N;
-        if (!dst_ok) set_status(status, STATUS_BAD_INPUT);
+        // video rows go to their original index, context rows to their own row
+        size_t orow;
+        bool dst_ok;
+        if (!ctx_cta) {
+          const int orig = perm[(size_t)bh * N + a0 * BLK + r];
+          dst_ok = (unsigned)orig < (unsigned)N;
+          if (!dst_ok) set_status(status, STATUS_BAD_INPUT);
+          orow = (size_t)bh * N + (dst_ok ? orig : 0);
+        } else {
+          dst_ok = crow0 + r < C;
+          orow = (size_t)bh * C + (dst_ok ? crow0 + r : 0);
+        }
+        float* lse_out = ctx_cta ? lsec : lse;
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)bh * N + (dst_ok ? orig : 0)) * D);
+        uint4* dst = reinterpret_cast<uint4*>((ctx_cta ? outc : out) + orow * D);
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
@@ -514,7 +553,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
             }
           }
         }
-        if (lse != nullptr && dst_ok) lse[(size_t)bh * N + orig] = (m_ref + log2f(l)) * 0.6931471805599453f;
+        if (lse_out != nullptr && dst_ok) lse_out[orow] = (m_ref + log2f(l)) * 0.6931471805599453f;
       }
     }
   } else if (warp == 8 || warp == 9) {
@@ -522,12 +561,15 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
     const int s = warp - 8;
     if (lane == 0 && T[s] > 0) {
       const int a0 = 2 * (SLOTS * blockIdx.x + s);
+      const int crow0 = (SLOTS * ((int)blockIdx.x - nvid) + s) * ROWS;   // context CTAs
       mbar_arrive_tx(q_full(s), L::Q_BYTES);
 #pragma unroll
-      for (int a = 0; a < L::KATOMS; ++a)
-        tma_load_2d(sQ(s) + a * L::Q_ATOM, &maps.q, 64 * a, bh * N + a0 * BLK, q_full(s));
+      for (int a = 0; a < L::KATOMS; ++a) {
+        if (!ctx_cta) tma_load_2d(sQ(s) + a * L::Q_ATOM, &maps.q, 64 * a, bh * N + a0 * BLK, q_full(s));
+        else tma_load_2d(sQ(s) + a * L::Q_ATOM, &maps.qc, 64 * a, bh * C + crow0, q_full(s));
+      }
       const uint32_t* um = unionm[s];
-      int cur = next_block(um, 0, nwords);
+      int cur = ctx_cta ? 0 : next_block(um, 0, nwords);
       int ik = 0, iv = 0;
       for (int j = 0; j < T[s]; ++j) {
         const int st = j % STAGES;
@@ -535,14 +577,20 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
         const CUtensorMap *mk, *mv;
         int row;
         if (j < TE[s]) {
-          row = bh * N + cur * BLK;
-          cur = next_block(um, cur + 1, nwords);
+          // union block (video pair) or every block in turn (context chunk)
+          const int b = ctx_cta ? j : cur;
+          row = bh * N + b * BLK;
+          if (!ctx_cta) cur = next_block(um, cur + 1, nwords);
           mk = &maps.k;
           mv = &maps.v;
-        } else {
+        } else if (j < TX[s]) {
           row = bh * nb_pad + (j - TE[s]) * KEYS;
           mk = &maps.kt;
           mv = &maps.vt;
+        } else {
+          row = bh * C + (j - TX[s]) * KEYS;
+          mk = &maps.kc;
+          mv = &maps.vc;
         }
         // K_j once S_{j-STAGES} has read the stage
         if (j >= STAGES && !mbar_wait(k_empty(s, st), ph, status)) {
@@ -692,7 +740,7 @@ static bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, int d, int 
 
 template <int D>
 static cudaError_t run(const Plan& pl, const int32_t* perm, const int32_t* sel, uint16_t* out, float* lse,
-                       void* ws, int* status, cudaStream_t s) {
+                       void* ws, int* status, cudaStream_t s, const JointContext* ctx) {
   using Lay = Layout<D>;
   Maps maps;
   const uint64_t rows = (uint64_t)pl.BH * pl.N, srows = (uint64_t)pl.BH * pl.nb_pad;
@@ -703,22 +751,36 @@ static cudaError_t run(const Plan& pl, const int32_t* perm, const int32_t* sel, 
       !make_map(&maps.kt, ws_at<void>(ws, pl.off_kt), srows, D, 64) ||
       !make_map(&maps.vt, ws_at<void>(ws, pl.off_vt), srows, D, 64))
     return cudaErrorInvalidValue;
+  const int C = ctx ? ctx->C : 0;
+  if (C > 0) {
+    const uint64_t crows = (uint64_t)pl.BH * C;
+    if (!make_map(&maps.qc, ctx->qc, crows, D, ROWS) || !make_map(&maps.kc, ctx->kc, crows, D, 64) ||
+        !make_map(&maps.vc, ctx->vc, crows, D, 64))
+      return cudaErrorInvalidValue;
+  } else {
+    maps.qc = maps.q;
+    maps.kc = maps.k;
+    maps.vc = maps.v;
+  }
   auto kern = attn_tc_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
   if (e != cudaSuccess) return e;
   const int npairs = (pl.nb + 1) / 2;
+  const int nvid = (npairs + SLOTS - 1) / SLOTS;
+  const int nctx = C > 0 ? ((C + ROWS - 1) / ROWS + SLOTS - 1) / SLOTS : 0;   // context query chunks, two per CTA
   const float* ttab = pl.tail == SPARK_TAIL_BLOCK ? ws_at<float>(ws, pl.off_tail) : nullptr;
-  kern<<<dim3((npairs + SLOTS - 1) / SLOTS, pl.BH), THREADS, Lay::SMEM, s>>>(maps, ws_at<float>(ws, pl.off_beta), ttab, perm, sel,
-                                                                 pl.N, pl.nb, pl.nb_pad, pl.ksel, out, lse, status);
+  kern<<<dim3(nvid + nctx, pl.BH), THREADS, Lay::SMEM, s>>>(
+      maps, ws_at<float>(ws, pl.off_beta), ttab, perm, sel, pl.N, pl.nb, pl.nb_pad, pl.ksel, out, lse, C, nvid,
+      ctx ? ctx->outc : nullptr, ctx ? ctx->lsec : nullptr, status);
   return cudaGetLastError();
 }
 
 }  // namespace tc
 
 cudaError_t launch_attn_tc(const Plan& pl, const int32_t* perm, const int32_t* sel, uint16_t* out, float* lse,
-                           void* ws, int* status, cudaStream_t s) {
-  if (pl.d == 128) return tc::run<128>(pl, perm, sel, out, lse, ws, status, s);
-  return tc::run<64>(pl, perm, sel, out, lse, ws, status, s);
+                           void* ws, int* status, cudaStream_t s, const JointContext* ctx) {
+  if (pl.d == 128) return tc::run<128>(pl, perm, sel, out, lse, ws, status, s, ctx);
+  return tc::run<64>(pl, perm, sel, out, lse, ws, status, s, ctx);
 }
 
 }  // namespace spark

@@ -67,7 +67,18 @@ cudaError_t launch_positional(const Plan& pl, int F, int Hl, int Wl, int32_t* pe
 cudaError_t launch_select(const Plan& pl, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                           const int32_t* perm, const double* qmean, int32_t* sel, int summary,
                           void* ws, int* status, cudaStream_t s);
+// Context segment of joint attention: qc, kc, vc [BH, C, d] bf16 (C >= 1);
+// outc [BH, C, d] bf16, lsec [BH, C] float32 or null.
+struct JointContext {
+  const void* qc;
+  const void* kc;
+  const void* vc;
+  int C;
+  uint16_t* outc;
+  float* lsec;
+};
 cudaError_t launch_attn_tc(const Plan& pl, const int32_t* perm, const int32_t* sel, uint16_t* out,
-                           float* lse, void* ws, int* status, cudaStream_t s);
+                           float* lse, void* ws, int* status, cudaStream_t s,
+                           const JointContext* ctx = nullptr);
 
 }  // namespace spark

@@ -281,6 +281,61 @@ spark_status spark_attn_fwd(const spark_params* p, const int32_t* perm, const in
   return cuda_status(launch_attn_tc(pl, perm, sel, (uint16_t*)out, lse, ws, status_ptr(), stream));
 }
 
+static spark_status check_context(const spark_params* p, const void* qc, const void* kc, const void* vc,
+                                  int32_t C, const void* outc) {
+  if (C < 1 || !qc || !kc || !vc || !outc) return SPARK_ERR_INVALID_ARG;
+  if (!aligned16(qc) || !aligned16(kc) || !aligned16(vc) || !aligned16(outc)) return SPARK_ERR_INVALID_ARG;
+  if ((long)p->B * p->H * C > (long)INT32_MAX / 2) return SPARK_ERR_UNSUPPORTED;
+  return SPARK_OK;
+}
+
+spark_status spark_attn_fwd_joint(const spark_params* p, const int32_t* perm, const int32_t* sel,
+                                  const void* qc, const void* kc, const void* vc, int32_t C, void* out,
+                                  float* lse, void* outc, float* lsec, void* ws, size_t ws_bytes,
+                                  cudaStream_t stream) {
+  const spark_status v = validate(p);
+  if (v != SPARK_OK) return v;
+  Plan pl;
+  make_plan(p, &pl);
+  if (!perm || !sel || !out || !aligned16(out)) return SPARK_ERR_INVALID_ARG;
+  const spark_status c = check_context(p, qc, kc, vc, C, outc);
+  if (c != SPARK_OK) return c;
+  const spark_status w = check_ws(pl, ws, ws_bytes);
+  if (w != SPARK_OK) return w;
+  const JointContext ctx{qc, kc, vc, C, (uint16_t*)outc, lsec};
+  return cuda_status(launch_attn_tc(pl, perm, sel, (uint16_t*)out, lse, ws, status_ptr(), stream, &ctx));
+}
+
+spark_status spark_forward_joint(const spark_params* p, const void* q, const void* k, const void* v,
+                                 const void* qc, const void* kc, const void* vc, int32_t C, void* out,
+                                 float* lse, void* outc, float* lsec, void* ws, size_t ws_bytes,
+                                 cudaStream_t stream) {
+  const spark_status vs = validate(p);
+  if (vs != SPARK_OK) return vs;
+  Plan pl;
+  make_plan(p, &pl);
+  if (!q || !k || !v || !out) return SPARK_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SPARK_ERR_INVALID_ARG;
+  const spark_status c = check_context(p, qc, kc, vc, C, outc);
+  if (c != SPARK_OK) return c;
+  const spark_status w = check_ws(pl, ws, ws_bytes);
+  if (w != SPARK_OK) return w;
+  double* MQ = ws_at<double>(ws, pl.off_MQ);
+  double* MK = ws_at<double>(ws, pl.off_MK);
+  double* qmean = ws_at<double>(ws, pl.off_qmean);
+  int32_t* perm = ws_at<int32_t>(ws, pl.off_perm);
+  int32_t* sel = ws_at<int32_t>(ws, pl.off_sel);
+  cudaError_t e = launch_moments(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, ws, stream);
+  if (e != cudaSuccess) return SPARK_ERR_CUDA;
+  e = reblock_layout(pl, q, k, MQ, MK, perm, ws, stream);
+  if (e != cudaSuccess) return SPARK_ERR_CUDA;
+  e = launch_select(pl, (const uint16_t*)q, (const uint16_t*)k, (const uint16_t*)v, perm, qmean, sel,
+                    p->summary, ws, status_ptr(), stream);
+  if (e != cudaSuccess) return SPARK_ERR_CUDA;
+  const JointContext ctx{qc, kc, vc, C, (uint16_t*)outc, lsec};
+  return cuda_status(launch_attn_tc(pl, perm, sel, (uint16_t*)out, lse, ws, status_ptr(), stream, &ctx));
+}
+
 spark_status spark_forward(const spark_params* p, const void* q, const void* k, const void* v,
                            void* out, float* lse, int32_t* perm_out, int32_t* sel_out, void* ws,
                            size_t ws_bytes, cudaStream_t stream) {

@@ -203,6 +203,31 @@ spark_status spark_attn_fwd(const spark_params* p, const int32_t* perm, const in
                             void* out, float* lse, void* ws, size_t ws_bytes,
                             cudaStream_t stream);
 
+/* Joint attention with an exact context segment (the video pass joined with
+ * C text / audio / conditioning tokens, as in the model's joint attention
+ * layers; "Spark-H3" news post, model section; reading: context tokens take
+ * no part in moments, partition, selection or summaries). Video query i gets,
+ * in its one softmax, its exact and compressed terms as in spark_attn_fwd
+ * plus every context key j (logit q_i.kc_j/sqrt(d), value vc_j); context
+ * query c attends densely to all N video keys and all C context keys.
+ *   perm, sel       : as for spark_attn_fwd (spark_select ran on this ws)
+ *   qc, kc, vc      : [B,H,C,d] bf16 device, C >= 1, 16-byte aligned
+ *   out, lse        : video rows, as for spark_attn_fwd
+ *   outc            : [B,H,C,d] bf16 device, written; lsec: [B,H,C] f32 or NULL
+ * One kernel launch: video query pairs and context query chunks of 128
+ * share the grid. */
+spark_status spark_attn_fwd_joint(const spark_params* p, const int32_t* perm, const int32_t* sel,
+                                  const void* qc, const void* kc, const void* vc, int32_t C, void* out,
+                                  float* lse, void* outc, float* lsec, void* ws, size_t ws_bytes,
+                                  cudaStream_t stream);
+
+/* Steps 1-3 on the video tokens, then spark_attn_fwd_joint (perm and sel
+ * stay in ws). */
+spark_status spark_forward_joint(const spark_params* p, const void* q, const void* k, const void* v,
+                                 const void* qc, const void* kc, const void* vc, int32_t C, void* out,
+                                 float* lse, void* outc, float* lsec, void* ws, size_t ws_bytes,
+                                 cudaStream_t stream);
+
 /* The whole pass (steps 1-4) for device tensors. perm_out / sel_out are
  * optional device outputs (NULL: kept in ws). */
 spark_status spark_forward(const spark_params* p, const void* q, const void* k, const void* v,

@@ -205,6 +205,47 @@ def test_separate_layout_forward_matches_stages():
         check_head(r, 0, h, layout="separate")
 
 
+@pytest.mark.parametrize("C", [100, 320])
+def test_joint_attention_context_segment(C):
+    """Joint attention: video rows with the context keys as exact terms, and
+    context rows dense over both segments (C not a multiple of 64 or 128:
+    ragged context tiles and a partial last context chunk)."""
+    import torch
+    from spark_gen import f32_to_bf16_bits
+    w = tiny_workload("joint", 2, (2, 16, 64), 128, 0.25, seed_index=900)
+    q, k, v = make_inputs(w)
+    B, H, N, d = q.shape
+    rng = np.random.default_rng(4242 + C)
+    ctx = [f32_to_bf16_bits((rng.standard_normal((B, H, C, d)) * s).astype(np.float32)) for s in (0.8, 0.8, 1.0)]
+    p = spark.params(B, H, N, d, w.ratio)
+    ws = spark.alloc_workspace(p)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    MQ, MK, qmean = spark.moments(p, qd, kd, ws)
+    perm = spark.reblock(p, qd, kd, MQ, MK, ws)
+    sel = spark.select(p, qd, kd, vd, perm, qmean, ws)
+    qc, kc, vc = (to_dev(c) for c in ctx)
+    out, outc, lse, lsec = spark.attn_fwd_joint(p, perm, sel, qc, kc, vc, ws, return_lse=True)
+    assert spark.get_status() == 0
+    out, outc = bf16_to_f64(out), bf16_to_f64(outc)
+    lse, lsec = lse.cpu().numpy(), lsec.cpu().numpy()
+    perm_h, sel_h = perm.cpu().numpy(), sel.cpu().numpy()
+    for h in range(H):
+        qh, kh, vh = (bf16_bits_to_f64(x[0, h]) for x in (q, k, v))
+        ch = [bf16_bits_to_f64(c[0, h]) for c in ctx]
+        pm = perm_h[0, h].astype(np.int64)
+        kt, vt, beta = so.summaries(kh, vh, pm, so.anchor(qh))
+        ref, ref_lse, refc, refc_lse = so.joint_attention(qh, kh, vh, pm, sel_h[0, h].astype(np.int64), kt, vt, beta,
+                                                          *ch)
+        for got, want, gl, wl in ((out[0, h], ref, lse[0, h], ref_lse), (outc[0, h], refc, lsec[0, h], refc_lse)):
+            e = parity.out_errors(got, want)
+            assert e["max_rel_to_bound"] <= 1.0, e
+            assert e["max_abs"] <= 2 ** -7 * np.abs(want).max() + 4e-3 * e["ref_rms"], e
+            assert np.abs(gl - wl).max() <= 1e-3 * (1 + np.abs(wl).max())
+    # the whole pass with the context segment gives the same rows
+    o2, oc2 = spark.forward_joint(p, qd, kd, vd, qc, kc, vc, ws=ws)
+    assert np.array_equal(bf16_to_f64(o2), out) and np.array_equal(bf16_to_f64(oc2), outc)
+
+
 def test_topk_blocks_and_batch():
     w = tiny_workload("tb", 3, (2, 16, 32), 128, 0.2, seed_index=500, B=2)
     r = run_stages(w, topk_blocks=5)

@@ -241,7 +241,9 @@ struct Maps {
   CUtensorMap qc, kc, vc;      // context segment (joint attention); copies of q, k, v when absent
 };
 
-template <int D>
+// EXT: the block tail granularity or a context segment may be present (an
+// instance without them carries none of their per-tile branches).
+template <int D, bool EXT>
 __global__ void __launch_bounds__(THREADS, 1)
 attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta, const float* __restrict__ ttab,
                const int32_t* __restrict__ perm, const int32_t* __restrict__ sel, int N, int nb,
@@ -338,10 +340,10 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
   // Tiles of a unit. Video pairs (blockIdx.x < nvid): the union blocks, then
   // the summaries, then the context keys (joint attention, C > 0). Context
   // query chunks (blockIdx.x >= nvid): every video block, then the context keys.
-  const bool ctx_cta = (int)blockIdx.x >= nvid;
+  const bool ctx_cta = EXT && (int)blockIdx.x >= nvid;
   int TE[SLOTS], T[SLOTS], TX[SLOTS];                  // exact (or dense) tiles, all tiles, first context tile
   const int TS = (nb + KEYS - 1) / KEYS;               // summary tiles
-  const int TC = (C + KEYS - 1) / KEYS;                // context tiles
+  const int TC = EXT ? (C + KEYS - 1) / KEYS : 0;     // context tiles
 #pragma unroll
   for (int s = 0; s < SLOTS; ++s) {
     if (!ctx_cta) {
@@ -384,18 +386,18 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
         const uint32_t sc = tbase + 64u * (uint32_t)(j & 1);   // this tile's S (and P) columns
         // the tile's block (or summary range) and this row's mask, before the wait;
         // kind 0: exact keys, 1: summaries, 2: context keys (per-column masks for 1, 2)
-        const int kind = j < TEs ? 0 : (j < TXs ? 1 : 2);
+        const int kind = j < TEs ? 0 : ((!EXT || j < TXs) ? 1 : 2);
         const bool comp = kind != 0;
         bool take;
         uint32_t ex0 = ~0u, ex1 = ~0u;
         int c0 = 0;
-        if (kind == 0 && ctx_cta) {
+        if (EXT && kind == 0 && ctx_cta) {
           take = row_valid;                              // dense: every video block
         } else if (kind == 0) {
           const int b = cur;
           cur = next_block(um, b + 1, nwords);
           take = row_valid && ((mymask[b >> 5] >> (b & 31)) & 1u);
-        } else if (kind == 2) {
+        } else if (EXT && kind == 2) {
           const int vc = C - (j - TXs) * KEYS;           // valid context keys in this tile (>= 1)
           take = row_valid;
           ex0 = vc >= 32 ? 0u : (~0u << vc);
@@ -435,8 +437,8 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
             // x = s / sqrt(d) + beta (log2 units), -inf where the row selected the block;
             // block tail granularity: the query block's precomputed logit row instead;
             // context keys: s / sqrt(d), -inf past the end of the segment
-            const bool tab = kind == 1 && ttab != nullptr;
-            const float* brow = kind == 2 ? nullptr
+            const bool tab = EXT && kind == 1 && ttab != nullptr;
+            const float* brow = (EXT && kind == 2) ? nullptr
                                 : tab    ? ttab + ((size_t)bh * nb + a0 + qh) * nb_pad + c0
                                          : beta + (size_t)bh * nb_pad + c0;
 #pragma unroll
@@ -583,7 +585,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
           if (!ctx_cta) cur = next_block(um, cur + 1, nwords);
           mk = &maps.k;
           mv = &maps.v;
-        } else if (j < TX[s]) {
+        } else if (!EXT || j < TX[s]) {
           row = bh * nb_pad + (j - TE[s]) * KEYS;
           mk = &maps.kt;
           mv = &maps.vt;
@@ -762,7 +764,8 @@ static cudaError_t run(const Plan& pl, const int32_t* perm, const int32_t* sel, 
     maps.kc = maps.k;
     maps.vc = maps.v;
   }
-  auto kern = attn_tc_kernel<D>;
+  const bool ext = pl.tail == SPARK_TAIL_BLOCK || (ctx != nullptr && ctx->C > 0);
+  auto kern = ext ? attn_tc_kernel<D, true> : attn_tc_kernel<D, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
   if (e != cudaSuccess) return e;
   const int npairs = (pl.nb + 1) / 2;

@@ -99,9 +99,10 @@ def normalized_whitened(x, L):
     return round_bf16(out)
 
 
-def split_direction(U):
+def split_direction(U, iters=POWER_ITERS):
     """R6: top principal direction of the group's centered covariance by a
-    fixed number of power iterations from the all-ones direction.
+    fixed number of power iterations from the all-ones direction (iters; the
+    "Lite" reblock takes fewer, reading R18).
 
     U: [n, d] normalised whitened vectors of one group. Returns (v, mu, p)
     where p_i = v . (U_i - mu) is each token's projection."""
@@ -110,7 +111,7 @@ def split_direction(U):
     C = U - mu
     S = C.T @ C / n
     v = np.full(d, 1.0 / math.sqrt(d))
-    for _ in range(POWER_ITERS):
+    for _ in range(iters):
         w = S @ v
         nw = math.sqrt(float(w @ w))
         if nw == 0.0:
@@ -121,7 +122,7 @@ def split_direction(U):
     return v, mu, p
 
 
-def split_group(U, ids):
+def split_group(U, ids, iters=POWER_ITERS):
     """R6: capacity-constrained bisection of one group of g = n/64 blocks
     ([P1] "the hierarchical partitioner keeps splitting groups until every
     leaf reaches the target block size"; [P2] "capacity-constrained tree
@@ -134,7 +135,7 @@ def split_group(U, ids):
     ids = np.asarray(ids)
     n = ids.shape[0]
     g = n // BLOCK
-    v, mu, p = split_direction(U)
+    v, mu, p = split_direction(U, iters)
     a = np.abs(p)
     top = ids[a == a.max()].min()
     if p[ids == top][0] < 0:
@@ -167,7 +168,7 @@ def tree_nodes(nb: int):
     return levels
 
 
-def reblock(x, M):
+def reblock(x, M, iters=POWER_ITERS):
     """a2 Reblock, R5-R8: partition tokens of one head into 64-token blocks.
 
     x: the side that is partitioned (queries for q_reuse_k), M: the opposite
@@ -183,7 +184,7 @@ def reblock(x, M):
     def rec(ids):
         if ids.shape[0] <= BLOCK:
             return [np.sort(ids)]
-        left, right, _ = split_group(U[ids], ids)
+        left, right, _ = split_group(U[ids], ids, iters)
         return rec(left) + rec(right)
 
     leaves = rec(np.arange(N))
@@ -414,7 +415,8 @@ def dense_attention(q, k, v):
 # whole forward pass of one head
 
 def forward_head(q, k, v, ratio=0.2, topk_blocks=0, layout="q_reuse_k",
-                 summary="reweight", perm=None, rows=None, tail="query", perm_k=None):
+                 summary="reweight", perm=None, rows=None, tail="query", perm_k=None,
+                 power_iters=POWER_ITERS):
     """Every intermediate of the forward pass for one (batch item, head).
 
     layout: "q_reuse_k" partitions the queries under M_K and reuses that
@@ -430,11 +432,11 @@ def forward_head(q, k, v, ratio=0.2, topk_blocks=0, layout="q_reuse_k",
     nb = N // BLOCK
     MQ, MK, qbar = second_moment(q), second_moment(k), anchor(q)
     if layout == "q_reuse_k":
-        perm = reblock(q, MK)
+        perm = reblock(q, MK, power_iters)
     elif layout == "k_reuse_q":
-        perm = reblock(k, MQ)
+        perm = reblock(k, MQ, power_iters)
     elif layout == "separate":
-        perm, perm_k = reblock(q, MK), reblock(k, MQ)
+        perm, perm_k = reblock(q, MK, power_iters), reblock(k, MQ, power_iters)
     elif layout != "given":
         raise ValueError(layout)
     perm = np.asarray(perm)

@@ -37,7 +37,7 @@ def check_perm_structure(perm, N):
     assert np.all(np.diff(blocks, axis=1) > 0)
 
 
-def certify_perm(x, M, perm, tau=TAU_P, U=None):
+def certify_perm(x, M, perm, tau=TAU_P, U=None, iters=so.POWER_ITERS):
     """Replay the oracle's splits on the CUDA path's sets.
 
     x: [N, d] float64 (partitioned side), M: float64 moment of the opposite
@@ -56,7 +56,7 @@ def certify_perm(x, M, perm, tau=TAU_P, U=None):
     for level in so.tree_nodes(nb):
         for first, g in level:
             ids = perm[64 * first:64 * (first + g)]
-            left, _, info = so.split_group(U[ids], ids)
+            left, _, info = so.split_group(U[ids], ids, iters)
             gl = set(perm[64 * first:64 * (first + g // 2)].tolist())
             ol = set(left.tolist())
             stats["nodes"] += 1

@@ -553,6 +553,31 @@ def test_joint_attention_lse_merge():
     assert np.allclose(out, w * res["out"] + (1 - w) * o_ctx, rtol=1e-10, atol=1e-12)
 
 
+@pytest.mark.parametrize("iters", [1, 4, 16])
+def test_split_direction_is_normalised_matrix_power(iters):
+    """With T power steps the direction is S^T 1 / |S^T 1| (one matrix power,
+    no per-step rescaling), for the Lite count as for the default."""
+    r = np.random.default_rng(77)
+    U = bf16(r.standard_normal((256, 12)))
+    v, mu, p = so.split_direction(U, iters)
+    C = U - U.mean(axis=0)
+    S = C.T @ C / len(U)
+    w = np.linalg.matrix_power(S, iters) @ np.ones(12)
+    assert np.allclose(v, w / np.linalg.norm(w), rtol=1e-10, atol=1e-12)
+    assert np.allclose(p, C @ v, rtol=1e-12, atol=1e-12)
+
+
+def test_lite_split_equals_full_split_for_rank_one_groups():
+    """A group whose centred vectors share one direction: one power step
+    already finds it, so 4 and 16 steps give the same partition."""
+    r = np.random.default_rng(78)
+    d = 16
+    u = r.standard_normal(d)
+    x = np.outer(r.standard_normal(512), u) + 1e-3      # rank one after centring
+    M = np.eye(d)
+    assert np.array_equal(so.reblock(x, M, 4), so.reblock(x, M, 16))
+
+
 # ------------------------------------------------------------------ statistics
 
 def test_mass_recall_is_100_at_density_one():

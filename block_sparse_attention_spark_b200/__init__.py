@@ -40,7 +40,8 @@ class Params(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("topk_ratio", ctypes.c_double),
                 ("topk_blocks", ctypes.c_int32), ("layout", ctypes.c_int32),
-                ("summary", ctypes.c_int32), ("tail", ctypes.c_int32)]
+                ("summary", ctypes.c_int32), ("tail", ctypes.c_int32),
+                ("power_iters", ctypes.c_int32)]
 
     def __repr__(self):
         return (f"Params(B={self.B}, H={self.H}, N={self.N}, d={self.d}, "
@@ -99,9 +100,9 @@ def _check(code: int, where: str):
 
 
 def params(B, H, N, d, topk_ratio=0.2, topk_blocks=0, layout="q_reuse_k",
-           summary="reweight", tail="query") -> Params:
+           summary="reweight", tail="query", power_iters=0) -> Params:
     return Params(B, H, N, d, float(topk_ratio), int(topk_blocks), LAYOUTS[layout],
-                  SUMMARIES[summary], TAILS[tail])
+                  SUMMARIES[summary], TAILS[tail], int(power_iters))
 
 
 def validate(p: Params) -> int:

@@ -20,6 +20,7 @@ struct Plan {
   int tail = 0;                   // SPARK_TAIL_*
   int layout = 0;                 // SPARK_LAYOUT_*
   int nperm = 1;                  // permutations per pass (2 for SPARK_LAYOUT_SEPARATE)
+  int power_iters = 16;           // power iterations per split
   int nlevels = 0;
   std::vector<int> level_count;   // nodes that split at each level
   std::vector<int> level_off;     // offset of each level in the node table

@@ -33,7 +33,6 @@
 namespace spark {
 
 constexpr double REG_EPS = 1e-6;   // relative diagonal jitter before the Cholesky factor
-constexpr int POWER_ITERS = 16;
 constexpr int NORM_EVERY = 4;      // power-iteration steps between rescalings of v
 
 // ------------------------------------------------------------------ whitening factor
@@ -333,7 +332,7 @@ __device__ uint64_t radix_select_u64(int n, int rank, int nbits, GetKey getkey, 
   return prefix;
 }
 
-// Power iteration v <- S v / |S v| (float64), POWER_ITERS steps from the
+// Power iteration v <- S v / |S v| (float64), iters steps (16 by default) from the
 // all-ones direction; S is a D x D row-major matrix in shared memory (the
 // buffer is reused as scratch afterwards). Thread (rg, cg) holds rows
 // rg*RPT.. and columns cg*CPT.. of S in registers and its own copy of v on
@@ -341,10 +340,10 @@ __device__ uint64_t radix_select_u64(int n, int rank, int nbits, GetKey getkey, 
 // slot of padding per column group: conflict-free reads) and |z|^2 through
 // per-warp partials, so a step needs one barrier. v is rescaled to unit
 // length every NORM_EVERY steps and after the last one (the direction after
-// POWER_ITERS steps is the same as with a rescale at every step). Writes v
+// iters steps is the same as with a rescale at every step). Writes v
 // to vs.
 template <int D>
-__device__ void power_iterate(double* acc64, double* vs) {
+__device__ void power_iterate(double* acc64, double* vs, int iters) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int RPT = D / 32, CPT = D / 8, ZP = D + D / CPT;
   const int rg = tid >> 3, cg = tid & 7;
@@ -364,9 +363,9 @@ __device__ void power_iterate(double* acc64, double* vs) {
   // v <- S v, scaled to unit length every NORM_EVERY steps and at the end:
   // scaling does not change the direction, and with |S| <= 1 (a covariance
   // of unit vectors) NORM_EVERY unscaled steps stay far from underflow
-  for (int iter = 0; iter < POWER_ITERS; ++iter) {
+  for (int iter = 0; iter < iters; ++iter) {
     double* z = zb + (iter & 1) * ZP;
-    const bool norm_step = (iter % NORM_EVERY) == NORM_EVERY - 1 || iter == POWER_ITERS - 1;
+    const bool norm_step = (iter % NORM_EVERY) == NORM_EVERY - 1 || iter == iters - 1;
     double sq = 0.0;
     double zr[RPT];
 #pragma unroll
@@ -574,7 +573,7 @@ template <int D>
 __global__ void __launch_bounds__(256, 1)
 big_solve_kernel(const int2* __restrict__ nodes, int nnodes, int chunks, const double* __restrict__ part,
                  double* __restrict__ info, int derive, const double* __restrict__ gpar, int npar,
-                 double* __restrict__ gout) {
+                 double* __restrict__ gout, int iters) {
   // The group's Gram sum G = sum u u^T and column sums: from its own chunk
   // partials, or (derive) a right child's as its parent's minus its left
   // sibling's, the parent's having been stored one level up. Stored again
@@ -624,7 +623,7 @@ big_solve_kernel(const int2* __restrict__ nodes, int nnodes, int chunks, const d
     }
   }
   __syncthreads();
-  power_iterate<D>(Smat, vs);
+  power_iterate<D>(Smat, vs, iters);
   double* out = info + (size_t)(bh * nnodes + k) * (D + 1);
   if (tid < D) out[tid] = vs[tid];
   if (tid == 0) {
@@ -780,7 +779,7 @@ template <int D>
 __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* ids, uint16_t* loc,
                               uint16_t* stok, double* zp, double* mus, double* vs, double* red_d, int* red_i,
                               double* sh_sgn, int* hist, int* sh_sel, unsigned long long* sh_key,
-                              int* warp_tot, int* status, int s0, int nn) {
+                              int* warp_tot, int* status, int s0, int nn, int iters) {
   using G = Gram<D>;
   using SM = SubSmem<D>;
   constexpr int RS = SM::RS;
@@ -846,9 +845,9 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
 #pragma unroll
   for (int j = 0; j < G::NT * 2; ++j) vl[j] = 1.0 / sqrt((double)D);
   bool zero_dir = false;
-  for (int iter = 0; iter < POWER_ITERS; ++iter) {
+  for (int iter = 0; iter < iters; ++iter) {
     double* z = zp + (iter & 1) * 2 * D;        // [wn][row]: the two column halves' partial sums
-    const bool norm_step = (iter % NORM_EVERY) == NORM_EVERY - 1 || iter == POWER_ITERS - 1;
+    const bool norm_step = (iter % NORM_EVERY) == NORM_EVERY - 1 || iter == iters - 1;
     double zr[G::MT][2];
 #pragma unroll
     for (int mt = 0; mt < G::MT; ++mt) { zr[mt][0] = 0.0; zr[mt][1] = 0.0; }
@@ -974,7 +973,7 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
 template <int D>
 __global__ void __launch_bounds__(256, 1)
 subtree_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restrict__ nodes,
-               int32_t* __restrict__ idx, int* status) {
+               int32_t* __restrict__ idx, int* status, int iters) {
   using SM = SubSmem<D>;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   uint16_t* rows = reinterpret_cast<uint16_t*>(smem_raw + SM::off_rows);
@@ -1021,7 +1020,7 @@ subtree_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restrict_
       const int2 nd = lvl[cur][i];
       if (nd.y >= 2)
         subtree_split<D>(rows, pv, ids, loc, stok, zp, mus, vs, red_d, red_i, &sh_sgn, hist, sh_sel, &sh_key,
-                         warp_tot, status, nd.x * BLK, nd.y * BLK);
+                         warp_tot, status, nd.x * BLK, nd.y * BLK, iters);
     }
     if (tid == 0) {
       int m = 0;
@@ -1126,7 +1125,7 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
   for (int lv = 0; lv < pl.nlevels; ++lv) {
     if (pl.level_maxg[lv] <= SUB_BLOCKS) {   // this level and everything below it, in shared memory
       subtree_kernel<D><<<dim3(pl.level_count[lv], pl.BH), 256, smem_t, s>>>(uhat, pl.N, nodes + pl.level_off[lv],
-                                                                            idx, status);
+                                                                            idx, status, pl.power_iters);
       break;
     }
     // each group spread over chunk CTAs; a right child's Gram derived from its parent's
@@ -1138,7 +1137,8 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
     double* gout = pl.level_store[lv] ? gstore[lv & 1] : nullptr;
     big_gram_kernel<D><<<dim3(ch, cnt / kstep, pl.BH), 256, smem_s, s>>>(uhat, pl.N, nd, cnt, ch, kstep, idx, bpart);
     big_solve_kernel<D><<<dim3(cnt, pl.BH), 256, smem_solve, s>>>(nd, cnt, ch, bpart, binfo, derive, gpar,
-                                                                   derive ? pl.level_count[lv - 1] : 0, gout);
+                                                                   derive ? pl.level_count[lv - 1] : 0, gout,
+                                                                   pl.power_iters);
     big_project_kernel<D><<<dim3(ch, cnt, pl.BH), 256, smem_proj, s>>>(uhat, pl.N, nd, cnt, ch, idx, binfo, pval,
                                                                       pidx, bcand);
     big_select_kernel<<<dim3(cnt, pl.BH), 256, 0, s>>>(pl.N, nd, cnt, ch, bcand, idx, pval, pidx, status);

@@ -35,6 +35,7 @@ static spark_status validate(const spark_params* p) {
     return SPARK_ERR_INVALID_ARG;
   if (p->summary != SPARK_SUMMARY_REWEIGHT && p->summary != SPARK_SUMMARY_MEANPOOL) return SPARK_ERR_INVALID_ARG;
   if (p->tail != SPARK_TAIL_QUERY && p->tail != SPARK_TAIL_BLOCK) return SPARK_ERR_INVALID_ARG;
+  if (p->power_iters < 0 || p->power_iters > 64) return SPARK_ERR_INVALID_ARG;
   if (p->N % SPARK_BLOCK != 0) return SPARK_ERR_UNSUPPORTED;
   if (p->d != 64 && p->d != 128) return SPARK_ERR_UNSUPPORTED;
   const long nb = p->N / SPARK_BLOCK;
@@ -54,6 +55,7 @@ bool make_plan(const spark_params* p, Plan* pl) {
   P.BH = p->B * p->H;
   P.tail = p->tail;
   P.layout = p->layout;
+  P.power_iters = p->power_iters > 0 ? p->power_iters : 16;
   P.nperm = p->layout == SPARK_LAYOUT_SEPARATE ? 2 : 1;
   P.nb = p->N / SPARK_BLOCK;
   P.ksel = num_selected_impl(P.nb, p->topk_ratio, p->topk_blocks);

@@ -96,6 +96,9 @@ typedef struct {
   int32_t layout;              /* SPARK_LAYOUT_* */
   int32_t summary;             /* SPARK_SUMMARY_* */
   int32_t tail;                /* SPARK_TAIL_* */
+  int32_t power_iters;         /* power iterations per split: 0 = 16 (default); the "Lite"
+                                  reblock ("Spark-H3" news post: halved reblock latency, method
+                                  not given) takes fewer, e.g. 4; 1..64 accepted */
 } spark_params;
 
 /* Checks a parameter block. SPARK_OK or the error the other calls would give. */

@@ -35,8 +35,17 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_params_struct_layout():
-    assert ctypes.sizeof(spark.Params) == 40
+    # B, H, N, d, topk_ratio (8-aligned), topk_blocks, layout, summary, tail, power_iters, padding
+    assert ctypes.sizeof(spark.Params) == 48
     assert spark.Params.topk_ratio.offset == 16
+    assert spark.Params.power_iters.offset == 40
+
+
+def test_power_iters_range():
+    assert spark.validate(P(power_iters=4)) == 0
+    assert spark.validate(P(power_iters=64)) == 0
+    assert spark.validate(P(power_iters=65)) == 1
+    assert spark.validate(P(power_iters=-1)) == 1
 
 
 def P(**kw):

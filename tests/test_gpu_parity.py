@@ -27,11 +27,12 @@ def bf16_to_f64(t):
 
 
 def run_stages(w, ratio=None, layout="q_reuse_k", summary="reweight", topk_blocks=0, qkv=None,
-               perm=None, tail="query"):
+               perm=None, tail="query", power_iters=0):
     import torch
     q, k, v = qkv if qkv is not None else make_inputs(w)
     B, H, N, d = q.shape
-    p = spark.params(B, H, N, d, ratio if ratio is not None else w.ratio, topk_blocks, layout, summary, tail)
+    p = spark.params(B, H, N, d, ratio if ratio is not None else w.ratio, topk_blocks, layout, summary, tail,
+                     power_iters)
     ws = spark.alloc_workspace(p)
     qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
     MQ, MK, qmean = spark.moments(p, qd, kd, ws)
@@ -54,7 +55,7 @@ def run_stages(w, ratio=None, layout="q_reuse_k", summary="reweight", topk_block
 
 
 def check_head(r, b, h, layout="q_reuse_k", summary="reweight", rows=None, check_perm=True,
-               report=None, tail="query"):
+               report=None, tail="query", power_iters=so.POWER_ITERS):
     q = bf16_bits_to_f64(r["q"][b, h])
     k = bf16_bits_to_f64(r["k"][b, h])
     v = bf16_bits_to_f64(r["v"][b, h])
@@ -72,7 +73,7 @@ def check_head(r, b, h, layout="q_reuse_k", summary="reweight", rows=None, check
         if check_perm:
             # the workspace's u_hat is the key side's (the second reblock); the
             # query side is replayed with the oracle's own u_hat
-            st = parity.certify_perm(q, MK, perm)
+            st = parity.certify_perm(q, MK, perm, iters=power_iters)
             print("perm q", b, h, st)
             assert st["failures"] == 0, st
         xs, Ms = k, MQ
@@ -93,7 +94,7 @@ def check_head(r, b, h, layout="q_reuse_k", summary="reweight", rows=None, check
             ref_ulp = np.ldexp(1.0, np.frexp(np.abs(U[diff]))[1] - 8)
             dev = np.abs(r["uhat"][b, h][diff] - U[diff])
             assert np.all(dev <= np.maximum(ref_ulp, 4e-6)), dev.max()
-        st = parity.certify_perm(xs, Ms, perm_side, U=r["uhat"][b, h])
+        st = parity.certify_perm(xs, Ms, perm_side, U=r["uhat"][b, h], iters=power_iters)
         print("perm", b, h, st)
         assert st["failures"] == 0, st
         if report is not None:
@@ -244,6 +245,15 @@ def test_joint_attention_context_segment(C):
     # the whole pass with the context segment gives the same rows
     o2, oc2 = spark.forward_joint(p, qd, kd, vd, qc, kc, vc, ws=ws)
     assert np.array_equal(bf16_to_f64(o2), out) and np.array_equal(bf16_to_f64(oc2), outc)
+
+
+def test_lite_reblock_power_iters():
+    """The Lite reblock reading: 4 power iterations per split; every split is
+    replayed by the oracle with the same count."""
+    w = tiny_workload("lite", 2, (2, 16, 64), 128, 0.2, seed_index=1000)
+    r = run_stages(w, power_iters=4)
+    for h in range(2):
+        check_head(r, 0, h, power_iters=4)
 
 
 def test_topk_blocks_and_batch():

@@ -343,20 +343,33 @@ __device__ uint64_t radix_select_u64(int n, int rank, int nbits, GetKey getkey, 
 // iters steps is the same as with a rescale at every step). Writes v
 // to vs.
 template <int D>
+__device__ void power_iterate_regs(const double (&Sr)[D / 32][D / 8], double* zb, double* vs, int iters);
+
+template <int D>
 __device__ void power_iterate(double* acc64, double* vs, int iters) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  constexpr int RPT = D / 32, CPT = D / 8, ZP = D + D / CPT;
+  const int tid = threadIdx.x;
+  constexpr int RPT = D / 32, CPT = D / 8;
   const int rg = tid >> 3, cg = tid & 7;
   double Sr[RPT][CPT];
 #pragma unroll
   for (int i = 0; i < RPT; ++i)
 #pragma unroll
     for (int j = 0; j < CPT; ++j) Sr[i][j] = acc64[(rg * RPT + i) * D + cg * CPT + j];
+  __syncthreads();                           // S has been copied to registers: acc64 becomes the z buffers
+  power_iterate_regs<D>(Sr, acc64, vs, iters);
+}
+
+// The power iteration proper. Thread (rg, cg) = (tid / 8, tid % 8) holds rows
+// rg*RPT.. and columns cg*CPT.. of S in Sr; zb: shared scratch of at least
+// 2 * (D + D / CPT) + 16 doubles.
+template <int D>
+__device__ void power_iterate_regs(const double (&Sr)[D / 32][D / 8], double* zb, double* vs, int iters) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int RPT = D / 32, CPT = D / 8, ZP = D + D / CPT;
+  const int rg = tid >> 3, cg = tid & 7;
   double vloc[CPT];
 #pragma unroll
   for (int j = 0; j < CPT; ++j) vloc[j] = 1.0 / sqrt((double)D);
-  double* zb = acc64;                        // S has been copied to registers: reuse as z buffers
-  __syncthreads();
   auto zpad = [](int c) { return c + c / CPT; };
   bool zero_dir = false;
   double* nparts = zb + 2 * ZP;               // [2][8] per-warp partial |z|^2
@@ -578,9 +591,9 @@ big_solve_kernel(const int2* __restrict__ nodes, int nnodes, int chunks, const d
   // partials, or (derive) a right child's as its parent's minus its left
   // sibling's, the parent's having been stored one level up. Stored again
   // (gout) when the next level derives from this one.
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  double* Smat = reinterpret_cast<double*>(smem_raw);      // D x D
+  constexpr int RPT = D / 32, CPT = D / 8;
   __shared__ double mus[D], vs[D];
+  __shared__ double zbuf[2 * (D + D / CPT) + 16];
   const int tid = threadIdx.x, k = blockIdx.x, bh = blockIdx.y;
   const int2 node = nodes[k];
   const int n = node.y * BLK;
@@ -599,37 +612,39 @@ big_solve_kernel(const int2* __restrict__ nodes, int nnodes, int chunks, const d
     mus[tid] = t * invn;
   }
   __syncthreads();
-  // 8 elements per thread at a time, so that their loads are in flight together
-  for (int e0 = tid; e0 < D * D; e0 += 8 * blockDim.x) {
-    double t[8];
+  // each thread reads its own RPT x CPT block of G straight into the
+  // power iteration's register layout (all loads in flight together)
+  const int rg = tid >> 3, cg = tid & 7;
+  double Sr[RPT][CPT];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) t[u] = 0.0;
-    for (int c = 0; c < used; ++c) {
-      const double* pc = src + (size_t)c * (D * D + D);
+  for (int i = 0; i < RPT; ++i)
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int e = e0 + u * blockDim.x;
-        if (e < D * D) t[u] += pc[e];
-      }
-    }
+    for (int j = 0; j < CPT; ++j) Sr[i][j] = 0.0;
+  for (int c = 0; c < used; ++c) {
+    const double* pc = src + (size_t)c * (D * D + D);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int e = e0 + u * blockDim.x;
-      if (e < D * D) {
-        const double g = right ? par[e] - t[u] : t[u];
-        if (gsave) gsave[e] = g;
-        Smat[e] = g * invn - mus[e / D] * mus[e % D];
-      }
-    }
+    for (int i = 0; i < RPT; ++i)
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) Sr[i][j] += pc[(rg * RPT + i) * D + cg * CPT + j];
   }
-  __syncthreads();
-  power_iterate<D>(Smat, vs, iters);
+#pragma unroll
+  for (int i = 0; i < RPT; ++i)
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      const int row = rg * RPT + i, col = cg * CPT + j;
+      const double g = right ? par[row * D + col] - Sr[i][j] : Sr[i][j];
+      if (gsave) gsave[row * D + col] = g;
+      Sr[i][j] = g * invn - mus[row] * mus[col];
+    }
+  power_iterate_regs<D>(Sr, zbuf, vs, iters);
   double* out = info + (size_t)(bh * nnodes + k) * (D + 1);
   if (tid < D) out[tid] = vs[tid];
-  if (tid == 0) {
+  if (tid < 32) {
     double vmu = 0.0;
-    for (int j = 0; j < D; ++j) vmu = fma(vs[j], mus[j], vmu);
-    out[D] = vmu;
+    for (int j = tid; j < D; j += 32) vmu = fma(vs[j], mus[j], vmu);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) vmu += __shfl_xor_sync(0xffffffffu, vmu, o);
+    if (tid == 0) out[D] = vmu;
   }
 }
 
@@ -816,16 +831,34 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
     }
   }
   {
-    // column sums: thread covers column tid % D over tokens (tid / D) + k * (256 / D)
-    constexpr int RSTEP = 256 / D;
-    float c4[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int t = tid / D, k = 0; t < nn; t += RSTEP, ++k) c4[k & 3] += bf2f(rows[(size_t)lo[t] * RS + (tid % D)]);
-    double* cs = zp;   // scratch before the power iteration uses it
-    cs[tid] = (double)((c4[0] + c4[1]) + (c4[2] + c4[3]));
+    // column sums: thread = 8 columns (one 16-byte load per row) x every
+    // RG-th token; the row groups of a warp are folded by shuffles, the
+    // warps' float partials by one float64 pass
+    constexpr int CG = D / 8, RG = 256 / CG;
+    const int cg = tid % CG, rg = tid / CG;
+    float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int t = rg; t < nn; t += RG) {
+      const uint4 w = *reinterpret_cast<const uint4*>(rows + (size_t)lo[t] * RS + cg * 8);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        a8[2 * e] += bf_lo(ws[e]);
+        a8[2 * e + 1] += bf_hi(ws[e]);
+      }
+    }
+#pragma unroll
+    for (int o = CG; o < 32; o <<= 1)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) a8[e] += __shfl_xor_sync(0xffffffffu, a8[e], o);
+    float* cs = reinterpret_cast<float*>(zp);   // [8 warps][D] scratch before the power iteration uses it
+    if (lane < CG) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cs[warp * D + cg * 8 + e] = a8[e];
+    }
     __syncthreads();
     if (tid < D) {
       double t = 0.0;
-      for (int k = 0; k < RSTEP; ++k) t += cs[tid + k * D];
+      for (int w = 0; w < 8; ++w) t += (double)cs[w * D + tid];
       mus[tid] = t / (double)nn;
     }
   }
@@ -910,32 +943,48 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
     double vr[QD];
 #pragma unroll
     for (int j = 0; j < QD; ++j) vr[j] = vs[qd * QD + j];
-    double vmu = 0.0;
-#pragma unroll 8
-    for (int j = 0; j < D; ++j) vmu = fma(vs[j], mus[j], vmu);
-    for (int b0 = 0; b0 < nn; b0 += 64) {
-      const int t = b0 + tk;
-      const uint4* rr = reinterpret_cast<const uint4*>(rows + (size_t)lo[t] * RS + qd * QD);
-      double s4[4] = {0.0, 0.0, 0.0, 0.0};
+    double vmu = 0.0;                                   // v . mu, the same order in every warp
+    for (int j = lane; j < D; j += 32) vmu = fma(vs[j], mus[j], vmu);
 #pragma unroll
-      for (int c = 0; c < QD / 8; ++c) {
-        const uint4 w = rr[c];
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    for (int o = 16; o > 0; o >>= 1) vmu += __shfl_xor_sync(0xffffffffu, vmu, o);
+    // two tokens per thread and pass (independent float64 chains)
+    for (int b0 = 0; b0 < nn; b0 += 128) {
+      const bool two = b0 + 64 < nn;                  // nn is a multiple of 64: uniform
+      double sacc[2];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          s4[e] = fma(vr[8 * c + 2 * e], (double)bf_lo(ws[e]), s4[e]);
-          s4[e] = fma(vr[8 * c + 2 * e + 1], (double)bf_hi(ws[e]), s4[e]);
+      for (int u = 0; u < 2; ++u) {
+        const int t = b0 + 64 * u + tk;
+        double s4[4] = {0.0, 0.0, 0.0, 0.0};
+        if (u == 0 || two) {
+          const uint4* rr = reinterpret_cast<const uint4*>(rows + (size_t)lo[t] * RS + qd * QD);
+#pragma unroll
+          for (int c = 0; c < QD / 8; ++c) {
+            const uint4 w = rr[c];
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              s4[e] = fma(vr[8 * c + 2 * e], (double)bf_lo(ws[e]), s4[e]);
+              s4[e] = fma(vr[8 * c + 2 * e + 1], (double)bf_hi(ws[e]), s4[e]);
+            }
+          }
         }
+        sacc[u] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       }
-      double sacc = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-      sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
-      sacc += __shfl_xor_sync(0xffffffffu, sacc, 2);
-      sacc -= vmu;
-      if (qd == 0) {
-        pv[t] = sacc;
-        const int id = ids[lo[t]];
-        const double a = fabs(sacc);
-        if (a > best_abs || (a == best_abs && id < best_id)) { best_abs = a; best_p = sacc; best_id = id; }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        sacc[u] += __shfl_xor_sync(0xffffffffu, sacc[u], 1);
+        sacc[u] += __shfl_xor_sync(0xffffffffu, sacc[u], 2);
+        sacc[u] -= vmu;
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int t = b0 + 64 * u + tk;
+        if (qd == 0 && (u == 0 || two)) {
+          pv[t] = sacc[u];
+          const int id = ids[lo[t]];
+          const double a = fabs(sacc[u]);
+          if (a > best_abs || (a == best_abs && id < best_id)) { best_abs = a; best_p = sacc[u]; best_id = id; }
+        }
       }
     }
   }
@@ -1112,9 +1161,7 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(big_gram_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s);
   if (e != cudaSuccess) return e;
-  const size_t smem_solve = sizeof(double) * D * D;
-  e = cudaFuncSetAttribute(big_solve_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_solve);
-  if (e != cudaSuccess) return e;
+  const size_t smem_solve = 0;                     // S goes straight to registers
   const size_t smem_proj = sizeof(uint16_t) * Gram<D>::TILE * 3;
   e = cudaFuncSetAttribute(big_project_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_proj);
   if (e != cudaSuccess) return e;

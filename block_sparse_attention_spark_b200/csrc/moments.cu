@@ -8,6 +8,7 @@
 // column sums, float64-accumulated. Kernel 2 (moments_reduce) adds the
 // partials of a head in a fixed order (deterministic) and divides by N.
 #include "gram.cuh"
+#include "gram_tc.cuh"
 #include "plan.h"
 
 namespace spark {
@@ -91,9 +92,36 @@ __global__ void moments_reduce_kernel(const double* __restrict__ part, int split
   }
 }
 
+// d = 128: the same partial sums on the tcgen05 tensor cores (gram_tc.cuh).
+__global__ void __launch_bounds__(tc::GT_THREADS, 1)
+moments_partial_tc_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, int N,
+                          int blocks_per_split, double* __restrict__ part, int* status) {
+  constexpr int D = tc::GramTcLayout::D;
+  const int split = blockIdx.x, bh = blockIdx.y, t = blockIdx.z;
+  const int BH = gridDim.y, splits = gridDim.x;
+  const uint16_t* X = (t == 0 ? q : k) + (size_t)bh * N * D;
+  const int nb = N / BLK;
+  const int b0 = split * blocks_per_split;
+  const int b1 = min(nb, b0 + blocks_per_split);
+  double* out = part + ((size_t)(t * BH + bh) * splits + split) * (size_t)(D * D + D);
+  tc::gram_tc_body<true>(X, [=](int tt, int r) { return (b0 + tt) * BLK + r; }, max(0, b1 - b0), out, status);
+}
+
 template <int D>
 static cudaError_t run_moments(const Plan& pl, const uint16_t* q, const uint16_t* k, double* MQ,
-                               double* MK, double* qmean, void* ws, cudaStream_t s) {
+                               double* MK, double* qmean, void* ws, int* status, cudaStream_t s) {
+  if constexpr (D == 128) {
+    const int splits = pl.moment_splits;
+    const int bps = (pl.nb + splits - 1) / splits;
+    double* part = ws_at<double>(ws, pl.off_mpart);
+    cudaError_t e = cudaFuncSetAttribute(moments_partial_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         tc::GramTcLayout::SMEM);
+    if (e != cudaSuccess) return e;
+    moments_partial_tc_kernel<<<dim3(splits, pl.BH, 2), tc::GT_THREADS, tc::GramTcLayout::SMEM, s>>>(q, k, pl.N, bps,
+                                                                                                       part, status);
+    moments_reduce_kernel<D><<<dim3(pl.BH, 2), 256, 0, s>>>(part, splits, pl.N, MQ, MK, qmean);
+    return cudaGetLastError();
+  }
   constexpr int STAGES = 3;
   using G = Gram<D>;
   const size_t smem = sizeof(double) * G::ACC * G::THREADS + sizeof(uint16_t) * G::TILE * STAGES;
@@ -109,9 +137,9 @@ static cudaError_t run_moments(const Plan& pl, const uint16_t* q, const uint16_t
 }
 
 cudaError_t launch_moments(const Plan& pl, const uint16_t* q, const uint16_t* k, double* MQ,
-                           double* MK, double* qmean, void* ws, cudaStream_t s) {
-  if (pl.d == 128) return run_moments<128>(pl, q, k, MQ, MK, qmean, ws, s);
-  return run_moments<64>(pl, q, k, MQ, MK, qmean, ws, s);
+                           double* MK, double* qmean, void* ws, int* status, cudaStream_t s) {
+  if (pl.d == 128) return run_moments<128>(pl, q, k, MQ, MK, qmean, ws, status, s);
+  return run_moments<64>(pl, q, k, MQ, MK, qmean, ws, status, s);
 }
 
 }  // namespace spark

@@ -60,7 +60,7 @@ inline T* ws_at(void* ws, size_t off) {
 
 // ---- launchers (each returns cudaGetLastError() of its launches)
 cudaError_t launch_moments(const Plan& pl, const uint16_t* q, const uint16_t* k, double* MQ,
-                           double* MK, double* qmean, void* ws, cudaStream_t s);
+                           double* MK, double* qmean, void* ws, int* status, cudaStream_t s);
 cudaError_t launch_reblock(const Plan& pl, const uint16_t* x, const double* M, int32_t* perm,
                            void* ws, int* status, cudaStream_t s);
 cudaError_t launch_positional(const Plan& pl, int F, int Hl, int Wl, int32_t* perm,

@@ -28,6 +28,7 @@
 #include <math.h>
 
 #include "gram.cuh"
+#include "gram_tc.cuh"
 #include "plan.h"
 
 namespace spark {
@@ -580,6 +581,21 @@ big_gram_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restrict
     for (int kk = 0; kk < 256 / D; ++kk) t += cs[tid + kk * D];
     out[D * D + tid] = t;
   }
+}
+
+// d = 128: the chunk's Gram sums on the tcgen05 tensor cores (gram_tc.cuh);
+// same output as big_gram_kernel.
+__global__ void __launch_bounds__(tc::GT_THREADS, 1)
+big_gram_tc_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restrict__ nodes, int nnodes,
+                   int chunks, int kstep, const int32_t* __restrict__ idx, double* __restrict__ part, int* status) {
+  constexpr int D = tc::GramTcLayout::D;
+  const int c = blockIdx.x, k = blockIdx.y * kstep, bh = blockIdx.z;
+  const int2 node = nodes[k];
+  const int t0 = c * BIG_CHUNK_TILES, t1 = min(node.y, t0 + BIG_CHUNK_TILES);
+  const uint16_t* X = uhat + (size_t)bh * N * D;
+  const int32_t* ids = idx + (size_t)bh * N + (size_t)node.x * BLK + (size_t)t0 * BLK;
+  double* out = part + ((size_t)(bh * nnodes + k) * chunks + c) * (size_t)(D * D + D);
+  tc::gram_tc_body<false>(X, [=](int tt, int r) { return ids[tt * BLK + r]; }, max(0, t1 - t0), out, status);
 }
 
 template <int D>
@@ -1161,6 +1177,10 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(big_gram_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s);
   if (e != cudaSuccess) return e;
+  if (D == 128) {
+    e = cudaFuncSetAttribute(big_gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::GramTcLayout::SMEM);
+    if (e != cudaSuccess) return e;
+  }
   const size_t smem_solve = 0;                     // S goes straight to registers
   const size_t smem_proj = sizeof(uint16_t) * Gram<D>::TILE * 3;
   e = cudaFuncSetAttribute(big_project_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_proj);
@@ -1182,7 +1202,11 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
     const int kstep = derive ? 2 : 1;
     double* gpar = derive ? gstore[(lv - 1) & 1] : nullptr;
     double* gout = pl.level_store[lv] ? gstore[lv & 1] : nullptr;
-    big_gram_kernel<D><<<dim3(ch, cnt / kstep, pl.BH), 256, smem_s, s>>>(uhat, pl.N, nd, cnt, ch, kstep, idx, bpart);
+    if (D == 128)
+      big_gram_tc_kernel<<<dim3(ch, cnt / kstep, pl.BH), tc::GT_THREADS, tc::GramTcLayout::SMEM, s>>>(
+          uhat, pl.N, nd, cnt, ch, kstep, idx, bpart, status);
+    else
+      big_gram_kernel<D><<<dim3(ch, cnt / kstep, pl.BH), 256, smem_s, s>>>(uhat, pl.N, nd, cnt, ch, kstep, idx, bpart);
     big_solve_kernel<D><<<dim3(cnt, pl.BH), 256, smem_solve, s>>>(nd, cnt, ch, bpart, binfo, derive, gpar,
                                                                    derive ? pl.level_count[lv - 1] : 0, gout,
                                                                    pl.power_iters);

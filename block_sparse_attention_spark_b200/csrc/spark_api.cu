@@ -215,7 +215,7 @@ spark_status spark_moments(const spark_params* p, const void* q, const void* k, 
   if (!q || !k || !MQ || !MK || !qmean || !aligned16(q) || !aligned16(k)) return SPARK_ERR_INVALID_ARG;
   const spark_status w = check_ws(pl, ws, ws_bytes);
   if (w != SPARK_OK) return w;
-  return cuda_status(launch_moments(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, ws, stream));
+  return cuda_status(launch_moments(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, ws, status_ptr(), stream));
 }
 
 // The partition(s) of the layout: queries under M_K, keys under M_Q, or both
@@ -327,7 +327,7 @@ spark_status spark_forward_joint(const spark_params* p, const void* q, const voi
   double* qmean = ws_at<double>(ws, pl.off_qmean);
   int32_t* perm = ws_at<int32_t>(ws, pl.off_perm);
   int32_t* sel = ws_at<int32_t>(ws, pl.off_sel);
-  cudaError_t e = launch_moments(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, ws, stream);
+  cudaError_t e = launch_moments(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, ws, status_ptr(), stream);
   if (e != cudaSuccess) return SPARK_ERR_CUDA;
   e = reblock_layout(pl, q, k, MQ, MK, perm, ws, stream);
   if (e != cudaSuccess) return SPARK_ERR_CUDA;
@@ -354,7 +354,7 @@ spark_status spark_forward(const spark_params* p, const void* q, const void* k, 
   double* qmean = ws_at<double>(ws, pl.off_qmean);
   int32_t* perm = perm_out ? perm_out : ws_at<int32_t>(ws, pl.off_perm);
   int32_t* sel = sel_out ? sel_out : ws_at<int32_t>(ws, pl.off_sel);
-  cudaError_t e = launch_moments(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, ws, stream);
+  cudaError_t e = launch_moments(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, ws, status_ptr(), stream);
   if (e != cudaSuccess) return SPARK_ERR_CUDA;
   e = reblock_layout(pl, q, k, MQ, MK, perm, ws, stream);
   if (e != cudaSuccess) return SPARK_ERR_CUDA;

@@ -182,8 +182,8 @@ def attn_traffic(w):
     import hashlib
     try:
         rec = json.load(open(os.path.join(ROOT, "profiles", "attn_traffic.json")))
-        src = open(os.path.join(ROOT, rec["source"]), "rb").read()
-        if hashlib.sha256(src).hexdigest() != rec["source_sha256"]:
+        src = b"".join(open(os.path.join(ROOT, f), "rb").read() for f in rec["sources"])
+        if hashlib.sha256(src).hexdigest() != rec["sources_sha256"]:
             return None
         per_head = rec["dram_bytes_per_launch_8_heads"] / rec["heads_captured"]
         return per_head * w.H * w.B

@@ -47,14 +47,25 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["spark", "reference"], default="spark")
-    ap.add_argument("--workload", default="ref_72576")
-    ap.add_argument("--ratio", type=float, default=0.2)
+    ap.add_argument("--workload", default=None,
+                    help="default ref_72576 (long_104832 for --report dense, stress_129024 for --report stats)")
+    ap.add_argument("--ratio", type=float, default=None,
+                    help="default 0.2 (0.1 for --report dense)")
+    ap.add_argument("--report", choices=["dense", "stats"], default=None,
+                    help="a side run of the measurement plan instead of the bench line: "
+                         "'dense' = stage times, the density-1.0 path and torch SDPA at one shape; "
+                         "'stats' = mass recall and log-mass error of three layout/summary variants")
     ap.add_argument("--heads", type=int, default=0,
                     help="use only the first H heads (smaller case for profiling)")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    return ap.parse_args()
+    a = ap.parse_args()
+    if a.workload is None:
+        a.workload = {"dense": "long_104832", "stats": "stress_129024"}.get(a.report, "ref_72576")
+    if a.ratio is None:
+        a.ratio = 0.1 if a.report == "dense" else 0.2
+    return a
 
 
 # ------------------------------------------------------------------ helpers
@@ -433,10 +444,177 @@ def run_spark(a):
     return 0
 
 
+# ------------------------------------------------------------------ side reports
+
+def head_block_stats(q, k, perm, sel, kt, beta, blocks, chunk=4):
+    """Mass recall and log-mass error of one head, float64 on the device
+    (reporting only: the hot path does not use it).
+
+    q, k: [N, d] bf16 in original order; perm: [N] (permuted position ->
+    original token); sel: [nb, Ksel] selected key blocks per query block;
+    kt: [>= nb, d] key summaries; beta: [>= nb] biases; blocks: the query
+    blocks sampled. Mass recall of query i of block a: the share of its
+    softmax mass over all N keys (scale 1/sqrt(d)) that falls on the keys of
+    a's selected blocks. Log-mass error: |q_i . k~_b / sqrt(d) + beta_b -
+    ln sum_{j in b} exp(q_i . k_j / sqrt(d))| over the blocks b that a did not
+    select. Returns (sum of recall, rows, sum of error, (row, block) pairs).
+    """
+    import torch
+    N, d = q.shape
+    nb = N // 64
+    dev = q.device
+    pl = perm.long()
+    kp = k.index_select(0, pl).double()
+    ktd = kt[:nb].double()
+    bd = beta[:nb].double()
+    scale = 1.0 / math.sqrt(d)
+    rs, nr, es, ne = 0.0, 0, 0.0, 0
+    for c0 in range(0, len(blocks), chunk):
+        bl = blocks[c0:c0 + chunk]
+        rows = (bl[:, None] * 64 + torch.arange(64, device=dev)[None, :]).reshape(-1)
+        qi = q.index_select(0, pl[rows]).double()
+        lse_b = torch.logsumexp(((qi @ kp.T) * scale).view(len(rows), nb, 64), dim=2)
+        lse_all = torch.logsumexp(lse_b, dim=1)
+        mask = torch.zeros(len(bl), nb, dtype=torch.bool, device=dev)
+        mask.scatter_(1, sel[bl].long(), True)
+        mask = mask.repeat_interleave(64, dim=0)
+        lse_sel = torch.logsumexp(lse_b.masked_fill(~mask, -math.inf), dim=1)
+        rs += float(torch.exp(lse_sel - lse_all).sum())
+        nr += len(rows)
+        err = ((qi @ ktd.T) * scale + bd[None, :] - lse_b).abs().masked_fill(mask, 0.0)
+        es += float(err.sum())
+        ne += int((~mask).sum())
+    return rs, nr, es, ne
+
+
+def _upload(w):
+    import numpy as np
+    import torch
+    qh, kh, vh = make_inputs_parallel(w)          # before the first CUDA call
+
+    def up(x):
+        return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    return up(qh), up(kh), up(vh)
+
+
+def run_report_stats(a):
+    """Mass recall and log-mass error (float64, 32 seeded query blocks per
+    head, every head) of three variants on the same inputs: positional tiles
+    + mean-pool summaries, reblock + mean-pool, reblock + reweight."""
+    import numpy as np
+    import torch
+    import block_sparse_attention_spark_b200 as spark
+    w = workload(a)
+    q, k, v = _upload(w)
+    nb = w.N // 64
+    nsamp = min(32, nb)
+    rng = np.random.default_rng(0x57A75)
+    blocks = [[torch.from_numpy(np.sort(rng.choice(nb, nsamp, replace=False))).cuda()
+               for _ in range(w.H)] for _ in range(w.B)]
+    res = {}
+    for name, layout, summ in (("positional+meanpool", "positional", "meanpool"),
+                               ("reblock+meanpool", "reblock", "meanpool"),
+                               ("reblock+reweight", "reblock", "reweight")):
+        p = spark.params(w.B, w.H, w.N, w.d, a.ratio, summary=summ)
+        ws = spark.alloc_workspace(p)
+        MQ, MK, qm = spark.moments(p, q, k, ws)
+        perm = spark.positional_perm(p, w.grid) if layout == "positional" else spark.reblock(p, q, k, MQ, MK, ws)
+        sel = spark.select(p, q, k, v, perm, qm, ws)
+        nbp = spark.workspace_region(p, "BETA")[1] // (4 * w.B * w.H)
+        kt = spark.ws_view(ws, p, "KT", torch.bfloat16, (w.B, w.H, nbp, w.d))
+        beta = spark.ws_view(ws, p, "BETA", torch.float32, (w.B, w.H, nbp))
+        ksel = spark.num_selected(p)
+        sv = sel.view(w.B, w.H, nb, ksel)
+        if spark.get_status() != 0:
+            raise RuntimeError("device status not OK")
+        tot = [0.0, 0, 0.0, 0]
+        for b in range(w.B):
+            for h in range(w.H):
+                r = head_block_stats(q[b, h], k[b, h], perm[b, h], sv[b, h], kt[b, h], beta[b, h], blocks[b][h])
+                tot = [x + y for x, y in zip(tot, r)]
+        res[name] = {"mass_recall_points": 100.0 * tot[0] / tot[1], "log_mass_error": tot[2] / tot[3]}
+        del ws
+        torch.cuda.empty_cache()
+    print(json.dumps({"report": "stats", "workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                      "topk_ratio": a.ratio, "ksel": ksel,
+                      "sample": "%d seeded query blocks per head, all %d heads, float64" % (nsamp, w.B * w.H),
+                      "variants": res}))
+    return 0
+
+
+def run_report_dense(a):
+    """One shape: the hot path's stage times (CUDA events, mean of the timed
+    steps), the build's own density-1.0 path (identity permutation, every
+    block selected: plain softmax attention through the same kernels) and
+    torch's scaled_dot_product_attention (timing context only)."""
+    import torch
+    import block_sparse_attention_spark_b200 as spark
+    w = workload(a)
+    q, k, v = _upload(w)
+    _, _, dense = flops(w, 0)
+
+    def timed(fn, steps):
+        for _ in range(max(1, a.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    steps = max(1, min(a.steps, 5))
+    p = spark.params(w.B, w.H, w.N, w.d, a.ratio)
+    ws = spark.alloc_workspace(p)
+    st = {}
+    MQ, MK, qm = spark.moments(p, q, k, ws)
+    perm = spark.reblock(p, q, k, MQ, MK, ws)
+    sel = spark.select(p, q, k, v, perm, qm, ws)
+    st["moments"] = timed(lambda: spark.moments(p, q, k, ws), steps)
+    st["reblock"] = timed(lambda: spark.reblock(p, q, k, MQ, MK, ws), steps)
+    st["select"] = timed(lambda: spark.select(p, q, k, v, perm, qm, ws), steps)
+    st["attention"] = timed(lambda: spark.attn_fwd(p, perm, sel, ws), steps)
+    sparse_ms = sum(st.values())
+    del ws
+    torch.cuda.empty_cache()
+    # density 1.0, identity permutation
+    p1 = spark.params(w.B, w.H, w.N, w.d, 1.0)
+    ws1 = spark.alloc_workspace(p1)
+    MQ, MK, qm = spark.moments(p1, q, k, ws1)
+    ident = torch.arange(w.N, dtype=torch.int32, device="cuda").repeat(w.B * w.H).view(w.B, w.H, w.N)
+    sel1 = spark.select(p1, q, k, v, ident, qm, ws1)
+    full_ms = timed(lambda: spark.attn_fwd(p1, ident, sel1, ws1), steps)
+    o1 = spark.attn_fwd(p1, ident, sel1, ws1)
+    if spark.get_status() != 0:
+        raise RuntimeError("device status not OK")
+    sdpa = torch.nn.functional.scaled_dot_product_attention
+    try:
+        sdpa_ms = timed(lambda: sdpa(q, k, v), steps)
+        o2 = sdpa(q, k, v)
+        diff = float((o1[:, :, ::97].float() - o2[:, :, ::97].float()).abs().max())
+    except Exception as e:                    # timing context only: report, do not fail
+        sdpa_ms, diff = None, "torch SDPA unavailable: %s" % str(e).splitlines()[0][:120]
+    tf = lambda ms: None if ms is None else dense / (ms * 1e-3) / 1e12
+    print(json.dumps({"report": "dense", "workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                      "topk_ratio": a.ratio, "ksel": spark.num_selected(p), "stages_ms": st,
+                      "sparse_ms_per_layer": sparse_ms, "sparse_eff_tflops": tf(sparse_ms),
+                      "density1_attn_ms": full_ms, "density1_tflops": tf(full_ms),
+                      "torch_sdpa_ms": sdpa_ms, "torch_sdpa_tflops": tf(sdpa_ms),
+                      "density1_vs_sdpa_max_abs_diff_sampled_rows": diff,
+                      "speedup_sparse_vs_sdpa": None if sdpa_ms is None else sdpa_ms / sparse_ms}))
+    return 0
+
+
 def main():
     a = parse()
     if a.impl == "reference":
         return run_reference(a)
+    if a.report == "stats":
+        return run_report_stats(a)
+    if a.report == "dense":
+        return run_report_dense(a)
     return run_spark(a)
 
 

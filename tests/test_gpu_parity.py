@@ -380,3 +380,34 @@ def test_reference_size_sampled():
         assert e["max_rel_to_bound"] <= 1.0, e
         assert e["max_abs"] <= 2 ** -7 * np.abs(ref[mask]).max() + 4e-3 * e["ref_rms"], e
     print(rep)
+
+
+@pytest.mark.parametrize("summary", ["reweight", "meanpool"])
+def test_report_stats_match_oracle_definitions(summary):
+    """bench.py --report stats computes mass recall and log-mass error on the
+    device in float64; on the GPU's own perm, sel and summaries they equal
+    the oracle's definitions of the two statistics."""
+    import torch
+    import bench
+    w = WORKLOADS["mid_16128"]
+    r = run_stages(w, summary=summary)
+    B, H, N, d = r["q"].shape
+    nb = N // 64
+    ksel = r["sel"].shape[-1] if r["sel"].ndim == 4 else spark.num_selected(r["p"])
+    sel = r["sel"].reshape(B, H, nb, ksel)
+    blocks = np.array([0, 5, 17, nb - 1])
+    for h in (0, 3):
+        q = bf16_bits_to_f64(r["q"][0, h])
+        k = bf16_bits_to_f64(r["k"][0, h])
+        perm = r["perm"][0, h].astype(np.int64)
+        rec = so.mass_recall(q, k, perm, sel[0, h], blocks)
+        lme = so.log_mass_error(q, k, perm, sel[0, h], r["kt"][0, h], r["beta"][0, h], blocks)
+        kt = torch.from_numpy(r["kt"][0, h]).cuda().to(torch.bfloat16)      # bf16 values, exactly
+        rs, nr, es, ne = bench.head_block_stats(
+            to_dev(r["q"][0, h]), to_dev(r["k"][0, h]), torch.from_numpy(perm).cuda(),
+            torch.from_numpy(sel[0, h]).cuda(), kt, torch.from_numpy(r["beta"][0, h]).cuda(),
+            torch.from_numpy(blocks).cuda(), chunk=3)
+        assert nr == 64 * len(blocks)
+        assert ne == 64 * len(blocks) * (nb - ksel)
+        assert 100.0 * rs / nr == pytest.approx(rec, rel=1e-9, abs=1e-9)
+        assert es / ne == pytest.approx(lme, rel=1e-9, abs=1e-12)

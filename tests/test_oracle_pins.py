@@ -11,7 +11,7 @@ import pytest
 
 from oracle import brute_force
 from oracle import spark_oracle as so
-from spark_gen import bf16_bits_to_f64, f32_to_bf16_bits
+from spark_gen import WORKLOADS, bf16_bits_to_f64, f32_to_bf16_bits, make_inputs
 
 RNG = np.random.default_rng(1234)
 
@@ -606,3 +606,24 @@ def test_log_mass_error_zero_for_identical_keys():
     res = _run(q, kb, r.standard_normal((64 * nb, d)), 0.25, np.arange(64 * nb))
     e = so.log_mass_error(q, kb, res["perm"], res["sel"], res["kt"], res["beta"], range(nb))
     assert e < 1e-12
+
+
+@pytest.mark.parametrize("summary", ["reweight", "meanpool"])
+def test_report_stats_helper_matches_oracle(summary):
+    """The statistics helper of bench.py's stats report (float64 torch ops,
+    run here on the CPU) equals the oracle's mass recall and log-mass error
+    on the oracle's own permutation, selection and summaries."""
+    import torch
+    import bench
+    w = WORKLOADS["tiny_4096"]
+    q, k, v = (bf16_bits_to_f64(x[0, 0]) for x in make_inputs(w, heads=[0]))
+    r = so.forward_head(q, k, v, ratio=0.2, summary=summary)
+    nb = q.shape[0] // 64
+    blocks = np.array([1, 9, 30, nb - 1])
+    rec = so.mass_recall(q, k, r["perm"], r["sel"], blocks)
+    lme = so.log_mass_error(q, k, r["perm"], r["sel"], r["kt"], r["beta"], blocks)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a))
+    rs, nr, es, ne = bench.head_block_stats(t(q), t(k), t(r["perm"]), t(r["sel"]), t(r["kt"]), t(r["beta"]),
+                                            t(blocks), chunk=3)
+    assert 100.0 * rs / nr == pytest.approx(rec, rel=1e-10)
+    assert es / ne == pytest.approx(lme, rel=1e-10)

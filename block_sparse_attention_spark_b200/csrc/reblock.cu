@@ -43,7 +43,9 @@ whiten_prep_kernel(const double* __restrict__ M, float* __restrict__ Lout, int* 
   extern __shared__ __align__(128) unsigned char smem_raw[];
   double* A = reinterpret_cast<double*>(smem_raw);
   __shared__ double tr_sh;
+  __shared__ double colj[D];                 // column j of the factor (conflict-free reads)
   const int tid = threadIdx.x, bh = blockIdx.x;
+  const int warp = tid >> 5, lane = tid & 31, nwarps = blockDim.x >> 5;
   const double* Mb = M + (size_t)bh * D * D;
   for (int e = tid; e < D * D; e += blockDim.x) A[e] = Mb[e];
   __syncthreads();
@@ -69,12 +71,16 @@ whiten_prep_kernel(const double* __restrict__ M, float* __restrict__ Lout, int* 
     }
     __syncthreads();
     const double dj = A[j * D + j];
-    for (int i = j + 1 + tid; i < D; i += blockDim.x) A[i * D + j] = dj > 0.0 ? A[i * D + j] / dj : 0.0;
+    for (int i = j + 1 + tid; i < D; i += blockDim.x) {
+      const double l = dj > 0.0 ? A[i * D + j] / dj : 0.0;
+      A[i * D + j] = l;
+      colj[i] = l;
+    }
     __syncthreads();
-    const int m = D - j - 1;
-    for (int e = tid; e < m * m; e += blockDim.x) {
-      const int i = j + 1 + e / m, kk = j + 1 + e % m;
-      if (kk <= i) A[i * D + kk] -= A[i * D + j] * A[kk * D + j];
+    // trailing update of the lower triangle: warp per row, lanes along it
+    for (int i = j + 1 + warp; i < D; i += nwarps) {
+      const double li = colj[i];
+      for (int kk = j + 1 + lane; kk <= i; kk += 32) A[i * D + kk] -= li * colj[kk];
     }
     __syncthreads();
   }
@@ -252,11 +258,16 @@ __global__ void init_idx_kernel(int32_t* idx, int N, long total) {
 }
 
 // ------------------------------------------------------------------ block-wide helpers
-__device__ __forceinline__ int block_excl_scan_256(int flag, int* warp_tot, int& total) {
+// Exclusive prefix sum of per-thread counts over a 256-thread block (and the total).
+__device__ __forceinline__ int block_excl_sum_256(int v, int* warp_tot, int& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const unsigned m = __ballot_sync(0xffffffffu, flag);
-  const int within = __popc(m & ((1u << lane) - 1u));
-  if (lane == 0) warp_tot[warp] = __popc(m);
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
   __syncthreads();
   int before = 0, tot = 0;
 #pragma unroll
@@ -267,12 +278,15 @@ __device__ __forceinline__ int block_excl_scan_256(int flag, int* warp_tot, int&
   }
   __syncthreads();
   total = tot;
-  return before + within;
+  return before + incl - v;
 }
+
+constexpr int SEL_UNR = 8;   // members per thread and pass in the select and the partition
 
 // Radix select over 8-bit digits: finds the key of rank `rank` (1-based)
 // among the n keys produced by getkey(i) whose high bits match. Keys are
 // uint64 (digits from bit 56 down). All 256 threads must call it.
+
 template <class GetKey>
 __device__ uint64_t radix_select_u64(int n, int rank, int nbits, GetKey getkey, int* hist,
                                      int* sh_sel, unsigned long long* sh_key) {
@@ -281,15 +295,22 @@ __device__ uint64_t radix_select_u64(int n, int rank, int nbits, GetKey getkey, 
   for (int shift = nbits - 8; shift >= 0; shift -= 8) {
     for (int b = tid; b < 256; b += blockDim.x) hist[b] = 0;
     __syncthreads();
-    for (int i0 = 0; i0 < n; i0 += blockDim.x) {   // uniform trip count: warp-aggregated adds
-      const int i = i0 + tid;
-      int bkt = -1;
-      if (i < n) {
-        const uint64_t k = getkey(i);
-        if ((k & mask) == prefix) bkt = (int)((k >> shift) & 255);
+    // uniform trip count, SEL_UNR independent key loads in flight per thread,
+    // then warp-aggregated adds
+    for (int i0 = 0; i0 < n; i0 += blockDim.x * SEL_UNR) {
+      uint64_t kk[SEL_UNR];
+#pragma unroll
+      for (int u = 0; u < SEL_UNR; ++u) {
+        const int i = i0 + u * blockDim.x + tid;
+        kk[u] = i < n ? getkey(i) : 0ull;
       }
-      const unsigned peers = __match_any_sync(0xffffffffu, bkt);
-      if (bkt >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bkt], __popc(peers));
+#pragma unroll
+      for (int u = 0; u < SEL_UNR; ++u) {
+        const int i = i0 + u * blockDim.x + tid;
+        const int bkt = (i < n && (kk[u] & mask) == prefix) ? (int)((kk[u] >> shift) & 255) : -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, bkt);
+        if (bkt >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bkt], __popc(peers));
+      }
     }
     __syncthreads();
     if (tid < 32) {
@@ -320,6 +341,7 @@ __device__ uint64_t radix_select_u64(int n, int rank, int nbits, GetKey getkey, 
     __syncthreads();
     if (in_bucket == 1 && shift > 0) {
       // a single key carries this prefix: it is the answer
+#pragma unroll 4
       for (int i = tid; i < n; i += blockDim.x) {
         const uint64_t k = getkey(i);
         if ((k & mask) == prefix) *sh_key = k;
@@ -439,6 +461,7 @@ __device__ void cut_partition(int n, int nL, KeyF pkey, IdF pid, PutF put, int* 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint64_t kstar = radix_select_u64(n, nL, 64, pkey, hist, sh_sel, sh_key);
   int c_less = 0, c_eq = 0;
+#pragma unroll 8
   for (int i = tid; i < n; i += blockDim.x) {
     const uint64_t k = pkey(i);
     c_less += (k < kstar);
@@ -467,24 +490,38 @@ __device__ void cut_partition(int n, int nL, KeyF pkey, IdF pid, PutF put, int* 
     };
     istar = (int32_t)radix_select_u64(n, need, 32, ikey, hist, sh_sel, sh_key);
   }
+  // stable partition: thread t takes SEL_UNR consecutive members per pass,
+  // one block scan of the per-thread left counts places them
   int left_done = 0, right_done = 0;
-  for (int base = 0; base < n; base += blockDim.x) {
-    const int i = base + tid;
-    int goleft = 0;
-    if (i < n) {
-      const uint64_t k = pkey(i);
-      goleft = (k < kstar) || (k == kstar && pid(i) <= istar);
+  for (int base = 0; base < n; base += blockDim.x * SEL_UNR) {
+    const int i0 = base + tid * SEL_UNR;
+    bool gl[SEL_UNR];
+    int cnt = 0;
+#pragma unroll
+    for (int u = 0; u < SEL_UNR; ++u) {
+      const int i = i0 + u;
+      gl[u] = false;
+      if (i < n) {
+        const uint64_t k = pkey(i);
+        gl[u] = (k < kstar) || (k == kstar && pid(i) <= istar);
+      }
+      cnt += gl[u];
     }
     int tot;
-    const int lpos = block_excl_scan_256(goleft, warp_tot, tot);
-    if (i < n) {
-      const int dst = goleft ? left_done + lpos : nL + right_done + (tid - lpos);
-      const bool in_side = goleft ? (dst < nL) : (dst < n);
-      if (in_side) put(dst, i);
-      else set_status(status, STATUS_BAD_INPUT);
+    int l = block_excl_sum_256(cnt, warp_tot, tot);
+    int r = max(0, min(tid * SEL_UNR, n - base)) - l;          // members before this thread going right
+#pragma unroll
+    for (int u = 0; u < SEL_UNR; ++u) {
+      const int i = i0 + u;
+      if (i < n) {
+        const int dst = gl[u] ? left_done + l++ : nL + right_done + r++;
+        const bool in_side = gl[u] ? (dst < nL) : (dst < n);
+        if (in_side) put(dst, i);
+        else set_status(status, STATUS_BAD_INPUT);
+      }
     }
     left_done += tot;
-    right_done += min((int)blockDim.x, n - base) - tot;
+    right_done += min((int)blockDim.x * SEL_UNR, n - base) - tot;
   }
 }
 

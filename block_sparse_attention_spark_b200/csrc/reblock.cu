@@ -281,13 +281,12 @@ __device__ __forceinline__ int block_excl_sum_256(int v, int* warp_tot, int& tot
   return before + incl - v;
 }
 
-constexpr int SEL_UNR = 8;   // members per thread and pass in the select and the partition
-
 // Radix select over 8-bit digits: finds the key of rank `rank` (1-based)
 // among the n keys produced by getkey(i) whose high bits match. Keys are
-// uint64 (digits from bit 56 down). All 256 threads must call it.
-
-template <class GetKey>
+// uint64 (digits from bit 56 down). All 256 threads must call it. UNR keys
+// per thread and pass are loaded before they are counted (several loads in
+// flight for keys in global memory; 1 for keys in shared memory).
+template <int UNR, class GetKey>
 __device__ uint64_t radix_select_u64(int n, int rank, int nbits, GetKey getkey, int* hist,
                                      int* sh_sel, unsigned long long* sh_key) {
   uint64_t prefix = 0, mask = 0;
@@ -295,17 +294,17 @@ __device__ uint64_t radix_select_u64(int n, int rank, int nbits, GetKey getkey, 
   for (int shift = nbits - 8; shift >= 0; shift -= 8) {
     for (int b = tid; b < 256; b += blockDim.x) hist[b] = 0;
     __syncthreads();
-    // uniform trip count, SEL_UNR independent key loads in flight per thread,
-    // then warp-aggregated adds
-    for (int i0 = 0; i0 < n; i0 += blockDim.x * SEL_UNR) {
-      uint64_t kk[SEL_UNR];
+    // uniform trip count, UNR independent key loads per thread, then
+    // warp-aggregated adds
+    for (int i0 = 0; i0 < n; i0 += blockDim.x * UNR) {
+      uint64_t kk[UNR];
 #pragma unroll
-      for (int u = 0; u < SEL_UNR; ++u) {
+      for (int u = 0; u < UNR; ++u) {
         const int i = i0 + u * blockDim.x + tid;
         kk[u] = i < n ? getkey(i) : 0ull;
       }
 #pragma unroll
-      for (int u = 0; u < SEL_UNR; ++u) {
+      for (int u = 0; u < UNR; ++u) {
         const int i = i0 + u * blockDim.x + tid;
         const int bkt = (i < n && (kk[u] & mask) == prefix) ? (int)((kk[u] >> shift) & 255) : -1;
         const unsigned peers = __match_any_sync(0xffffffffu, bkt);
@@ -403,13 +402,16 @@ __device__ void power_iterate_regs(const double (&Sr)[D / 32][D / 8], double* zb
     double* z = zb + (iter & 1) * ZP;
     const bool norm_step = (iter % NORM_EVERY) == NORM_EVERY - 1 || iter == iters - 1;
     double sq = 0.0;
-    double zr[RPT];
+    double ze[RPT][2];                         // two chains per row (column parity), folded below
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) zr[i] = 0.0;
+    for (int i = 0; i < RPT; ++i) { ze[i][0] = 0.0; ze[i][1] = 0.0; }
 #pragma unroll
     for (int j = 0; j < CPT; ++j)
 #pragma unroll
-      for (int i = 0; i < RPT; ++i) zr[i] = fma(Sr[i][j], vloc[j], zr[i]);
+      for (int i = 0; i < RPT; ++i) ze[i][j & 1] = fma(Sr[i][j], vloc[j], ze[i][j & 1]);
+    double zr[RPT];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) zr[i] = ze[i][0] + ze[i][1];
 #pragma unroll
     for (int o = 1; o <= 4; o <<= 1)
 #pragma unroll
@@ -454,12 +456,13 @@ __device__ void power_iterate_regs(const double (&Sr)[D / 32][D / 8], double* zb
 // (block radix select on the ordered float64 projection, then index ties),
 // then a stable partition: the nL smallest keys to positions 0..nL-1, the
 // rest after them. pkey(i) / pid(i): ordered key and token index of member
-// i; put(dst, i) moves member i to position dst.
-template <class KeyF, class IdF, class PutF>
+// i; put(dst, i) moves member i to position dst. UNR: members per thread and
+// pass (8 for keys in global memory, 1 for keys in shared memory).
+template <int UNR, class KeyF, class IdF, class PutF>
 __device__ void cut_partition(int n, int nL, KeyF pkey, IdF pid, PutF put, int* hist, int* sh_sel,
                               unsigned long long* sh_key, int* warp_tot, int* red_i, int* status) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint64_t kstar = radix_select_u64(n, nL, 64, pkey, hist, sh_sel, sh_key);
+  const uint64_t kstar = radix_select_u64<UNR>(n, nL, 64, pkey, hist, sh_sel, sh_key);
   int c_less = 0, c_eq = 0;
 #pragma unroll 8
   for (int i = tid; i < n; i += blockDim.x) {
@@ -488,17 +491,17 @@ __device__ void cut_partition(int n, int nL, KeyF pkey, IdF pid, PutF put, int* 
     auto ikey = [&](int i) -> uint64_t {
       return (pkey(i) == kstar) ? (uint64_t)(uint32_t)pid(i) : 0xffffffffull;
     };
-    istar = (int32_t)radix_select_u64(n, need, 32, ikey, hist, sh_sel, sh_key);
+    istar = (int32_t)radix_select_u64<UNR>(n, need, 32, ikey, hist, sh_sel, sh_key);
   }
-  // stable partition: thread t takes SEL_UNR consecutive members per pass,
-  // one block scan of the per-thread left counts places them
+  // stable partition: thread t takes UNR consecutive members per pass, one
+  // block scan of the per-thread left counts places them
   int left_done = 0, right_done = 0;
-  for (int base = 0; base < n; base += blockDim.x * SEL_UNR) {
-    const int i0 = base + tid * SEL_UNR;
-    bool gl[SEL_UNR];
+  for (int base = 0; base < n; base += blockDim.x * UNR) {
+    const int i0 = base + tid * UNR;
+    bool gl[UNR];
     int cnt = 0;
 #pragma unroll
-    for (int u = 0; u < SEL_UNR; ++u) {
+    for (int u = 0; u < UNR; ++u) {
       const int i = i0 + u;
       gl[u] = false;
       if (i < n) {
@@ -509,9 +512,9 @@ __device__ void cut_partition(int n, int nL, KeyF pkey, IdF pid, PutF put, int* 
     }
     int tot;
     int l = block_excl_sum_256(cnt, warp_tot, tot);
-    int r = max(0, min(tid * SEL_UNR, n - base)) - l;          // members before this thread going right
+    int r = max(0, min(tid * UNR, n - base)) - l;              // members before this thread going right
 #pragma unroll
-    for (int u = 0; u < SEL_UNR; ++u) {
+    for (int u = 0; u < UNR; ++u) {
       const int i = i0 + u;
       if (i < n) {
         const int dst = gl[u] ? left_done + l++ : nL + right_done + r++;
@@ -521,7 +524,7 @@ __device__ void cut_partition(int n, int nL, KeyF pkey, IdF pid, PutF put, int* 
       }
     }
     left_done += tot;
-    right_done += min((int)blockDim.x * SEL_UNR, n - base) - tot;
+    right_done += min((int)blockDim.x * UNR, n - base) - tot;
   }
 }
 
@@ -530,7 +533,7 @@ __device__ void cut_partition(int n, int nL, KeyF pkey, IdF pid, PutF put, int* 
 __device__ void cut_and_partition(int n, int nL, double sgn, const double* pv, const int32_t* pi,
                                   int32_t* ids, int* hist, int* sh_sel, unsigned long long* sh_key,
                                   int* warp_tot, int* red_i, int* status) {
-  cut_partition(
+  cut_partition<8>(
       n, nL, [&](int i) -> uint64_t { return ordered_key(sgn * pv[i]); }, [&](int i) { return pi[i]; },
       [&](int dst, int i) { ids[dst] = pi[i]; }, hist, sh_sel, sh_key, warp_tot, red_i, status);
 }
@@ -934,9 +937,12 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
   for (int iter = 0; iter < iters; ++iter) {
     double* z = zp + (iter & 1) * 2 * D;        // [wn][row]: the two column halves' partial sums
     const bool norm_step = (iter % NORM_EVERY) == NORM_EVERY - 1 || iter == iters - 1;
-    double zr[G::MT][2];
+    // eight independent chains (row pair x column parity), folded afterwards
+    double ze[G::MT][2][2];
 #pragma unroll
-    for (int mt = 0; mt < G::MT; ++mt) { zr[mt][0] = 0.0; zr[mt][1] = 0.0; }
+    for (int mt = 0; mt < G::MT; ++mt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) { ze[mt][h][0] = 0.0; ze[mt][h][1] = 0.0; }
 #pragma unroll
     for (int nt = 0; nt < G::NT; ++nt)
 #pragma unroll
@@ -944,7 +950,13 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
 #pragma unroll
         for (int mt = 0; mt < G::MT; ++mt)
 #pragma unroll
-          for (int h = 0; h < 2; ++h) zr[mt][h] = fma(S[(mt * G::NT + nt) * 4 + 2 * h + e], vl[nt * 2 + e], zr[mt][h]);
+          for (int h = 0; h < 2; ++h)
+            ze[mt][h][e] = fma(S[(mt * G::NT + nt) * 4 + 2 * h + e], vl[nt * 2 + e], ze[mt][h][e]);
+    double zr[G::MT][2];
+#pragma unroll
+    for (int mt = 0; mt < G::MT; ++mt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) zr[mt][h] = ze[mt][h][0] + ze[mt][h][1];
 #pragma unroll
     for (int o = 1; o <= 2; o <<= 1)
 #pragma unroll
@@ -973,12 +985,13 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
       inv = rsqrt(sq);
     }
 #pragma unroll
-    for (int nt = 0; nt < G::NT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int col = n0 + nt * 8 + 2 * (lane & 3) + e;
-        vl[nt * 2 + e] = (z[col] + z[D + col]) * inv;
-      }
+    for (int nt = 0; nt < G::NT; ++nt) {
+      const int col = n0 + nt * 8 + 2 * (lane & 3);     // even: 16-byte aligned pairs
+      const double2 z0 = *reinterpret_cast<const double2*>(z + col);
+      const double2 z1 = *reinterpret_cast<const double2*>(z + D + col);
+      vl[nt * 2] = (z0.x + z1.x) * inv;
+      vl[nt * 2 + 1] = (z0.y + z1.y) * inv;
+    }
   }
   if (wm == 0 && lane < 4) {
 #pragma unroll
@@ -1064,7 +1077,7 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
   // slice, the rest the right child's (order inside a child is irrelevant:
   // it is cut again, and leaves are sorted by index at the end)
   const int nL = BLK * ((nn / BLK) / 2);
-  cut_partition(
+  cut_partition<1>(
       nn, nL, [&](int t) -> uint64_t { return ordered_key(sgn * pv[t]); }, [&](int t) { return ids[lo[t]]; },
       [&](int dst, int t) { stok[dst] = lo[t]; }, hist, sh_sel, sh_key, warp_tot, red_i, status);
   __syncthreads();

@@ -258,6 +258,25 @@ __global__ void init_idx_kernel(int32_t* idx, int N, long total) {
 }
 
 // ------------------------------------------------------------------ block-wide helpers
+// Exclusive prefix count of 0/1 flags over a 256-thread block (and the total).
+__device__ __forceinline__ int block_excl_scan_256(int flag, int* warp_tot, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned m = __ballot_sync(0xffffffffu, flag);
+  const int within = __popc(m & ((1u << lane) - 1u));
+  if (lane == 0) warp_tot[warp] = __popc(m);
+  __syncthreads();
+  int before = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    const int c = warp_tot[w];
+    before += (w < warp) ? c : 0;
+    tot += c;
+  }
+  __syncthreads();
+  total = tot;
+  return before + within;
+}
+
 // Exclusive prefix sum of per-thread counts over a 256-thread block (and the total).
 __device__ __forceinline__ int block_excl_sum_256(int v, int* warp_tot, int& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -402,16 +421,13 @@ __device__ void power_iterate_regs(const double (&Sr)[D / 32][D / 8], double* zb
     double* z = zb + (iter & 1) * ZP;
     const bool norm_step = (iter % NORM_EVERY) == NORM_EVERY - 1 || iter == iters - 1;
     double sq = 0.0;
-    double ze[RPT][2];                         // two chains per row (column parity), folded below
+    double zr[RPT];
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) { ze[i][0] = 0.0; ze[i][1] = 0.0; }
+    for (int i = 0; i < RPT; ++i) zr[i] = 0.0;
 #pragma unroll
     for (int j = 0; j < CPT; ++j)
 #pragma unroll
-      for (int i = 0; i < RPT; ++i) ze[i][j & 1] = fma(Sr[i][j], vloc[j], ze[i][j & 1]);
-    double zr[RPT];
-#pragma unroll
-    for (int i = 0; i < RPT; ++i) zr[i] = ze[i][0] + ze[i][1];
+      for (int i = 0; i < RPT; ++i) zr[i] = fma(Sr[i][j], vloc[j], zr[i]);
 #pragma unroll
     for (int o = 1; o <= 4; o <<= 1)
 #pragma unroll
@@ -511,7 +527,7 @@ __device__ void cut_partition(int n, int nL, KeyF pkey, IdF pid, PutF put, int* 
       cnt += gl[u];
     }
     int tot;
-    int l = block_excl_sum_256(cnt, warp_tot, tot);
+    int l = UNR == 1 ? block_excl_scan_256(cnt, warp_tot, tot) : block_excl_sum_256(cnt, warp_tot, tot);
     int r = max(0, min(tid * UNR, n - base)) - l;              // members before this thread going right
 #pragma unroll
     for (int u = 0; u < UNR; ++u) {
@@ -937,12 +953,9 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
   for (int iter = 0; iter < iters; ++iter) {
     double* z = zp + (iter & 1) * 2 * D;        // [wn][row]: the two column halves' partial sums
     const bool norm_step = (iter % NORM_EVERY) == NORM_EVERY - 1 || iter == iters - 1;
-    // eight independent chains (row pair x column parity), folded afterwards
-    double ze[G::MT][2][2];
+    double zr[G::MT][2];
 #pragma unroll
-    for (int mt = 0; mt < G::MT; ++mt)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) { ze[mt][h][0] = 0.0; ze[mt][h][1] = 0.0; }
+    for (int mt = 0; mt < G::MT; ++mt) { zr[mt][0] = 0.0; zr[mt][1] = 0.0; }
 #pragma unroll
     for (int nt = 0; nt < G::NT; ++nt)
 #pragma unroll
@@ -950,13 +963,7 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
 #pragma unroll
         for (int mt = 0; mt < G::MT; ++mt)
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
-            ze[mt][h][e] = fma(S[(mt * G::NT + nt) * 4 + 2 * h + e], vl[nt * 2 + e], ze[mt][h][e]);
-    double zr[G::MT][2];
-#pragma unroll
-    for (int mt = 0; mt < G::MT; ++mt)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) zr[mt][h] = ze[mt][h][0] + ze[mt][h][1];
+          for (int h = 0; h < 2; ++h) zr[mt][h] = fma(S[(mt * G::NT + nt) * 4 + 2 * h + e], vl[nt * 2 + e], zr[mt][h]);
 #pragma unroll
     for (int o = 1; o <= 2; o <<= 1)
 #pragma unroll
@@ -985,13 +992,12 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
       inv = rsqrt(sq);
     }
 #pragma unroll
-    for (int nt = 0; nt < G::NT; ++nt) {
-      const int col = n0 + nt * 8 + 2 * (lane & 3);     // even: 16-byte aligned pairs
-      const double2 z0 = *reinterpret_cast<const double2*>(z + col);
-      const double2 z1 = *reinterpret_cast<const double2*>(z + D + col);
-      vl[nt * 2] = (z0.x + z1.x) * inv;
-      vl[nt * 2 + 1] = (z0.y + z1.y) * inv;
-    }
+    for (int nt = 0; nt < G::NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int col = n0 + nt * 8 + 2 * (lane & 3) + e;
+        vl[nt * 2 + e] = (z[col] + z[D + col]) * inv;
+      }
   }
   if (wm == 0 && lane < 4) {
 #pragma unroll

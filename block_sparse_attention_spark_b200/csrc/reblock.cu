@@ -231,6 +231,199 @@ normalize_kernel(const uint16_t* __restrict__ X, const float* __restrict__ Lall,
   cp_async_wait<0>();
 }
 
+// d = 128: the same tile product on the tcgen05 tensor cores. Per CTA
+// (persistent over a contiguous range of (head, 128-token) tiles): the
+// head's three bf16 terms of L in shared memory as the B operand (row j =
+// column j of L, K-major, 128-byte swizzle), X tiles through a two-buffer
+// cp.async ring as the A operand, one thread issuing 3 x 8 M128 N128 K16
+// MMAs per tile into one of two TMEM accumulators (float32), and all eight
+// warps turning the previous tile's accumulator into u_hat: warps w and
+// w + 4 hold the two column halves of the same 32 tokens, their float64
+// partial norms meet in shared memory, each writes its half of the rows.
+struct NormTcLayout {
+  static constexpr int D = 128, TOK = 128;
+  static constexpr int ATOM_X = TOK * 128;           // 128 tokens x 64 dims
+  static constexpr int XTILE = 2 * ATOM_X;
+  static constexpr int ATOM_L = D * 128;             // 128 outputs x 64 inputs
+  static constexpr int LTERM = 2 * ATOM_L;
+  static constexpr int OFF_X = 3 * LTERM;
+  static constexpr int SMEM = OFF_X + 2 * XTILE + 1024;
+  // kind::f16, F32 accumulate, BF16 A and B, both K-major, N = M = 128
+  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(D >> 3) << 17) |
+                                    ((uint32_t)(TOK >> 4) << 24);
+};
+
+__global__ void __launch_bounds__(256, 1)
+normalize_tc_kernel(const uint16_t* __restrict__ X, const float* __restrict__ Lall, int N, int BH,
+                    uint16_t* __restrict__ uhat, int* status) {
+  using NL = NormTcLayout;
+  constexpr int D = NL::D, TOK = NL::TOK;
+  extern __shared__ unsigned char nsm_raw[];
+  __shared__ __align__(8) uint64_t nbar[3];          // two accumulators' MMA done, drain
+  __shared__ uint32_t ntmem_sh;
+  __shared__ double nsq[8][32];
+  __shared__ int nabort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tpb = (N + TOK - 1) / TOK;
+  const long items = (long)BH * tpb;
+  const long per = (items + gridDim.x - 1) / gridDim.x;
+  const long it0 = (long)blockIdx.x * per, it1 = min(items, it0 + per);
+  if (it0 >= it1) return;
+  const int nloc = (int)(it1 - it0);
+  const uint32_t base = (smem_u32(nsm_raw) + 1023u) & ~1023u;
+  unsigned char* const sbase = nsm_raw + (base - smem_u32(nsm_raw));
+  const uint32_t bar0 = smem_u32(&nbar[0]);
+  if (tid == 0) {
+    tc::mbar_init(bar0, 1);
+    tc::mbar_init(bar0 + 8, 1);
+    tc::mbar_init(bar0 + 16, 1);
+    nabort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&ntmem_sh)),
+                 "r"(256));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = ntmem_sh;
+
+  auto load_x = [&](int k) {
+    const long it = it0 + k;
+    const int bh = (int)(it / tpb), t0 = (int)(it % tpb) * TOK;
+    unsigned char* xb = sbase + NL::OFF_X + (k & 1) * NL::XTILE;
+    for (int c = tid; c < TOK * (D / 8); c += 256) {
+      const int r = c / (D / 8), ch = c % (D / 8);
+      unsigned char* dst = xb + (ch >> 3) * NL::ATOM_X + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
+      if (t0 + r < N) cp_async16(dst, X + ((size_t)bh * N + t0 + r) * D + ch * 8);
+      else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  // the three bf16 terms of L (they sum to L within 2^-24 relative), B[j][i] = term of L[i][j]
+  auto build_l = [&](int bh) {
+    const float* L = Lall + (size_t)bh * D * D;
+    for (int e = tid; e < D * D; e += 256) {
+      const int i = e / D, j = e % D;
+      const float l = L[e];
+      const __nv_bfloat16 h1 = __float2bfloat16_rn(l);
+      const float r1 = l - __bfloat162float(h1);
+      const __nv_bfloat16 h2 = __float2bfloat16_rn(r1);
+      const float r2 = r1 - __bfloat162float(h2);
+      const __nv_bfloat16 h3 = __float2bfloat16_rn(r2);
+      const int off = (i >> 6) * NL::ATOM_L + j * 128 + ((((i & 63) >> 3) ^ (j & 7)) << 4) + (i & 7) * 2;
+      *reinterpret_cast<uint16_t*>(sbase + off) = __bfloat16_as_ushort(h1);
+      *reinterpret_cast<uint16_t*>(sbase + NL::LTERM + off) = __bfloat16_as_ushort(h2);
+      *reinterpret_cast<uint16_t*>(sbase + 2 * NL::LTERM + off) = __bfloat16_as_ushort(h3);
+    }
+  };
+  auto mma_wait = [&](int k, bool ok) -> bool {
+    return ok && __all_sync(0xffffffffu, tc::mbar_wait(bar0 + 8u * (uint32_t)(k & 1), (uint32_t)((k >> 1) & 1), status));
+  };
+  // u_hat rows of tile k from accumulator k & 1
+  auto epilogue = [&](int k) {
+    const long it = it0 + k;
+    const int bh = (int)(it / tpb), t0 = (int)(it % tpb) * TOK;
+    const int qd = warp & 3, half = warp >> 2;
+    const int tok = t0 + 32 * qd + lane;
+    const uint32_t ta = tmem + ((uint32_t)(32 * qd) << 16) + 128u * (uint32_t)(k & 1) + 64u * (uint32_t)half;
+    uint32_t v[64];
+    tc::tmem_ld32p(ta, v);
+    tc::tmem_ld32p(ta + 32u, v + 32);
+    tc::tmem_ld_wait();
+    double sq = 0.0;
+#pragma unroll
+    for (int e = 0; e < 64; ++e) {
+      const double x = (double)__uint_as_float(v[e]);
+      sq = fma(x, x, sq);
+    }
+    nsq[warp][lane] = sq;
+    __syncthreads();
+    const double n = nsq[qd][lane] + nsq[qd + 4][lane];
+    const double inv = n > 0.0 ? 1.0 / sqrt(n) : 0.0;
+    if (tok < N) {
+      uint4* dst = reinterpret_cast<uint4*>(uhat + ((size_t)bh * N + tok) * D + 64 * half);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const int e = 8 * c + 2 * e2;
+          w[e2] = (uint32_t)__bfloat16_as_ushort(__double2bfloat16((double)__uint_as_float(v[e]) * inv)) |
+                  ((uint32_t)__bfloat16_as_ushort(__double2bfloat16((double)__uint_as_float(v[e + 1]) * inv)) << 16);
+        }
+        dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  };
+
+  bool ok = true;
+  int cur_bh = -1;
+  load_x(0);
+  cp_async_commit();
+  for (int k = 0; k < nloc; ++k) {
+    const int bh = (int)((it0 + k) / tpb);
+    cp_async_wait<0>();
+    tc::fence_proxy_async();                             // cp.async / zero fill -> tensor core reads
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    if (bh != cur_bh) {
+      // a new head: L is rewritten once the previous tile's MMAs have read it
+      if (k > 0) ok = mma_wait(k - 1, ok);
+      build_l(bh);
+      tc::fence_proxy_async();
+      __syncthreads();
+      cur_bh = bh;
+    }
+    if (tid == 0 && ok) {
+      tc::fence_after();
+      const uint32_t xa = base + (uint32_t)(NL::OFF_X + (k & 1) * NL::XTILE);
+      const uint32_t d = tmem + 128u * (uint32_t)(k & 1);
+      for (int term = 0; term < 3; ++term) {
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t ko = (uint32_t)((ks >> 2) * NL::ATOM_X + (ks & 3) * 32);
+          const uint32_t lo = (uint32_t)(term * NL::LTERM + (ks >> 2) * NL::ATOM_L + (ks & 3) * 32);
+          tc::mma_f16(d, tc::sdesc(xa + ko, 16, 1024), tc::sdesc(base + lo, 16, 1024), NL::IDESC,
+                      (term > 0 || ks > 0) ? 1u : 0u);
+        }
+      }
+      tc::mma_commit(bar0 + 8u * (uint32_t)(k & 1));
+    }
+    if (k > 0) {
+      ok = mma_wait(k - 1, ok);                          // also frees the X buffer of tile k - 1
+      tc::fence_after();
+    }
+    if (k + 1 < nloc) load_x(k + 1);
+    cp_async_commit();
+    if (k > 0) {
+      if (ok) epilogue(k - 1);
+      else __syncthreads();                              // the epilogue's barrier, kept uniform
+      tc::fence_before();
+    }
+  }
+  ok = mma_wait(nloc - 1, ok);
+  tc::fence_after();
+  if (ok) epilogue(nloc - 1);
+  else __syncthreads();
+  if (!ok) atomicExch(&nabort, 1);
+  cp_async_wait<0>();
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  if (nabort && tid == 0) {
+    // a wait gave up: one more commit, whose arrival means no MMA of this CTA is in flight
+    tc::mma_commit(bar0 + 16);
+    tc::mbar_wait(bar0 + 16, 0, status);
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
+}
+
 // ------------------------------------------------------------------ tree table
 // Nodes that split, level by level: (first block, g blocks). Same recursion
 // as the host side make_plan() uses for the counts.
@@ -1211,16 +1404,22 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
   if (e != cudaSuccess) return e;
   whiten_prep_kernel<D><<<pl.BH, 256, smem_w, s>>>(M, L, status);
 
-  const size_t smem_n = NormSmem<D>::bytes;
-  e = cudaFuncSetAttribute(normalize_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_n);
-  if (e != cudaSuccess) return e;
   {
     int sms = 148;
     int dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long items = (long)pl.BH * ((pl.N + NormSmem<D>::TOK - 1) / NormSmem<D>::TOK);
     const int grid = (int)std::min<long>(items, sms);
-    normalize_kernel<D><<<grid, 256, smem_n, s>>>(x, L, pl.N, pl.BH, uhat);
+    if (D == 128) {
+      e = cudaFuncSetAttribute(normalize_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, NormTcLayout::SMEM);
+      if (e != cudaSuccess) return e;
+      normalize_tc_kernel<<<grid, 256, NormTcLayout::SMEM, s>>>(x, L, pl.N, pl.BH, uhat, status);
+    } else {
+      const size_t smem_n = NormSmem<D>::bytes;
+      e = cudaFuncSetAttribute(normalize_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_n);
+      if (e != cudaSuccess) return e;
+      normalize_kernel<D><<<grid, 256, smem_n, s>>>(x, L, pl.N, pl.BH, uhat);
+    }
   }
 
   tree_build_kernel<<<1, 1, 0, s>>>(pl.nb, nodes);

@@ -1410,7 +1410,7 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long items = (long)pl.BH * ((pl.N + NormSmem<D>::TOK - 1) / NormSmem<D>::TOK);
     const int grid = (int)std::min<long>(items, sms);
-    if (D == 128) {
+    if constexpr (D == 128) {
       e = cudaFuncSetAttribute(normalize_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, NormTcLayout::SMEM);
       if (e != cudaSuccess) return e;
       normalize_tc_kernel<<<grid, 256, NormTcLayout::SMEM, s>>>(x, L, pl.N, pl.BH, uhat, status);
@@ -1430,12 +1430,12 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
   const size_t smem_t = SubSmem<D>::bytes;
   e = cudaFuncSetAttribute(subtree_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_t);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(big_gram_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s);
-  if (e != cudaSuccess) return e;
-  if (D == 128) {
+  if constexpr (D == 128) {
     e = cudaFuncSetAttribute(big_gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::GramTcLayout::SMEM);
-    if (e != cudaSuccess) return e;
+  } else {
+    e = cudaFuncSetAttribute(big_gram_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s);
   }
+  if (e != cudaSuccess) return e;
   const size_t smem_solve = 0;                     // S goes straight to registers
   const size_t smem_proj = sizeof(uint16_t) * Gram<D>::TILE * 3;
   e = cudaFuncSetAttribute(big_project_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_proj);
@@ -1457,7 +1457,7 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
     const int kstep = derive ? 2 : 1;
     double* gpar = derive ? gstore[(lv - 1) & 1] : nullptr;
     double* gout = pl.level_store[lv] ? gstore[lv & 1] : nullptr;
-    if (D == 128)
+    if constexpr (D == 128)
       big_gram_tc_kernel<<<dim3(ch, cnt / kstep, pl.BH), tc::GT_THREADS, tc::GramTcLayout::SMEM, s>>>(
           uhat, pl.N, nd, cnt, ch, kstep, idx, bpart, status);
     else

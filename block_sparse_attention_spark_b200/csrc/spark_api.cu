@@ -4,6 +4,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "plan.h"
@@ -365,6 +366,43 @@ spark_status spark_forward(const spark_params* p, const void* q, const void* k, 
   return cuda_status(e);
 }
 
+// Copy streams and events of the host-buffer entry point, one set per device,
+// created on first use and kept for the life of the process.
+namespace {
+constexpr int HOST_CHUNKS = 4;             // head chunks pipelined through copy-in, compute, copy-out
+constexpr int HOST_MAX_DEVICES = 64;
+struct HostPipe {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t entry = nullptr, done = nullptr, in[HOST_CHUNKS] = {}, comp[HOST_CHUNKS] = {};
+  bool ready = false;
+};
+std::mutex g_host_mu;                       // one call enqueues at a time: the events are shared
+HostPipe g_host_pipe[HOST_MAX_DEVICES];
+
+HostPipe* host_pipe() {                     // call with g_host_mu held
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= HOST_MAX_DEVICES) return nullptr;
+  HostPipe& hp = g_host_pipe[dev];
+  if (!hp.ready) {
+    bool ok = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.entry, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.done, cudaEventDisableTiming) == cudaSuccess;
+    for (int c = 0; ok && c < HOST_CHUNKS; ++c)
+      ok = cudaEventCreateWithFlags(&hp.in[c], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&hp.comp[c], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) return nullptr;
+    hp.ready = true;
+  }
+  return &hp;
+}
+}  // namespace
+
+// Heads are independent, so the pass runs in up to HOST_CHUNKS chunks of
+// consecutive heads: chunk c + 1 is copied in (one copy stream) while chunk c
+// is computed on the caller's stream and chunk c - 1 is copied out (a second
+// copy stream). The copies start after the work already queued on the
+// caller's stream, and the caller's stream waits for the last copy out.
 spark_status spark_forward_host(const spark_params* p, const void* q_host, const void* k_host,
                                 const void* v_host, void* out_host, float* lse_host, void* ws,
                                 size_t ws_bytes, cudaStream_t stream) {
@@ -375,20 +413,52 @@ spark_status spark_forward_host(const spark_params* p, const void* q_host, const
   if (!q_host || !k_host || !v_host || !out_host) return SPARK_ERR_INVALID_ARG;
   if (ws == nullptr || !aligned16(ws)) return SPARK_ERR_INVALID_ARG;
   if (ws_bytes < pl.host_total) return SPARK_ERR_WORKSPACE;
-  const size_t tb = (size_t)pl.BH * pl.N * pl.d * 2;
-  void* dq = ws_at<char>(ws, pl.off_hq);
-  void* dk = ws_at<char>(ws, pl.off_hk);
-  void* dv = ws_at<char>(ws, pl.off_hv);
-  void* dout = ws_at<char>(ws, pl.off_hout);
+  char* dq = ws_at<char>(ws, pl.off_hq);
+  char* dk = ws_at<char>(ws, pl.off_hk);
+  char* dv = ws_at<char>(ws, pl.off_hv);
+  char* dout = ws_at<char>(ws, pl.off_hout);
   float* dlse = lse_host ? ws_at<float>(ws, pl.off_hlse) : nullptr;
-  if (cudaMemcpyAsync(dq, q_host, tb, cudaMemcpyHostToDevice, stream) != cudaSuccess) return SPARK_ERR_CUDA;
-  if (cudaMemcpyAsync(dk, k_host, tb, cudaMemcpyHostToDevice, stream) != cudaSuccess) return SPARK_ERR_CUDA;
-  if (cudaMemcpyAsync(dv, v_host, tb, cudaMemcpyHostToDevice, stream) != cudaSuccess) return SPARK_ERR_CUDA;
-  const spark_status r = spark_forward(p, dq, dk, dv, dout, dlse, nullptr, nullptr, ws, pl.total, stream);
-  if (r != SPARK_OK) return r;
-  if (cudaMemcpyAsync(out_host, dout, tb, cudaMemcpyDeviceToHost, stream) != cudaSuccess) return SPARK_ERR_CUDA;
-  if (lse_host && cudaMemcpyAsync(lse_host, dlse, (size_t)pl.BH * pl.N * 4, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
-    return SPARK_ERR_CUDA;
+  const size_t head_bytes = (size_t)pl.N * pl.d * 2;   // one head of q, k, v or out
+  const int nch = std::min(pl.BH, HOST_CHUNKS);
+
+  std::lock_guard<std::mutex> guard(g_host_mu);
+  HostPipe* hp = host_pipe();
+  if (hp == nullptr) return SPARK_ERR_CUDA;
+  if (cudaEventRecord(hp->entry, stream) != cudaSuccess) return SPARK_ERR_CUDA;
+  if (cudaStreamWaitEvent(hp->h2d, hp->entry, 0) != cudaSuccess) return SPARK_ERR_CUDA;
+  if (cudaStreamWaitEvent(hp->d2h, hp->entry, 0) != cudaSuccess) return SPARK_ERR_CUDA;
+  auto head0 = [&](int c) { return (int)(((long)pl.BH * c) / nch); };
+  for (int c = 0; c < nch; ++c) {
+    const size_t off = (size_t)head0(c) * head_bytes, len = (size_t)(head0(c + 1) - head0(c)) * head_bytes;
+    if (cudaMemcpyAsync(dq + off, (const char*)q_host + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
+        cudaMemcpyAsync(dk + off, (const char*)k_host + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
+        cudaMemcpyAsync(dv + off, (const char*)v_host + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
+        cudaEventRecord(hp->in[c], hp->h2d) != cudaSuccess)
+      return SPARK_ERR_CUDA;
+  }
+  for (int c = 0; c < nch; ++c) {
+    const int h0 = head0(c), hc = head0(c + 1) - h0;
+    const size_t off = (size_t)h0 * head_bytes, len = (size_t)hc * head_bytes;
+    // the chunk as a problem of its own: hc independent heads (the workspace,
+    // sized for all heads, is reused chunk after chunk on this stream)
+    spark_params pc = *p;
+    pc.B = 1;
+    pc.H = hc;
+    if (cudaStreamWaitEvent(stream, hp->in[c], 0) != cudaSuccess) return SPARK_ERR_CUDA;
+    const spark_status r = spark_forward(&pc, dq + off, dk + off, dv + off, dout + off,
+                                         dlse ? dlse + (size_t)h0 * pl.N : nullptr, nullptr, nullptr, ws, pl.total,
+                                         stream);
+    if (r != SPARK_OK) return r;
+    if (cudaEventRecord(hp->comp[c], stream) != cudaSuccess) return SPARK_ERR_CUDA;
+    if (cudaStreamWaitEvent(hp->d2h, hp->comp[c], 0) != cudaSuccess) return SPARK_ERR_CUDA;
+    if (cudaMemcpyAsync((char*)out_host + off, dout + off, len, cudaMemcpyDeviceToHost, hp->d2h) != cudaSuccess)
+      return SPARK_ERR_CUDA;
+    if (lse_host && cudaMemcpyAsync(lse_host + (size_t)h0 * pl.N, dlse + (size_t)h0 * pl.N, (size_t)hc * pl.N * 4,
+                                    cudaMemcpyDeviceToHost, hp->d2h) != cudaSuccess)
+      return SPARK_ERR_CUDA;
+  }
+  if (cudaEventRecord(hp->done, hp->d2h) != cudaSuccess) return SPARK_ERR_CUDA;
+  if (cudaStreamWaitEvent(stream, hp->done, 0) != cudaSuccess) return SPARK_ERR_CUDA;
   return SPARK_OK;
 }
 

@@ -250,9 +250,16 @@ size_t spark_host_workspace_size(const spark_params* p);
 
 /* The whole pass for HOST tensors (pinned memory recommended): copies q, k,
  * v to the device, runs spark_forward, copies out (and lse if not NULL)
- * back. Asynchronous like every call: the host buffers must stay valid until
- * the stream reaches the end of the call. ws is DEVICE memory of
- * spark_host_workspace_size() bytes. */
+ * back. Heads are independent, so the pass runs in up to four chunks of
+ * consecutive heads, pipelined: the next chunk is copied in and the previous
+ * one copied out while one is computed. The kernels run on `stream`; the
+ * copies run on two copy streams of the library (created on first use per
+ * device, kept for the life of the process), which start after the work
+ * already queued on `stream`, and `stream` waits for the last copy out.
+ * Asynchronous like every call: the host buffers must stay valid until the
+ * stream reaches the end of the call. ws is DEVICE memory of
+ * spark_host_workspace_size() bytes. Calls from several host threads are
+ * enqueued one at a time. */
 spark_status spark_forward_host(const spark_params* p, const void* q_host, const void* k_host,
                                 const void* v_host, void* out_host, float* lse_host,
                                 void* ws, size_t ws_bytes, cudaStream_t stream);

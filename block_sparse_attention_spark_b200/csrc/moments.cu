@@ -3,10 +3,12 @@
 // under the hood"; "Spark-H3" news post, Spark-Reweight bullet).
 //
 // Kernel 1 (moments_partial): grid (splits, B*H, 2 tensors). Each CTA streams
-// a contiguous token range of one head through shared memory (3-stage
-// cp.async pipeline, 16-byte loads) and forms the partial Gram X^T X plus the
-// column sums, float64-accumulated. Kernel 2 (moments_reduce) adds the
-// partials of a head in a fixed order (deterministic) and divides by N.
+// a contiguous token range of one head through shared memory and forms the
+// partial Gram X^T X plus the column sums, float64-accumulated: for d = 128
+// on the tcgen05 tensor cores (gram_tc.cuh, exact float64 column sums), for
+// d = 64 with mma.sync (3-stage cp.async pipeline, 16-byte loads). Kernel 2
+// (moments_reduce) adds the partials of a head in a fixed order
+// (deterministic) and divides by N.
 #include "gram.cuh"
 #include "gram_tc.cuh"
 #include "plan.h"

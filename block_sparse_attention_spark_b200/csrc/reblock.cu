@@ -13,12 +13,14 @@
 // Kernels, in launch order:
 //   whiten_prep  : one CTA per head - regularise M, float64 Cholesky -> L (f32)
 //   normalize    : persistent CTAs over 128-token tiles - U = X L on the tensor
-//                  cores (L as three bf16 terms), u_hat = bf16(u/|u|)
+//                  cores (L as three bf16 terms; tcgen05 + TMEM for d = 128,
+//                  mma.sync for d = 64), u_hat = bf16(u/|u|)
 //   tree_build   : node table (first block, g) per level; depends on nb only
 //   init_idx     : identity token order
 //   big_gram / big_solve / big_project / big_select, per level above the
-//                  subtree level - chunked Gram sums of the groups (mma.sync,
-//                  float64 flush; right halves derived from the parent level),
+//                  subtree level - chunked Gram sums of the groups (tcgen05
+//                  for d = 128, mma.sync for d = 64; float64 flush; right
+//                  halves derived from the parent level),
 //                  covariance and float64 power iteration in registers,
 //                  float64 projections, orientation, radix select of the cut,
 //                  stable partition of the group's index slice

@@ -282,7 +282,7 @@ def run_spark(a):
     def step(evs=None):
         if evs is not None:
             evs[0].record(stream)
-        MQ, MK, qmean = spark.moments(p, q, k, ws)
+        MQ, MK, qmean = spark.moments(p, q, k, ws, which="layout")
         if evs is not None:
             evs[1].record(stream)
         perm = spark.reblock(p, q, k, MQ, MK, ws)
@@ -517,7 +517,7 @@ def run_report_stats(a):
                                ("reblock+reweight", "reblock", "reweight")):
         p = spark.params(w.B, w.H, w.N, w.d, a.ratio, summary=summ)
         ws = spark.alloc_workspace(p)
-        MQ, MK, qm = spark.moments(p, q, k, ws)
+        MQ, MK, qm = spark.moments(p, q, k, ws, which="layout")
         perm = spark.positional_perm(p, w.grid) if layout == "positional" else spark.reblock(p, q, k, MQ, MK, ws)
         sel = spark.select(p, q, k, v, perm, qm, ws)
         nbp = spark.workspace_region(p, "BETA")[1] // (4 * w.B * w.H)
@@ -569,10 +569,10 @@ def run_report_dense(a):
     p = spark.params(w.B, w.H, w.N, w.d, a.ratio)
     ws = spark.alloc_workspace(p)
     st = {}
-    MQ, MK, qm = spark.moments(p, q, k, ws)
+    MQ, MK, qm = spark.moments(p, q, k, ws, which="layout")
     perm = spark.reblock(p, q, k, MQ, MK, ws)
     sel = spark.select(p, q, k, v, perm, qm, ws)
-    st["moments"] = timed(lambda: spark.moments(p, q, k, ws), steps)
+    st["moments"] = timed(lambda: spark.moments(p, q, k, ws, which="layout"), steps)
     st["reblock"] = timed(lambda: spark.reblock(p, q, k, MQ, MK, ws), steps)
     st["select"] = timed(lambda: spark.select(p, q, k, v, perm, qm, ws), steps)
     st["attention"] = timed(lambda: spark.attn_fwd(p, perm, sel, ws), steps)
@@ -582,7 +582,7 @@ def run_report_dense(a):
     # density 1.0, identity permutation
     p1 = spark.params(w.B, w.H, w.N, w.d, 1.0)
     ws1 = spark.alloc_workspace(p1)
-    MQ, MK, qm = spark.moments(p1, q, k, ws1)
+    MQ, MK, qm = spark.moments(p1, q, k, ws1, which="layout")
     ident = torch.arange(w.N, dtype=torch.int32, device="cuda").repeat(w.B * w.H).view(w.B, w.H, w.N)
     sel1 = spark.select(p1, q, k, v, ident, qm, ws1)
     full_ms = timed(lambda: spark.attn_fwd(p1, ident, sel1, ws1), steps)

@@ -180,13 +180,21 @@ def ws_view(ws, p: Params, name: str, dtype, shape):
     return ws[off:off + count * esz].view(dtype).view(*shape)
 
 
-def moments(p: Params, q, k, ws):
+def moments(p: Params, q, k, ws, which="both"):
+    """M_Q, M_K (float64 [B,H,d,d]) and the anchor qbar ([B,H,d]).
+    which="layout" forms only the moment(s) the layout partitions under (the
+    others come back as None), as spark_forward does."""
     torch = _torch()
     shp = (p.B, p.H, p.N, p.d)
     _need(q, torch.bfloat16, shp, "q")
     _need(k, torch.bfloat16, shp, "k")
-    MQ = torch.empty(p.B, p.H, p.d, p.d, dtype=torch.float64, device="cuda")
-    MK = torch.empty_like(MQ)
+    if which not in ("both", "layout"):
+        raise ValueError(which)
+    lay = p.layout
+    want_q = which == "both" or lay != LAYOUTS["q_reuse_k"]
+    want_k = which == "both" or lay != LAYOUTS["k_reuse_q"]
+    MQ = torch.empty(p.B, p.H, p.d, p.d, dtype=torch.float64, device="cuda") if want_q else None
+    MK = torch.empty(p.B, p.H, p.d, p.d, dtype=torch.float64, device="cuda") if want_k else None
     qmean = torch.empty(p.B, p.H, p.d, dtype=torch.float64, device="cuda")
     _check(lib().spark_moments(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(MQ), _ptr(MK), _ptr(qmean),
                                _ptr(ws), ws.numel(), _stream()), "spark_moments")

@@ -2,154 +2,249 @@
 // anchor qbar = E[q] ("MiniMax H3 Spark Attention (SM89)", "What it's doing
 // under the hood"; "Spark-H3" news post, Spark-Reweight bullet).
 //
-// Kernel 1 (moments_partial): grid (splits, B*H, 2 tensors). Each CTA streams
-// a contiguous token range of one head through shared memory and forms the
-// partial Gram X^T X plus the column sums, float64-accumulated: for d = 128
-// on the tcgen05 tensor cores (gram_tc.cuh, exact float64 column sums), for
-// d = 64 with mma.sync (3-stage cp.async pipeline, 16-byte loads). Kernel 2
-// (moments_reduce) adds the partials of a head in a fixed order
-// (deterministic) and divides by N.
-#include "gram.cuh"
-#include "gram_tc.cuh"
+// The moment a partition whitens with decides, through its Cholesky factor,
+// every bf16 rounding of the normalised whitened tokens, and one rounding that
+// lands on the other side of a bf16 midpoint moves a token across a cut. So
+// the Gram sums are float64 sums of exact products, as the plain definition
+// (1/N) sum_t x_t x_t^T evaluates them: bf16 inputs widened to float64 and
+// multiplied on the float64 tensor cores (dmma.cuh), never float32 partials.
+//
+// Kernel 1 (moments_gram64): grid (splits, B*H). Each CTA takes a contiguous
+// range of 64-token tiles of one head, widens each tile to float64 in shared
+// memory (double-buffered, the next tile's global loads in flight during the
+// current tile's MMAs) and accumulates the upper-triangle tiles of X^T X in
+// registers (72 of the 128 16x8 tiles for d = 128); with COLSUM also the
+// exact float64 column sums. Kernel 1b (moments_colsum): the column sums
+// alone, for the anchor when the query moment is not needed. Kernel 2
+// (moments_reduce) adds a head's partials in a fixed order, mirrors the
+// triangle and divides by N. The number of token chunks depends on N only, so
+// a head's sums are the same whatever else shares the call.
+#include "dmma.cuh"
 #include "plan.h"
 
 namespace spark {
 
-template <int D, int STAGES>
+template <int D>
+struct MomSmem {
+  static constexpr int TT = BLK;                      // tokens per tile
+  static constexpr int LD = D + 4;                    // float64 row stride (conflict-free fragments)
+  static constexpr int TILE = TT * LD;                // doubles per tile buffer
+  static constexpr size_t bytes = sizeof(double) * 2 * TILE;
+  static constexpr int CPT = TT * (D / 8) / 256;      // 16-byte chunks per thread and tile
+};
+
+template <int D, bool COLSUM>
 __global__ void __launch_bounds__(256, 1)
-moments_partial_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, int N,
-                       int blocks_per_split, double* __restrict__ part) {
-  using G = Gram<D>;
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  double* acc64 = reinterpret_cast<double*>(smem_raw);
-  uint16_t* tiles = reinterpret_cast<uint16_t*>(smem_raw + sizeof(double) * G::ACC * G::THREADS);
-  __shared__ double colsum_sh[D];
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int split = blockIdx.x, bh = blockIdx.y, t = blockIdx.z;
-  const int BH = gridDim.y, splits = gridDim.x;
-  const uint16_t* X = (t == 0 ? q : k) + (size_t)bh * N * D;
+moments_gram64_kernel(const uint16_t* __restrict__ X, int N, int blocks_per_split, double* __restrict__ part) {
+  using SM = MomSmem<D>;
+  using TRI = TriTiles<D>;
+  constexpr int LD = SM::LD;
+  constexpr int SLOTS = (TRI::PAIRS + 7) / 8;         // tiles per warp
+  extern __shared__ __align__(16) double msm[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
+  const int split = blockIdx.x, bh = blockIdx.y, splits = gridDim.x;
   const int nb = N / BLK;
-  const int b0 = split * blocks_per_split;
-  const int b1 = min(nb, b0 + blocks_per_split);
+  const int b0 = split * blocks_per_split, b1 = min(nb, b0 + blocks_per_split);
   const int ntiles = max(0, b1 - b0);
+  const uint16_t* Xh = X + ((size_t)bh * N + (size_t)b0 * BLK) * D;
 
-  for (int j = tid; j < G::ACC * G::THREADS; j += G::THREADS) acc64[j] = 0.0;
-  float acc[G::ACC];
+  int pr[SLOTS], pc[SLOTS];
+  bool pv[SLOTS];
 #pragma unroll
-  for (int j = 0; j < G::ACC; ++j) acc[j] = 0.f;
+  for (int s = 0; s < SLOTS; ++s) {
+    const int p = warp * SLOTS + s;
+    pv[s] = p < TRI::PAIRS;
+    pr[s] = 0;
+    pc[s] = 0;
+    if (pv[s]) TRI::decode(p, pr[s], pc[s]);
+  }
+  double acc[SLOTS][4];
+#pragma unroll
+  for (int s = 0; s < SLOTS; ++s)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[s][e] = 0.0;
   double csum = 0.0;
 
+  uint4 pre[SM::CPT];
+  auto fetch = [&](int t) {
 #pragma unroll
-  for (int s = 0; s < STAGES - 1; ++s) {
-    if (s < ntiles) G::load_tile(tiles + s * G::TILE, X, nullptr, (long)(b0 + s) * BLK, tid);
-    cp_async_commit();
+    for (int i = 0; i < SM::CPT; ++i) {
+      const int c = tid + 256 * i, r = c / (D / 8), ch = c % (D / 8);
+      pre[i] = __ldg(reinterpret_cast<const uint4*>(Xh + ((size_t)t * BLK + r) * D + ch * 8));
+    }
+  };
+  auto stash = [&](int buf) {
+#pragma unroll
+    for (int i = 0; i < SM::CPT; ++i) {
+      const int c = tid + 256 * i, r = c / (D / 8), ch = c % (D / 8);
+      bf8_to_f64(pre[i], msm + buf * SM::TILE + r * LD + ch * 8);
+    }
+  };
+
+  if (ntiles > 0) {
+    fetch(0);
+    stash(0);
   }
+  __syncthreads();
   for (int it = 0; it < ntiles; ++it) {
-    cp_async_wait<STAGES - 2>();
-    __syncthreads();
-    const int nxt = it + STAGES - 1;
-    if (nxt < ntiles) G::load_tile(tiles + (nxt % STAGES) * G::TILE, X, nullptr, (long)(b0 + nxt) * BLK, tid);
-    cp_async_commit();
-    const uint16_t* sm = tiles + (it % STAGES) * G::TILE;
-    G::tile_mma(sm, acc, warp, lane);
-    if (tid < D) {
+    const double* xs = msm + (it & 1) * SM::TILE;
+    if (it + 1 < ntiles) fetch(it + 1);
+    if (COLSUM && tid < D) {
       double s = 0.0;
-#pragma unroll 8
-      for (int r = 0; r < BLK; ++r) s += (double)bf2f(sm[r * G::RS + tid]);
+      for (int r = 0; r < BLK; ++r) s += xs[r * LD + tid];
       csum += s;
     }
-    if ((it + 1) % G::FLUSH == 0 || it == ntiles - 1) G::flush(acc, acc64, tid);
+#pragma unroll
+    for (int ks = 0; ks < BLK / 16; ++ks) {
+      const double* xk = xs + ks * 16 * LD;
+      double a[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a[i] = 0.0;
+#pragma unroll
+      for (int s = 0; s < SLOTS; ++s) {
+        if (!pv[s]) continue;                          // warp-uniform
+        if (s == 0 || pr[s] != pr[s - 1]) {
+          // A = X^T on this row tile: a[i] = x[token t + 4 (i / 2)][dim 16 r + g + 8 (i % 2)]
+#pragma unroll
+          for (int i = 0; i < 8; ++i) a[i] = xk[(t4 + 4 * (i / 2)) * LD + 16 * pr[s] + g + 8 * (i % 2)];
+        }
+        double b[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) b[i] = xk[(t4 + 4 * i) * LD + 8 * pc[s] + g];
+        dmma16816(acc[s], a, b);
+      }
+    }
+    if (it + 1 < ntiles) stash((it + 1) & 1);
+    __syncthreads();
   }
-  cp_async_wait<0>();
-  __syncthreads();
 
-  double* out = part + ((size_t)(t * BH + bh) * splits + split) * (size_t)(D * D + D);
-#pragma unroll 4
-  for (int j = 0; j < G::ACC; ++j) {
-    int row, col;
-    G::coord(j, warp, lane, row, col);
-    out[row * D + col] = acc64[j * G::THREADS + tid];
+  // upper triangle (row <= col) of this chunk's sums; the reduce mirrors it
+  double* out = part + ((size_t)bh * splits + split) * (size_t)(D * D + D);
+#pragma unroll
+  for (int s = 0; s < SLOTS; ++s) {
+    if (!pv[s]) continue;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int row = 16 * pr[s] + g + 8 * (e >> 1), col = 8 * pc[s] + 2 * t4 + (e & 1);
+      if (row <= col) out[row * D + col] = acc[s][e];
+    }
   }
-  if (tid < D) out[D * D + tid] = csum;
-  (void)colsum_sh;
+  if (COLSUM && tid < D) out[D * D + tid] = csum;
 }
 
+// Column sums alone (same tiles, same order of additions as the COLSUM path
+// of moments_gram64, so both give bit-identical anchors).
 template <int D>
-__global__ void moments_reduce_kernel(const double* __restrict__ part, int splits, int N,
-                                      double* __restrict__ MQ, double* __restrict__ MK,
-                                      double* __restrict__ qmean) {
+__global__ void __launch_bounds__(256)
+moments_colsum_kernel(const uint16_t* __restrict__ X, int N, int blocks_per_split, double* __restrict__ part) {
+  constexpr int CPT = BLK * (D / 8) / 256;
+  __shared__ __align__(16) uint16_t ts[2][BLK * D];
+  const int tid = threadIdx.x;
+  const int split = blockIdx.x, bh = blockIdx.y, splits = gridDim.x;
+  const int nb = N / BLK;
+  const int b0 = split * blocks_per_split, b1 = min(nb, b0 + blocks_per_split);
+  const int ntiles = max(0, b1 - b0);
+  const uint16_t* Xh = X + ((size_t)bh * N + (size_t)b0 * BLK) * D;
+  uint4 pre[CPT];
+  auto fetch = [&](int t) {
+#pragma unroll
+    for (int i = 0; i < CPT; ++i)
+      pre[i] = __ldg(reinterpret_cast<const uint4*>(Xh + (size_t)t * BLK * D) + tid + 256 * i);
+  };
+  auto stash = [&](int buf) {
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) reinterpret_cast<uint4*>(ts[buf])[tid + 256 * i] = pre[i];
+  };
+  double csum = 0.0;
+  if (ntiles > 0) {
+    fetch(0);
+    stash(0);
+  }
+  __syncthreads();
+  for (int it = 0; it < ntiles; ++it) {
+    if (it + 1 < ntiles) fetch(it + 1);
+    if (tid < D) {
+      const uint16_t* xs = ts[it & 1];
+      double s = 0.0;
+      for (int r = 0; r < BLK; ++r) s += (double)bf2f(xs[r * D + tid]);
+      csum += s;
+    }
+    if (it + 1 < ntiles) stash((it + 1) & 1);
+    __syncthreads();
+  }
+  if (tid < D) part[((size_t)bh * splits + split) * (size_t)(D * D + D) + D * D + tid] = csum;
+}
+
+// grid (B*H, 2 tensors): tensor 0 = q (its moment if gram_mask bit 0, and the
+// anchor), tensor 1 = k (its moment if gram_mask bit 1).
+template <int D>
+__global__ void moments_reduce_kernel(const double* __restrict__ part, int splits, int N, double* __restrict__ MQ,
+                                      double* __restrict__ MK, double* __restrict__ qmean, int gram_mask) {
   const int bh = blockIdx.x, t = blockIdx.y, BH = gridDim.x;
+  const bool gram = (gram_mask >> t) & 1;
   const double* src = part + (size_t)(t * BH + bh) * splits * (size_t)(D * D + D);
   double* M = (t == 0 ? MQ : MK) + (size_t)bh * D * D;
-  const double invN = 1.0 / (double)N;
+  const double dN = (double)N;
   for (int e = threadIdx.x; e < D * D + D; e += blockDim.x) {
-    double s = 0.0;
-    for (int i = 0; i < splits; ++i) s += src[(size_t)i * (D * D + D) + e];
     if (e < D * D) {
-      M[e] = s * invN;
+      if (!gram) continue;
+      const int i = e / D, j = e % D;
+      const int se = i <= j ? e : j * D + i;
+      double s = 0.0;
+      for (int c = 0; c < splits; ++c) s += src[(size_t)c * (D * D + D) + se];
+      M[e] = s / dN;
     } else if (t == 0) {
-      qmean[(size_t)bh * D + (e - D * D)] = s * invN;
+      double s = 0.0;
+      for (int c = 0; c < splits; ++c) s += src[(size_t)c * (D * D + D) + e];
+      qmean[(size_t)bh * D + (e - D * D)] = s / dN;
     }
   }
 }
 
-// d = 128: the same partial sums on the tcgen05 tensor cores (gram_tc.cuh).
-__global__ void __launch_bounds__(tc::GT_THREADS, 1)
-moments_partial_tc_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, int N,
-                          int blocks_per_split, double* __restrict__ part, int* status) {
-  constexpr int D = tc::GramTcLayout::D;
-  const int split = blockIdx.x, bh = blockIdx.y, t = blockIdx.z;
-  const int BH = gridDim.y, splits = gridDim.x;
-  const uint16_t* X = (t == 0 ? q : k) + (size_t)bh * N * D;
-  const int nb = N / BLK;
-  const int b0 = split * blocks_per_split;
-  const int b1 = min(nb, b0 + blocks_per_split);
-  double* out = part + ((size_t)(t * BH + bh) * splits + split) * (size_t)(D * D + D);
-  tc::gram_tc_body<true>(X, [=](int tt, int r) { return (b0 + tt) * BLK + r; }, max(0, b1 - b0), out, status);
-}
-
 template <int D>
-static cudaError_t run_moments(const Plan& pl, const uint16_t* q, const uint16_t* k, double* MQ,
-                               double* MK, double* qmean, void* ws, int* status, cudaStream_t s) {
-  if constexpr (D == 128) {
-    const int splits = pl.moment_splits;
-    const int bps = (pl.nb + splits - 1) / splits;
-    double* part = ws_at<double>(ws, pl.off_mpart);
-    cudaError_t e = cudaFuncSetAttribute(moments_partial_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         tc::GramTcLayout::SMEM);
-    if (e != cudaSuccess) return e;
-    moments_partial_tc_kernel<<<dim3(splits, pl.BH, 2), tc::GT_THREADS, tc::GramTcLayout::SMEM, s>>>(q, k, pl.N, bps,
-                                                                                                       part, status);
-    moments_reduce_kernel<D><<<dim3(pl.BH, 2), 256, 0, s>>>(part, splits, pl.N, MQ, MK, qmean);
-    return cudaGetLastError();
-  }
-  constexpr int STAGES = 3;
-  using G = Gram<D>;
-  const size_t smem = sizeof(double) * G::ACC * G::THREADS + sizeof(uint16_t) * G::TILE * STAGES;
-  auto kern = moments_partial_kernel<D, STAGES>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  const int splits = pl.moment_splits;
+static cudaError_t run_moments(const Plan& pl, const uint16_t* q, const uint16_t* k, double* MQ, double* MK,
+                               double* qmean, double* part, int splits, bool gram_q, bool gram_k,
+                               cudaStream_t s) {
+  using SM = MomSmem<D>;
   const int bps = (pl.nb + splits - 1) / splits;
-  double* part = ws_at<double>(ws, pl.off_mpart);
-  kern<<<dim3(splits, pl.BH, 2), G::THREADS, smem, s>>>(q, k, pl.N, bps, part);
-  moments_reduce_kernel<D><<<dim3(pl.BH, 2), 256, 0, s>>>(part, splits, pl.N, MQ, MK, qmean);
+  const size_t tstride = (size_t)pl.BH * splits * (D * D + D);
+  cudaError_t e;
+  if (gram_q) {
+    e = cudaFuncSetAttribute(moments_gram64_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SM::bytes);
+    if (e != cudaSuccess) return e;
+    moments_gram64_kernel<D, true><<<dim3(splits, pl.BH), 256, SM::bytes, s>>>(q, pl.N, bps, part);
+  } else {
+    moments_colsum_kernel<D><<<dim3(splits, pl.BH), 256, 0, s>>>(q, pl.N, bps, part);
+  }
+  if (gram_k) {
+    e = cudaFuncSetAttribute(moments_gram64_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SM::bytes);
+    if (e != cudaSuccess) return e;
+    moments_gram64_kernel<D, false><<<dim3(splits, pl.BH), 256, SM::bytes, s>>>(k, pl.N, bps, part + tstride);
+  }
+  moments_reduce_kernel<D><<<dim3(pl.BH, 2), 256, 0, s>>>(part, splits, pl.N, MQ, MK, qmean,
+                                                          (gram_q ? 1 : 0) | (gram_k ? 2 : 0));
   return cudaGetLastError();
 }
 
-cudaError_t launch_moments(const Plan& pl, const uint16_t* q, const uint16_t* k, double* MQ,
-                           double* MK, double* qmean, void* ws, int* status, cudaStream_t s) {
-  if (pl.d == 128) return run_moments<128>(pl, q, k, MQ, MK, qmean, ws, status, s);
-  return run_moments<64>(pl, q, k, MQ, MK, qmean, ws, status, s);
+cudaError_t launch_moments(const Plan& pl, const uint16_t* q, const uint16_t* k, double* MQ, double* MK,
+                           double* qmean, void* ws, bool gram_q, bool gram_k, cudaStream_t s) {
+  double* part = ws_at<double>(ws, pl.off_mpart);
+  if (pl.d == 128) return run_moments<128>(pl, q, k, MQ, MK, qmean, part, pl.moment_splits, gram_q, gram_k, s);
+  return run_moments<64>(pl, q, k, MQ, MK, qmean, part, pl.moment_splits, gram_q, gram_k, s);
 }
 
 }  // namespace spark
 
 // ------------------------------------------------------------------ allocation-free variant
-// spark_moments_noalloc: the same two kernels, with the per-chunk partial
-// sums kept in a fixed file-scope device array instead of the caller's
-// workspace, for callers that cannot hand over or allocate device memory.
+// spark_moments_noalloc: the same kernels as spark_moments, with the per-chunk
+// partial sums kept in a fixed file-scope device array instead of the
+// caller's workspace, for callers that cannot hand over or allocate device
+// memory. The token range of a head may be cut into fewer chunks than
+// spark_moments uses (so that every partial fits the array): the float64
+// sums are then added in another order and can differ from spark_moments'
+// in the last bits.
 #include <mutex>
 
 namespace spark {
@@ -161,42 +256,18 @@ constexpr size_t NOALLOC_SCRATCH_BYTES = (size_t)SPARK_NOALLOC_SCRATCH_BYTES;
 // stand-in symbol; the device address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) double g_moment_scratch[NOALLOC_SCRATCH_BYTES / sizeof(double)];
 
-constexpr int NOALLOC_MAX_DEVICES = 128;
 static std::mutex g_scratch_mutex;
-static double* g_scratch_addr[NOALLOC_MAX_DEVICES] = {};
 
-// Device address of g_moment_scratch on the current device. Looked up once
-// per device (on that device's first call) and cached.
+// Device address of g_moment_scratch on the current device, looked up on
+// every call with that device current (cheap, and still right after a
+// device reset has loaded the module again at another address).
 static cudaError_t moment_scratch_address(double** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_moment_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = static_cast<double*>(p);
-  }
-  *out = g_scratch_addr[dev];
-  return cudaSuccess;
-}
-
-template <int D>
-static cudaError_t run_moments_static(const Plan& pl, const uint16_t* q, const uint16_t* k, double* MQ,
-                                      double* MK, double* qmean, double* part, int splits,
-                                      cudaStream_t s) {
-  constexpr int STAGES = 3;
-  using G = Gram<D>;
-  const size_t smem = sizeof(double) * G::ACC * G::THREADS + sizeof(uint16_t) * G::TILE * STAGES;
-  auto kern = moments_partial_kernel<D, STAGES>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_moment_scratch);
   if (e != cudaSuccess) return e;
-  const int bps = (pl.nb + splits - 1) / splits;
-  kern<<<dim3(splits, pl.BH, 2), G::THREADS, smem, s>>>(q, k, pl.N, bps, part);
-  moments_reduce_kernel<D><<<dim3(pl.BH, 2), 256, 0, s>>>(part, splits, pl.N, MQ, MK, qmean);
-  return cudaGetLastError();
+  *out = static_cast<double*>(p);
+  return cudaSuccess;
 }
 
 }  // namespace spark
@@ -220,9 +291,9 @@ extern "C" spark_status spark_moments_noalloc(const spark_params* p, const void*
   double* scratch = nullptr;
   if (moment_scratch_address(&scratch) != cudaSuccess) return SPARK_ERR_CUDA;
   const cudaError_t e =
-      pl.d == 128 ? run_moments_static<128>(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean,
-                                            scratch, splits, stream)
-                  : run_moments_static<64>(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean,
-                                           scratch, splits, stream);
+      pl.d == 128 ? run_moments<128>(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, scratch, splits,
+                                     true, true, stream)
+                  : run_moments<64>(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, scratch, splits,
+                                    true, true, stream);
   return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
 }

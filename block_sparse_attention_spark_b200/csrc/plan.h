@@ -11,9 +11,11 @@
 
 namespace spark {
 
-// Number of token chunks each (head, tensor) is split into by the moments
-// kernel; partial Gram matrices are summed in float64 in a fixed order.
-constexpr int MOMENT_SPLITS_MAX = 64;
+// Token chunks of the moments kernels: 32 blocks of 64 tokens each (fewer,
+// larger chunks past MOMENT_SPLITS_MAX); the count depends on N only, and the
+// float64 partial sums of a head are added in a fixed order.
+constexpr int MOMENT_BLOCKS_PER_SPLIT = 32;
+constexpr int MOMENT_SPLITS_MAX = 256;
 
 struct Plan {
   int B = 0, H = 0, N = 0, d = 0, BH = 0, nb = 0, ksel = 0, nb_pad = 0;
@@ -59,8 +61,9 @@ inline T* ws_at(void* ws, size_t off) {
 }
 
 // ---- launchers (each returns cudaGetLastError() of its launches)
+// gram_q / gram_k: form M_Q / M_K (the anchor qbar is always formed).
 cudaError_t launch_moments(const Plan& pl, const uint16_t* q, const uint16_t* k, double* MQ,
-                           double* MK, double* qmean, void* ws, int* status, cudaStream_t s);
+                           double* MK, double* qmean, void* ws, bool gram_q, bool gram_k, cudaStream_t s);
 cudaError_t launch_reblock(const Plan& pl, const uint16_t* x, const double* M, int32_t* perm,
                            void* ws, int* status, cudaStream_t s);
 cudaError_t launch_positional(const Plan& pl, int F, int Hl, int Wl, int32_t* perm,

@@ -11,10 +11,10 @@
 // until every leaf holds exactly 64 tokens (O(N log N) levels).
 //
 // Kernels, in launch order:
-//   whiten_prep  : one CTA per head - regularise M, float64 Cholesky -> L (f32)
-//   normalize    : persistent CTAs over 128-token tiles - U = X L on the tensor
-//                  cores (L as three bf16 terms; tcgen05 + TMEM for d = 128,
-//                  mma.sync for d = 64), u_hat = bf16(u/|u|)
+//   whiten_prep  : one CTA per head - regularise M, float64 Cholesky -> L (f64)
+//   normalize64  : persistent CTAs over 32-token tiles - U = X L in float64 on
+//                  the float64 tensor cores, u_hat = bf16(u/|u|) from the
+//                  float64 quotient (the plain definition's value)
 //   tree_build   : node table (first block, g) per level; depends on nb only
 //   init_idx     : identity token order
 //   big_gram / big_solve / big_project / big_select, per level above the
@@ -29,6 +29,7 @@
 //   leaf_sort    : ascending original index inside every 64-token leaf -> perm
 #include <math.h>
 
+#include "dmma.cuh"
 #include "gram.cuh"
 #include "gram_tc.cuh"
 #include "plan.h"
@@ -41,7 +42,7 @@ constexpr int NORM_EVERY = 4;      // power-iteration steps between rescalings o
 // ------------------------------------------------------------------ whitening factor
 template <int D>
 __global__ void __launch_bounds__(256)
-whiten_prep_kernel(const double* __restrict__ M, float* __restrict__ Lout, int* status) {
+whiten_prep_kernel(const double* __restrict__ M, double* __restrict__ Lout, int* status) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   double* A = reinterpret_cast<double*>(smem_raw);
   __shared__ double tr_sh;
@@ -58,9 +59,9 @@ whiten_prep_kernel(const double* __restrict__ M, float* __restrict__ Lout, int* 
   }
   __syncthreads();
   const double tr = tr_sh;
-  float* L = Lout + (size_t)bh * D * D;
+  double* L = Lout + (size_t)bh * D * D;
   if (tr == 0.0) {   // all-zero moment: whiten with the identity
-    for (int e = tid; e < D * D; e += blockDim.x) L[e] = (e / D == e % D) ? 1.f : 0.f;
+    for (int e = tid; e < D * D; e += blockDim.x) L[e] = (e / D == e % D) ? 1.0 : 0.0;
     return;
   }
   if (tid < D) A[tid * D + tid] += REG_EPS * (tr / D);
@@ -88,342 +89,158 @@ whiten_prep_kernel(const double* __restrict__ M, float* __restrict__ Lout, int* 
   }
   for (int e = tid; e < D * D; e += blockDim.x) {
     const int i = e / D, j = e % D;
-    L[e] = (j <= i) ? (float)A[e] : 0.f;
+    L[e] = (j <= i) ? A[e] : 0.0;
   }
 }
 
-// Output dims [Q*D/4, (Q+1)*D/4) of u = L^T x; L is lower triangular, so
-// only inputs i >= Q*D/4 contribute. The inner loop is fully unrolled so the
-// token's x stays in registers.
 // ------------------------------------------------------------------ normalised whitened tokens
-// u_j = sum_{i >= j} L[i][j] x_i, u_hat = bf16(u / |u|), as the tile product
-// U = X L on the tensor cores (mma.sync m16n8k16, float32 accumulation).
-// x is exact in bf16; L (float32) is split into three bf16 terms that sum to
-// it to within 2^-24 relative, so the product is as accurate as a float32
-// evaluation. Blocks of L above the diagonal are zero and skipped. The norm
-// and the final scaling are float64, the rounding to bf16 is correct
-// rounding of the float64 quotient.
+// u_j = sum_{i >= j} L[i][j] x_i, u_hat = bf16(u / |u|), evaluated as the
+// plain definition does: u in float64 (bf16 x widened, float64 factor,
+// float64 tensor cores, dmma.cuh), |u| = sqrt of the float64 sum of squares,
+// the quotient u_j / |u| by IEEE division and one rounding to bf16 (nearest,
+// ties to even). Up to float64 summation order this is the oracle's value, so
+// u_hat, the vectors every later split reads, agrees bit for bit except where
+// a quotient sits within a float64 rounding of a bf16 midpoint.
 //
-// Persistent CTAs walk a contiguous range of (head, 128-token tile) items;
-// the three L terms of the current head sit transposed in shared memory
-// (row j = column j of L, for conflict-free ldmatrix B fragments), the X
-// tiles are double-buffered with cp.async. Warp w owns tokens 16w..16w+15
-// of a tile and all D outputs, and writes its bf16 rows back through its
-// own rows of the tile buffer for coalesced stores.
+// Persistent CTAs walk a contiguous range of (head, 32-token tile) items. The
+// head's factor L sits in shared memory in float64; token tiles are widened
+// to float64 in a double buffer, the next tile's global loads in flight
+// during the current tile's MMAs. Warp w owns the 16 tokens of m-tile w / 4
+// and a quarter of the outputs: the 8-column tiles {q, 7 - q, 8 + q, 15 - q}
+// (d = 128; {q, 7 - q} for d = 64), q = w % 4, which balances the work of the
+// triangular product (the k-chunks above the diagonal of L are skipped). The
+// quarters' partial norms meet in shared memory; rows are written back
+// through a bf16 staging tile with 16-byte stores.
 template <int D>
 struct NormSmem {
-  static constexpr int TOK = 128;                      // tokens per tile
-  static constexpr int RS = D + 8;                     // padded row (elements)
-  static constexpr size_t l_bytes = sizeof(uint16_t) * 3 * D * RS;
-  static constexpr size_t x_bytes = sizeof(uint16_t) * TOK * RS;
-  static constexpr size_t bytes = l_bytes + 2 * x_bytes;
+  static constexpr int TT = 32;                       // tokens per tile
+  static constexpr int LD = D + 4;                    // float64 row stride (conflict-free fragments)
+  static constexpr int L_DBL = D * LD;
+  static constexpr int X_DBL = TT * LD;
+  static constexpr size_t off_x = sizeof(double) * L_DBL;
+  static constexpr size_t off_o = off_x + sizeof(double) * 2 * X_DBL;
+  static constexpr size_t bytes = off_o + sizeof(uint16_t) * TT * D;
+  static constexpr int CPT = TT * (D / 8) / 256;      // 16-byte input chunks per thread and tile
+  static constexpr int CPW = D / 8 / 4;               // 8-column output tiles per warp
+  static constexpr int KC = D / 16;                   // 16-wide k-chunks
 };
 
 template <int D>
 __global__ void __launch_bounds__(256, 1)
-normalize_kernel(const uint16_t* __restrict__ X, const float* __restrict__ Lall, int N, int BH,
-                 uint16_t* __restrict__ uhat) {
+normalize64_kernel(const uint16_t* __restrict__ X, const double* __restrict__ Lall, int N, int BH,
+                   uint16_t* __restrict__ uhat) {
   using SM = NormSmem<D>;
-  constexpr int TOK = SM::TOK, RS = SM::RS, NT = D / 8;
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  uint16_t* Lt = reinterpret_cast<uint16_t*>(smem_raw);                 // [3][D][RS]
-  uint16_t* Xs = reinterpret_cast<uint16_t*>(smem_raw + SM::l_bytes);   // [2][TOK][RS]
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tpb = (N + TOK - 1) / TOK;
+  constexpr int TT = SM::TT, LD = SM::LD, CPW = SM::CPW;
+  extern __shared__ __align__(16) unsigned char nsm_raw[];
+  double* Ls = reinterpret_cast<double*>(nsm_raw);
+  double* Xs = reinterpret_cast<double*>(nsm_raw + SM::off_x);
+  uint16_t* Os = reinterpret_cast<uint16_t*>(nsm_raw + SM::off_o);
+  __shared__ double nsq[2][4][16];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
+  const int m = warp >> 2, q = warp & 3;
+  const int tpb = N / TT;
   const long items = (long)BH * tpb;
   const long per = (items + gridDim.x - 1) / gridDim.x;
   const long it0 = (long)blockIdx.x * per, it1 = min(items, it0 + per);
   if (it0 >= it1) return;
+  int cs[CPW];
+#pragma unroll
+  for (int j = 0; j < CPW; ++j) cs[j] = 8 * (j >> 1) + ((j & 1) ? 7 - q : q);
 
-  auto load_x = [&](long it, int buf) {
-    const int bh = (int)(it / tpb), t0 = (int)(it % tpb) * TOK;
-    uint16_t* dst = Xs + (size_t)buf * TOK * RS;
-    for (int c = tid; c < TOK * (D / 8); c += 256) {
-      const int r = c / (D / 8), ch = c % (D / 8);
-      if (t0 + r < N) cp_async16(dst + r * RS + ch * 8, X + ((size_t)bh * N + t0 + r) * D + ch * 8);
-      else *reinterpret_cast<uint4*>(dst + r * RS + ch * 8) = make_uint4(0u, 0u, 0u, 0u);
+  uint4 pre[SM::CPT];
+  auto fetch = [&](long it) {
+    const int bh = (int)(it / tpb), t0 = (int)(it % tpb) * TT;
+#pragma unroll
+    for (int i = 0; i < SM::CPT; ++i) {
+      const int c = tid + 256 * i, r = c / (D / 8), ch = c % (D / 8);
+      pre[i] = __ldg(reinterpret_cast<const uint4*>(X + ((size_t)bh * N + t0 + r) * D + ch * 8));
     }
   };
+  auto stash = [&](int buf) {
+#pragma unroll
+    for (int i = 0; i < SM::CPT; ++i) {
+      const int c = tid + 256 * i, r = c / (D / 8), ch = c % (D / 8);
+      bf8_to_f64(pre[i], Xs + buf * SM::X_DBL + r * LD + ch * 8);
+    }
+  };
+
   int cur_bh = -1;
-  load_x(it0, 0);
-  cp_async_commit();
+  fetch(it0);
+  stash(0);
   for (long it = it0; it < it1; ++it) {
     const int buf = (int)((it - it0) & 1);
-    const int bh = (int)(it / tpb), t0 = (int)(it % tpb) * TOK;
-    __syncthreads();                                   // every warp is done with the buffer refilled next
+    const int bh = (int)(it / tpb), t0 = (int)(it % tpb) * TT;
     if (bh != cur_bh) {
-      // three bf16 terms of L, transposed: Lt[term][j][i] = term of L[i][j]
-      const float* L = Lall + (size_t)bh * D * D;
-      for (int e = tid; e < D * D; e += 256) {
-        const int i = e / D, j = e % D;
-        const float l = L[e];
-        const __nv_bfloat16 h1 = __float2bfloat16_rn(l);
-        const float r1 = l - __bfloat162float(h1);
-        const __nv_bfloat16 h2 = __float2bfloat16_rn(r1);
-        const float r2 = r1 - __bfloat162float(h2);
-        const __nv_bfloat16 h3 = __float2bfloat16_rn(r2);
-        Lt[(0 * D + j) * RS + i] = __bfloat16_as_ushort(h1);
-        Lt[(1 * D + j) * RS + i] = __bfloat16_as_ushort(h2);
-        Lt[(2 * D + j) * RS + i] = __bfloat16_as_ushort(h3);
+      // a new head's factor (every warp is past the previous tile's MMAs:
+      // the barrier at the end of the last iteration)
+      const double2* Lg = reinterpret_cast<const double2*>(Lall + (size_t)bh * D * D);
+      for (int e = tid; e < D * D / 2; e += 256) {
+        const int i = (2 * e) / D, j = (2 * e) % D;
+        *reinterpret_cast<double2*>(Ls + i * LD + j) = Lg[e];
       }
       cur_bh = bh;
     }
-    if (it + 1 < it1) load_x(it + 1, buf ^ 1);
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-
-    uint16_t* xs = Xs + (size_t)buf * TOK * RS + (size_t)warp * 16 * RS;   // this warp's 16 rows
-    float acc[NT][4];
+    __syncthreads();                                    // tile `buf` and L are in place
+    if (it + 1 < it1) fetch(it + 1);
+    const double* xs = Xs + buf * SM::X_DBL + (16 * m) * LD;
+    double acc[CPW][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int j = 0; j < CPW; ++j)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+      for (int e = 0; e < 4; ++e) acc[j][e] = 0.0;
 #pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      uint32_t a[4];
-      ldsm_x4(a[0], a[1], a[2], a[3], xs + (lane & 15) * RS + ks * 16 + (lane >> 4) * 8);
+    for (int kc = 0; kc < SM::KC; ++kc) {
+      // A = this m-tile's tokens x dims 16 kc..: a[i] = x[g + 8 (i % 2)][16 kc + t + 4 (i / 2)]
+      double a[8];
 #pragma unroll
-      for (int np = 0; np < NT / 2; ++np) {
-        if (16 * ks + 15 < 16 * np) continue;          // L[i][j] = 0 for i < j: both n-tiles zero
+      for (int i = 0; i < 8; ++i) a[i] = xs[(g + 8 * (i % 2)) * LD + 16 * kc + t4 + 4 * (i / 2)];
 #pragma unroll
-        for (int term = 0; term < 3; ++term) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(b0, b1, b2, b3,
-                  Lt + (size_t)(term * D + 16 * np + (lane >> 4) * 8 + (lane & 7)) * RS + ks * 16 +
-                      ((lane >> 3) & 1) * 8);
-          mma_bf16(acc[2 * np], a, b0, b1);
-          mma_bf16(acc[2 * np + 1], a, b2, b3);
-        }
+      for (int j = 0; j < CPW; ++j) {
+        if (kc < (cs[j] >> 1)) continue;               // L is zero above its diagonal (warp-uniform)
+        double b[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) b[i] = Ls[(16 * kc + t4 + 4 * i) * LD + 8 * cs[j] + g];
+        dmma16816(acc[j], a, b);
       }
     }
-    // rows r0 = lane / 4 and r0 + 8 of this warp's 16; columns 8 nt + 2 (lane % 4) + {0, 1}
-    double n0 = 0.0, n1 = 0.0;
+    // |u|^2 of tokens g and g + 8 of the m-tile: this warp's columns, then the quarters
+    double s0 = 0.0, s1 = 0.0;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      n0 += (double)acc[nt][0] * acc[nt][0] + (double)acc[nt][1] * acc[nt][1];
-      n1 += (double)acc[nt][2] * acc[nt][2] + (double)acc[nt][3] * acc[nt][3];
+    for (int j = 0; j < CPW; ++j) {
+      s0 = fma(acc[j][0], acc[j][0], s0);
+      s0 = fma(acc[j][1], acc[j][1], s0);
+      s1 = fma(acc[j][2], acc[j][2], s1);
+      s1 = fma(acc[j][3], acc[j][3], s1);
     }
-    n0 += __shfl_xor_sync(0xffffffffu, n0, 1);
-    n0 += __shfl_xor_sync(0xffffffffu, n0, 2);
-    n1 += __shfl_xor_sync(0xffffffffu, n1, 1);
-    n1 += __shfl_xor_sync(0xffffffffu, n1, 2);
-    const double i0 = n0 > 0.0 ? 1.0 / sqrt(n0) : 0.0, i1 = n1 > 0.0 ? 1.0 / sqrt(n1) : 0.0;
-    __syncwarp();
-    const int r0 = lane >> 2, c0 = 2 * (lane & 3);
+    s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+    s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+    if (t4 == 0) {
+      nsq[m][q][g] = s0;
+      nsq[m][q][g + 8] = s1;
+    }
+    __syncthreads();
+    const double n0 = (nsq[m][0][g] + nsq[m][1][g]) + (nsq[m][2][g] + nsq[m][3][g]);
+    const double n1 = (nsq[m][0][g + 8] + nsq[m][1][g + 8]) + (nsq[m][2][g + 8] + nsq[m][3][g + 8]);
+    const double r0 = sqrt(n0), r1 = sqrt(n1);
+    auto q2 = [](double u, double r) -> uint32_t {
+      return r > 0.0 ? (uint32_t)__bfloat16_as_ushort(__double2bfloat16(u / r)) : 0u;
+    };
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const uint32_t w0 = (uint32_t)__bfloat16_as_ushort(__double2bfloat16((double)acc[nt][0] * i0)) |
-                          ((uint32_t)__bfloat16_as_ushort(__double2bfloat16((double)acc[nt][1] * i0)) << 16);
-      const uint32_t w1 = (uint32_t)__bfloat16_as_ushort(__double2bfloat16((double)acc[nt][2] * i1)) |
-                          ((uint32_t)__bfloat16_as_ushort(__double2bfloat16((double)acc[nt][3] * i1)) << 16);
-      *reinterpret_cast<uint32_t*>(xs + r0 * RS + 8 * nt + c0) = w0;
-      *reinterpret_cast<uint32_t*>(xs + (r0 + 8) * RS + 8 * nt + c0) = w1;
+    for (int j = 0; j < CPW; ++j) {
+      const int col = 8 * cs[j] + 2 * t4;
+      *reinterpret_cast<uint32_t*>(Os + (16 * m + g) * D + col) = q2(acc[j][0], r0) | (q2(acc[j][1], r0) << 16);
+      *reinterpret_cast<uint32_t*>(Os + (16 * m + g + 8) * D + col) = q2(acc[j][2], r1) | (q2(acc[j][3], r1) << 16);
     }
-    __syncwarp();
-    // this warp's 16 rows, 16-byte chunks
-    for (int c = lane; c < 16 * (D / 8); c += 32) {
+    if (it + 1 < it1) stash(buf ^ 1);
+    __syncthreads();
+    for (int c = tid; c < TT * (D / 8); c += 256) {
       const int r = c / (D / 8), ch = c % (D / 8);
-      const int tok = t0 + warp * 16 + r;
-      if (tok < N)
-        *reinterpret_cast<uint4*>(uhat + ((size_t)bh * N + tok) * D + ch * 8) =
-            *reinterpret_cast<const uint4*>(xs + r * RS + ch * 8);
+      *reinterpret_cast<uint4*>(uhat + ((size_t)bh * N + t0 + r) * D + ch * 8) =
+          *reinterpret_cast<const uint4*>(Os + r * D + ch * 8);
     }
   }
-  cp_async_wait<0>();
-}
-
-// d = 128: the same tile product on the tcgen05 tensor cores. Per CTA
-// (persistent over a contiguous range of (head, 128-token) tiles): the
-// head's three bf16 terms of L in shared memory as the B operand (row j =
-// column j of L, K-major, 128-byte swizzle), X tiles through a two-buffer
-// cp.async ring as the A operand, one thread issuing 3 x 8 M128 N128 K16
-// MMAs per tile into one of two TMEM accumulators (float32), and all eight
-// warps turning the previous tile's accumulator into u_hat: warps w and
-// w + 4 hold the two column halves of the same 32 tokens, their float64
-// partial norms meet in shared memory, each writes its half of the rows.
-struct NormTcLayout {
-  static constexpr int D = 128, TOK = 128;
-  static constexpr int ATOM_X = TOK * 128;           // 128 tokens x 64 dims
-  static constexpr int XTILE = 2 * ATOM_X;
-  static constexpr int ATOM_L = D * 128;             // 128 outputs x 64 inputs
-  static constexpr int LTERM = 2 * ATOM_L;
-  static constexpr int OFF_X = 3 * LTERM;
-  static constexpr int SMEM = OFF_X + 2 * XTILE + 1024;
-  // kind::f16, F32 accumulate, BF16 A and B, both K-major, N = M = 128
-  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(D >> 3) << 17) |
-                                    ((uint32_t)(TOK >> 4) << 24);
-};
-
-__global__ void __launch_bounds__(256, 1)
-normalize_tc_kernel(const uint16_t* __restrict__ X, const float* __restrict__ Lall, int N, int BH,
-                    uint16_t* __restrict__ uhat, int* status) {
-  using NL = NormTcLayout;
-  constexpr int D = NL::D, TOK = NL::TOK;
-  extern __shared__ unsigned char nsm_raw[];
-  __shared__ __align__(8) uint64_t nbar[3];          // two accumulators' MMA done, drain
-  __shared__ uint32_t ntmem_sh;
-  __shared__ double nsq[8][32];
-  __shared__ int nabort;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tpb = (N + TOK - 1) / TOK;
-  const long items = (long)BH * tpb;
-  const long per = (items + gridDim.x - 1) / gridDim.x;
-  const long it0 = (long)blockIdx.x * per, it1 = min(items, it0 + per);
-  if (it0 >= it1) return;
-  const int nloc = (int)(it1 - it0);
-  const uint32_t base = (smem_u32(nsm_raw) + 1023u) & ~1023u;
-  unsigned char* const sbase = nsm_raw + (base - smem_u32(nsm_raw));
-  const uint32_t bar0 = smem_u32(&nbar[0]);
-  if (tid == 0) {
-    tc::mbar_init(bar0, 1);
-    tc::mbar_init(bar0 + 8, 1);
-    tc::mbar_init(bar0 + 16, 1);
-    nabort = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&ntmem_sh)),
-                 "r"(256));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-  }
-  tc::fence_before();
-  __syncthreads();
-  tc::fence_after();
-  const uint32_t tmem = ntmem_sh;
-
-  auto load_x = [&](int k) {
-    const long it = it0 + k;
-    const int bh = (int)(it / tpb), t0 = (int)(it % tpb) * TOK;
-    unsigned char* xb = sbase + NL::OFF_X + (k & 1) * NL::XTILE;
-    for (int c = tid; c < TOK * (D / 8); c += 256) {
-      const int r = c / (D / 8), ch = c % (D / 8);
-      unsigned char* dst = xb + (ch >> 3) * NL::ATOM_X + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
-      if (t0 + r < N) cp_async16(dst, X + ((size_t)bh * N + t0 + r) * D + ch * 8);
-      else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-    }
-  };
-  // the three bf16 terms of L (they sum to L within 2^-24 relative), B[j][i] = term of L[i][j]
-  auto build_l = [&](int bh) {
-    const float* L = Lall + (size_t)bh * D * D;
-    for (int e = tid; e < D * D; e += 256) {
-      const int i = e / D, j = e % D;
-      const float l = L[e];
-      const __nv_bfloat16 h1 = __float2bfloat16_rn(l);
-      const float r1 = l - __bfloat162float(h1);
-      const __nv_bfloat16 h2 = __float2bfloat16_rn(r1);
-      const float r2 = r1 - __bfloat162float(h2);
-      const __nv_bfloat16 h3 = __float2bfloat16_rn(r2);
-      const int off = (i >> 6) * NL::ATOM_L + j * 128 + ((((i & 63) >> 3) ^ (j & 7)) << 4) + (i & 7) * 2;
-      *reinterpret_cast<uint16_t*>(sbase + off) = __bfloat16_as_ushort(h1);
-      *reinterpret_cast<uint16_t*>(sbase + NL::LTERM + off) = __bfloat16_as_ushort(h2);
-      *reinterpret_cast<uint16_t*>(sbase + 2 * NL::LTERM + off) = __bfloat16_as_ushort(h3);
-    }
-  };
-  auto mma_wait = [&](int k, bool ok) -> bool {
-    return ok && __all_sync(0xffffffffu, tc::mbar_wait(bar0 + 8u * (uint32_t)(k & 1), (uint32_t)((k >> 1) & 1), status));
-  };
-  // u_hat rows of tile k from accumulator k & 1
-  auto epilogue = [&](int k) {
-    const long it = it0 + k;
-    const int bh = (int)(it / tpb), t0 = (int)(it % tpb) * TOK;
-    const int qd = warp & 3, half = warp >> 2;
-    const int tok = t0 + 32 * qd + lane;
-    const uint32_t ta = tmem + ((uint32_t)(32 * qd) << 16) + 128u * (uint32_t)(k & 1) + 64u * (uint32_t)half;
-    uint32_t v[64];
-    tc::tmem_ld32p(ta, v);
-    tc::tmem_ld32p(ta + 32u, v + 32);
-    tc::tmem_ld_wait();
-    double sq = 0.0;
-#pragma unroll
-    for (int e = 0; e < 64; ++e) {
-      const double x = (double)__uint_as_float(v[e]);
-      sq = fma(x, x, sq);
-    }
-    nsq[warp][lane] = sq;
-    __syncthreads();
-    const double n = nsq[qd][lane] + nsq[qd + 4][lane];
-    const double inv = n > 0.0 ? 1.0 / sqrt(n) : 0.0;
-    if (tok < N) {
-      uint4* dst = reinterpret_cast<uint4*>(uhat + ((size_t)bh * N + tok) * D + 64 * half);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          const int e = 8 * c + 2 * e2;
-          w[e2] = (uint32_t)__bfloat16_as_ushort(__double2bfloat16((double)__uint_as_float(v[e]) * inv)) |
-                  ((uint32_t)__bfloat16_as_ushort(__double2bfloat16((double)__uint_as_float(v[e + 1]) * inv)) << 16);
-        }
-        dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-    }
-  };
-
-  bool ok = true;
-  int cur_bh = -1;
-  load_x(0);
-  cp_async_commit();
-  for (int k = 0; k < nloc; ++k) {
-    const int bh = (int)((it0 + k) / tpb);
-    cp_async_wait<0>();
-    tc::fence_proxy_async();                             // cp.async / zero fill -> tensor core reads
-    tc::fence_before();
-    __syncthreads();
-    tc::fence_after();
-    if (bh != cur_bh) {
-      // a new head: L is rewritten once the previous tile's MMAs have read it
-      if (k > 0) ok = mma_wait(k - 1, ok);
-      build_l(bh);
-      tc::fence_proxy_async();
-      __syncthreads();
-      cur_bh = bh;
-    }
-    if (tid == 0 && ok) {
-      tc::fence_after();
-      const uint32_t xa = base + (uint32_t)(NL::OFF_X + (k & 1) * NL::XTILE);
-      const uint32_t d = tmem + 128u * (uint32_t)(k & 1);
-      for (int term = 0; term < 3; ++term) {
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t ko = (uint32_t)((ks >> 2) * NL::ATOM_X + (ks & 3) * 32);
-          const uint32_t lo = (uint32_t)(term * NL::LTERM + (ks >> 2) * NL::ATOM_L + (ks & 3) * 32);
-          tc::mma_f16(d, tc::sdesc(xa + ko, 16, 1024), tc::sdesc(base + lo, 16, 1024), NL::IDESC,
-                      (term > 0 || ks > 0) ? 1u : 0u);
-        }
-      }
-      tc::mma_commit(bar0 + 8u * (uint32_t)(k & 1));
-    }
-    if (k > 0) {
-      ok = mma_wait(k - 1, ok);                          // also frees the X buffer of tile k - 1
-      tc::fence_after();
-    }
-    if (k + 1 < nloc) load_x(k + 1);
-    cp_async_commit();
-    if (k > 0) {
-      if (ok) epilogue(k - 1);
-      else __syncthreads();                              // the epilogue's barrier, kept uniform
-      tc::fence_before();
-    }
-  }
-  ok = mma_wait(nloc - 1, ok);
-  tc::fence_after();
-  if (ok) epilogue(nloc - 1);
-  else __syncthreads();
-  if (!ok) atomicExch(&nabort, 1);
-  cp_async_wait<0>();
-  tc::fence_before();
-  __syncthreads();
-  tc::fence_after();
-  if (nabort && tid == 0) {
-    // a wait gave up: one more commit, whose arrival means no MMA of this CTA is in flight
-    tc::mma_commit(bar0 + 16);
-    tc::mbar_wait(bar0 + 16, 0, status);
-  }
-  tc::fence_before();
-  __syncthreads();
-  tc::fence_after();
-  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
 }
 
 // ------------------------------------------------------------------ tree table
@@ -1393,7 +1210,7 @@ __global__ void positional_perm_kernel(int32_t* perm, int N, int Hl, int Wl, lon
 template <int D>
 static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* M, int32_t* perm,
                                void* ws, int* status, cudaStream_t s) {
-  float* L = ws_at<float>(ws, pl.off_L);
+  double* L = ws_at<double>(ws, pl.off_L);
   uint16_t* uhat = ws_at<uint16_t>(ws, pl.off_uhat);
   int32_t* idx = ws_at<int32_t>(ws, pl.off_idx);
   double* pval = ws_at<double>(ws, pl.off_pval);
@@ -1410,18 +1227,12 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
     int sms = 148;
     int dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const long items = (long)pl.BH * ((pl.N + NormSmem<D>::TOK - 1) / NormSmem<D>::TOK);
+    const long items = (long)pl.BH * (pl.N / NormSmem<D>::TT);
     const int grid = (int)std::min<long>(items, sms);
-    if constexpr (D == 128) {
-      e = cudaFuncSetAttribute(normalize_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, NormTcLayout::SMEM);
-      if (e != cudaSuccess) return e;
-      normalize_tc_kernel<<<grid, 256, NormTcLayout::SMEM, s>>>(x, L, pl.N, pl.BH, uhat, status);
-    } else {
-      const size_t smem_n = NormSmem<D>::bytes;
-      e = cudaFuncSetAttribute(normalize_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_n);
-      if (e != cudaSuccess) return e;
-      normalize_kernel<D><<<grid, 256, smem_n, s>>>(x, L, pl.N, pl.BH, uhat);
-    }
+    e = cudaFuncSetAttribute(normalize64_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)NormSmem<D>::bytes);
+    if (e != cudaSuccess) return e;
+    normalize64_kernel<D><<<grid, 256, NormSmem<D>::bytes, s>>>(x, L, pl.N, pl.BH, uhat);
   }
 
   tree_build_kernel<<<1, 1, 0, s>>>(pl.nb, nodes);

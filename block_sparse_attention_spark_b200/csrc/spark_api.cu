@@ -99,10 +99,7 @@ bool make_plan(const spark_params* p, Plan* pl) {
       }
     }
   }
-  {
-    const int want = (600 + 2 * P.BH - 1) / (2 * P.BH);
-    P.moment_splits = std::max(1, std::min({want, MOMENT_SPLITS_MAX, P.nb}));
-  }
+  P.moment_splits = std::min(MOMENT_SPLITS_MAX, (P.nb + MOMENT_BLOCKS_PER_SPLIT - 1) / MOMENT_BLOCKS_PER_SPLIT);
   const size_t BH = P.BH, N = P.N, d = P.d, nb = P.nb, nbp = P.nb_pad;
   size_t o = 0;
   auto take = [&](size_t bytes) { const size_t at = o; o = align_up(o + bytes); return at; };
@@ -110,7 +107,7 @@ bool make_plan(const spark_params* p, Plan* pl) {
   P.off_MK = take(BH * d * d * 8);
   P.off_qmean = take(BH * d * 8);
   P.off_mpart = take(BH * 2 * (size_t)P.moment_splits * (d * d + d) * 8);
-  P.off_L = take(BH * d * d * 4);
+  P.off_L = take(BH * d * d * 8);
   P.off_uhat = take(BH * N * d * 2);
   P.off_idx = take(BH * N * 4);
   P.off_pval = take(BH * N * 8);
@@ -172,6 +169,11 @@ static spark_status check_ws(const Plan& pl, const void* ws, size_t ws_bytes) {
 
 static spark_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA; }
 
+// The moments a layout partitions under: queries are whitened with M_K, keys
+// with M_Q. The whole pass forms only those (plus the anchor).
+static bool needs_mk(const Plan& pl) { return pl.layout != SPARK_LAYOUT_K_REUSE_Q; }
+static bool needs_mq(const Plan& pl) { return pl.layout != SPARK_LAYOUT_Q_REUSE_K; }
+
 }  // namespace spark
 
 using namespace spark;
@@ -213,10 +215,11 @@ spark_status spark_moments(const spark_params* p, const void* q, const void* k, 
   if (v != SPARK_OK) return v;
   Plan pl;
   make_plan(p, &pl);
-  if (!q || !k || !MQ || !MK || !qmean || !aligned16(q) || !aligned16(k)) return SPARK_ERR_INVALID_ARG;
+  if (!q || !k || !qmean || !aligned16(q) || !aligned16(k)) return SPARK_ERR_INVALID_ARG;
   const spark_status w = check_ws(pl, ws, ws_bytes);
   if (w != SPARK_OK) return w;
-  return cuda_status(launch_moments(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, ws, status_ptr(), stream));
+  return cuda_status(launch_moments(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, ws, MQ != nullptr,
+                                    MK != nullptr, stream));
 }
 
 // The partition(s) of the layout: queries under M_K, keys under M_Q, or both
@@ -236,7 +239,8 @@ spark_status spark_reblock(const spark_params* p, const void* q, const void* k, 
   if (v != SPARK_OK) return v;
   Plan pl;
   make_plan(p, &pl);
-  if (!q || !k || !MQ || !MK || !perm || !aligned16(q) || !aligned16(k)) return SPARK_ERR_INVALID_ARG;
+  if (!q || !k || !perm || !aligned16(q) || !aligned16(k)) return SPARK_ERR_INVALID_ARG;
+  if ((needs_mq(pl) && !MQ) || (needs_mk(pl) && !MK)) return SPARK_ERR_INVALID_ARG;
   const spark_status w = check_ws(pl, ws, ws_bytes);
   if (w != SPARK_OK) return w;
   return cuda_status(reblock_layout(pl, q, k, MQ, MK, perm, ws, stream));
@@ -328,7 +332,8 @@ spark_status spark_forward_joint(const spark_params* p, const void* q, const voi
   double* qmean = ws_at<double>(ws, pl.off_qmean);
   int32_t* perm = ws_at<int32_t>(ws, pl.off_perm);
   int32_t* sel = ws_at<int32_t>(ws, pl.off_sel);
-  cudaError_t e = launch_moments(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, ws, status_ptr(), stream);
+  cudaError_t e = launch_moments(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, ws, needs_mq(pl),
+                                 needs_mk(pl), stream);
   if (e != cudaSuccess) return SPARK_ERR_CUDA;
   e = reblock_layout(pl, q, k, MQ, MK, perm, ws, stream);
   if (e != cudaSuccess) return SPARK_ERR_CUDA;
@@ -355,7 +360,8 @@ spark_status spark_forward(const spark_params* p, const void* q, const void* k, 
   double* qmean = ws_at<double>(ws, pl.off_qmean);
   int32_t* perm = perm_out ? perm_out : ws_at<int32_t>(ws, pl.off_perm);
   int32_t* sel = sel_out ? sel_out : ws_at<int32_t>(ws, pl.off_sel);
-  cudaError_t e = launch_moments(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, ws, status_ptr(), stream);
+  cudaError_t e = launch_moments(pl, (const uint16_t*)q, (const uint16_t*)k, MQ, MK, qmean, ws, needs_mq(pl),
+                                 needs_mk(pl), stream);
   if (e != cudaSuccess) return SPARK_ERR_CUDA;
   e = reblock_layout(pl, q, k, MQ, MK, perm, ws, stream);
   if (e != cudaSuccess) return SPARK_ERR_CUDA;

@@ -116,8 +116,14 @@ size_t spark_workspace_size(const spark_params* p);
 /* Step 1 - second moments ([P2] under the hood: M_K = E[k k^T] for queries,
  * M_Q for keys) and the per-head mean query ([P1] Spark-Reweight bullet: the
  * mean video query is the anchor of each head). Uncentered, over all N tokens.
+ * Products of the bf16 inputs are exact in float64 and the sums are float64
+ * (float64 tensor cores), so the moments equal (1/N) sum x x^T up to float64
+ * summation order: the partition's whitening, and every bf16 rounding of the
+ * whitened tokens, then agree with a float64 evaluation of the definition.
  *   q, k   : [B,H,N,d] bf16 device, read only
- *   MQ, MK : [B,H,d,d] float64 device, written (row-major, symmetric)
+ *   MQ, MK : [B,H,d,d] float64 device, written (row-major, symmetric); either
+ *            may be NULL to skip that moment (q_reuse_k needs only M_K,
+ *            k_reuse_q only M_Q; spark_forward forms only what its layout needs)
  *   qmean  : [B,H,d] float64 device, written
  *   ws     : workspace of spark_workspace_size() bytes (scratch) */
 spark_status spark_moments(const spark_params* p, const void* q, const void* k,
@@ -128,19 +134,23 @@ spark_status spark_moments(const spark_params* p, const void* q, const void* k,
  * this is a convenience of this library for callers that cannot allocate or
  * lend device memory - for example code embedded in a host framework that
  * owns every device allocation and forbids new ones on its hot path, or a
- * caller with a fixed memory plan and no workspace to hand over. It computes
- * exactly what spark_moments computes (same kernels), but keeps the partial
- * sums in a fixed device array inside the library instead of a workspace.
+ * caller with a fixed memory plan and no workspace to hand over. It runs the
+ * kernels spark_moments runs (float64 Gram sums and anchor), but keeps the
+ * partial sums in a fixed device array inside the library instead of a
+ * workspace, and always forms both moments (MQ, MK and qmean must be non-NULL).
  *   - The array is SPARK_NOALLOC_SCRATCH_BYTES (16 MiB) per device; every GPU
  *     that loads the library holds it until the process exits.
  *   - Limit: 2 * B * H partial sums of (d*d + d) doubles must fit, i.e.
  *     B*H <= 63 for d = 128 and B*H <= 252 for d = 64; larger inputs return
  *     SPARK_ERR_UNSUPPORTED without launching anything. Within the limit the
- *     token range of a head is split into fewer chunks than spark_moments
- *     uses, so it can be slower.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     token range of a head may be cut into fewer chunks than spark_moments
+ *     uses, so it can be slower, and its float64 sums, added in another order,
+ *     can differ from spark_moments' in the last bits (a reblock run on them
+ *     can then, rarely, differ where a whitened value sits on a bf16 midpoint).
+ *   - Every call looks up the array's device address (cudaGetSymbolAddress)
+ *     with the current device, so it stays right after a device reset. That
+ *     lookup is a runtime call: make the first call on a device before any
+ *     stream capture.
  *   - All calls on a device share the one array and it keeps the last call's
  *     contents (nothing in it needs to start at zero: each call writes every
  *     partial before reading it). Calls whose kernels may overlap on the GPU
@@ -156,8 +166,12 @@ spark_status spark_moments_noalloc(const spark_params* p, const void* q, const v
  * for k_reuse_q, both in turn for separate) along the top principal direction of its whitened,
  * normalised vectors (Cholesky factor of the opposite side's moment),
  * split by rank into 64*floor(g/2) and the rest, down to 64-token leaves.
+ * The whitened tokens u = L^T x, their norms and the quotients u / |u| are
+ * float64 (float64 tensor cores) and each is rounded once to bf16, as a
+ * float64 evaluation of the definition rounds them.
  *   q, k   : [B,H,N,d] bf16 device, read only
- *   MQ, MK : from spark_moments, read only
+ *   MQ, MK : from spark_moments, read only; only the moment(s) the layout
+ *            uses must be non-NULL (M_K for q_reuse_k, M_Q for k_reuse_q)
  *   perm   : [B,H,N] int32 device, written: perm[pi] = original index of the
  *            token at permuted position pi; leaves in depth-first order,
  *            ascending original index inside each block. Q/K/V are never

@@ -32,7 +32,7 @@ import math
 
 import numpy as np
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_head", "bf16_bits_to_f64",
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_head", "host_procs", "bf16_bits_to_f64",
            "bf16_bits_to_f32", "f32_to_bf16_bits", "tiny_workload"]
 
 
@@ -149,18 +149,41 @@ def make_head(w: Workload, b: int, h: int):
     return f32_to_bf16_bits(q), f32_to_bf16_bits(k), f32_to_bf16_bits(vv)
 
 
-def make_inputs(w: Workload, heads=None):
+def _head_job(args):
+    w, b, h = args
+    return make_head(w, b, h)
+
+
+def make_inputs(w: Workload, heads=None, procs: int = 1):
     """Draw q, k, v as uint16 bf16 bit arrays of shape [B, H', N, d].
 
     heads: optional list of head indices (default: all H heads); batch items
-    are always all drawn.
+    are always all drawn. procs > 1 draws the heads in a pool of that many
+    fresh ("spawn") processes, which is safe after CUDA has been initialised
+    in this process; every head has its own seed, so the result is the same.
     """
     hs = list(range(w.H)) if heads is None else list(heads)
     shape = (w.B, len(hs), w.N, w.d)
     q = np.empty(shape, dtype=np.uint16)
     k = np.empty(shape, dtype=np.uint16)
     v = np.empty(shape, dtype=np.uint16)
-    for b in range(w.B):
-        for j, h in enumerate(hs):
-            q[b, j], k[b, j], v[b, j] = make_head(w, b, h)
+    jobs = [(w, b, h) for b in range(w.B) for h in hs]
+    if procs > 1 and len(jobs) > 1:
+        import multiprocessing as mp
+        with mp.get_context("spawn").Pool(min(procs, len(jobs))) as pool:
+            res = pool.map(_head_job, jobs)
+    else:
+        res = map(_head_job, jobs)
+    for (_, b, h), (qq, kk, vv) in zip(jobs, res):
+        j = hs.index(h)
+        q[b, j], k[b, j], v[b, j] = qq, kk, vv
     return q, k, v
+
+
+def host_procs() -> int:
+    """Host cores this process may use (for make_inputs' pool)."""
+    import os
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1

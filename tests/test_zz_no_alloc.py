@@ -39,7 +39,7 @@ def _compare(p, q, k):
         for a, b in ((MQ, MQ2), (MK, MK2)):
             a, b = a.cpu().numpy(), b.cpu().numpy()
             assert np.all(np.isfinite(b))
-            assert np.abs(a - b).max() <= 1e-6 * np.abs(a).max()
+            assert np.abs(a - b).max() <= 1e-12 * np.abs(a).max()
         a, b = qm.cpu().numpy(), qm2.cpu().numpy()
         assert np.abs(a - b).max() <= 1e-12 * (1 + np.abs(a).max())
 

@@ -27,12 +27,17 @@ __device__ __forceinline__ void dmma16816(double (&c)[4], const double (&a)[8], 
         "d"(b[0]), "d"(b[1]), "d"(b[2]), "d"(b[3]));
 }
 
-// Eight bf16 (one 16-byte chunk) widened to float64 and stored to shared memory.
-__device__ __forceinline__ void bf8_to_f64(const uint4 w, double* dst) {
-  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+// Eight bf16 (one 16-byte chunk) widened to float64 and stored to shared
+// memory as four 16-byte pairs. When the lanes of a warp hold consecutive
+// chunks of a row, their destinations are 64 bytes apart; each lane stores
+// its pairs in an order rotated by lane / 2, so that the eight lanes of a
+// quarter-warp hit eight different 16-byte bank groups at every step.
+__device__ __forceinline__ void bf8_to_f64(const uint4 w, double* dst, int lane) {
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    reinterpret_cast<double2*>(dst)[e] = make_double2((double)bf_lo(ws[e]), (double)bf_hi(ws[e]));
+  for (int i = 0; i < 4; ++i) {
+    const int e = (i + (lane >> 1)) & 3;
+    const uint32_t x = e == 0 ? w.x : e == 1 ? w.y : e == 2 ? w.z : w.w;
+    reinterpret_cast<double2*>(dst)[e] = make_double2((double)bf_lo(x), (double)bf_hi(x));
   }
 }
 

@@ -77,7 +77,7 @@ moments_gram64_kernel(const uint16_t* __restrict__ X, int N, int blocks_per_spli
 #pragma unroll
     for (int i = 0; i < SM::CPT; ++i) {
       const int c = tid + 256 * i, r = c / (D / 8), ch = c % (D / 8);
-      bf8_to_f64(pre[i], msm + buf * SM::TILE + r * LD + ch * 8);
+      bf8_to_f64(pre[i], msm + buf * SM::TILE + r * LD + ch * 8, lane);
     }
   };
 
@@ -175,8 +175,8 @@ moments_colsum_kernel(const uint16_t* __restrict__ X, int N, int blocks_per_spli
   if (tid < D) part[((size_t)bh * splits + split) * (size_t)(D * D + D) + D * D + tid] = csum;
 }
 
-// grid (B*H, 2 tensors): tensor 0 = q (its moment if gram_mask bit 0, and the
-// anchor), tensor 1 = k (its moment if gram_mask bit 1).
+// grid (B*H, 2 tensors, entry slices): tensor 0 = q (its moment if gram_mask
+// bit 0, and the anchor), tensor 1 = k (its moment if gram_mask bit 1).
 template <int D>
 __global__ void moments_reduce_kernel(const double* __restrict__ part, int splits, int N, double* __restrict__ MQ,
                                       double* __restrict__ MK, double* __restrict__ qmean, int gram_mask) {
@@ -185,7 +185,8 @@ __global__ void moments_reduce_kernel(const double* __restrict__ part, int split
   const double* src = part + (size_t)(t * BH + bh) * splits * (size_t)(D * D + D);
   double* M = (t == 0 ? MQ : MK) + (size_t)bh * D * D;
   const double dN = (double)N;
-  for (int e = threadIdx.x; e < D * D + D; e += blockDim.x) {
+  const int e0 = gram ? 0 : D * D;                    // without the moment only the column sums
+  for (int e = e0 + blockIdx.z * blockDim.x + threadIdx.x; e < D * D + D; e += gridDim.z * blockDim.x) {
     if (e < D * D) {
       if (!gram) continue;
       const int i = e / D, j = e % D;
@@ -223,8 +224,8 @@ static cudaError_t run_moments(const Plan& pl, const uint16_t* q, const uint16_t
     if (e != cudaSuccess) return e;
     moments_gram64_kernel<D, false><<<dim3(splits, pl.BH), 256, SM::bytes, s>>>(k, pl.N, bps, part + tstride);
   }
-  moments_reduce_kernel<D><<<dim3(pl.BH, 2), 256, 0, s>>>(part, splits, pl.N, MQ, MK, qmean,
-                                                          (gram_q ? 1 : 0) | (gram_k ? 2 : 0));
+  moments_reduce_kernel<D><<<dim3(pl.BH, 2, D / 8), 256, 0, s>>>(part, splits, pl.N, MQ, MK, qmean,
+                                                                 (gram_q ? 1 : 0) | (gram_k ? 2 : 0));
   return cudaGetLastError();
 }
 

@@ -12,7 +12,7 @@
 //
 // Kernels, in launch order:
 //   whiten_prep  : one CTA per head - regularise M, float64 Cholesky -> L (f64)
-//   normalize64  : persistent CTAs over 32-token tiles - U = X L in float64 on
+//   normalize64  : persistent CTAs over 16-token tiles - U = X L in float64 on
 //                  the float64 tensor cores, u_hat = bf16(u/|u|) from the
 //                  float64 quotient (the plain definition's value)
 //   tree_build   : node table (first block, g) per level; depends on nb only
@@ -97,149 +97,156 @@ whiten_prep_kernel(const double* __restrict__ M, double* __restrict__ Lout, int*
 // u_j = sum_{i >= j} L[i][j] x_i, u_hat = bf16(u / |u|), evaluated as the
 // plain definition does: u in float64 (bf16 x widened, float64 factor,
 // float64 tensor cores, dmma.cuh), |u| = sqrt of the float64 sum of squares,
-// the quotient u_j / |u| by IEEE division and one rounding to bf16 (nearest,
-// ties to even). Up to float64 summation order this is the oracle's value, so
-// u_hat, the vectors every later split reads, agrees bit for bit except where
-// a quotient sits within a float64 rounding of a bf16 midpoint.
+// and each u_j / |u| rounded once to bf16 (nearest, ties to even). Up to
+// float64 summation order this is the oracle's value, so u_hat, the vectors
+// every later split reads, agrees bit for bit except where a quotient sits
+// within a float64 rounding of a bf16 midpoint.
 //
-// Persistent CTAs walk a contiguous range of (head, 32-token tile) items. The
-// head's factor L sits in shared memory in float64; token tiles are widened
-// to float64 in a double buffer, the next tile's global loads in flight
-// during the current tile's MMAs. Warp w owns the 16 tokens of m-tile w / 4
-// and a quarter of the outputs: the 8-column tiles {q, 7 - q, 8 + q, 15 - q}
-// (d = 128; {q, 7 - q} for d = 64), q = w % 4, which balances the work of the
-// triangular product (the k-chunks above the diagonal of L are skipped). The
-// quarters' partial norms meet in shared memory; rows are written back
-// through a bf16 staging tile with 16-byte stores.
+// The quotient: q = u_j * (1 / |u|) is within 3 float64 ulps of the IEEE
+// quotient u_j / |u|, so both round to the same bf16 unless q's 45 bits
+// below the bf16 precision lie within 8 units of the halfway pattern; only
+// then (practically never) is the division carried out. Away from a
+// midpoint, rounding q to nearest keeps its top 19 bits (sign, 11-bit
+// exponent, 7 mantissa bits) plus one when the dropped bits exceed half, the
+// carry running into the exponent; the exponent is then rebased from
+// float64 to bf16. Zero, and magnitudes outside the bf16 normal range, take
+// the library conversion instead.
+//
+// Persistent CTAs, one per SM, each take a balanced contiguous range of the
+// layer's (head, 16-token tile) items, in segments of one head: per segment
+// the CTA loads that head's factor L into shared memory (float64), then its
+// eight warps each take their own tiles of the segment: rows staged as bf16
+// through a warp-private cp.async double buffer, widened to float64 as the A
+// fragments are read, 72 of the 128 16x8x16 products of the tile (the
+// k-chunks above the diagonal of L are skipped), the row norms by shuffles
+// inside the warp, and the bf16 rows written back through the staging
+// buffer just consumed. CTA-wide barriers only around the loads of L.
 template <int D>
 struct NormSmem {
-  static constexpr int TT = 32;                       // tokens per tile
-  static constexpr int LD = D + 4;                    // float64 row stride (conflict-free fragments)
-  static constexpr int L_DBL = D * LD;
-  static constexpr int X_DBL = TT * LD;
-  static constexpr size_t off_x = sizeof(double) * L_DBL;
-  static constexpr size_t off_o = off_x + sizeof(double) * 2 * X_DBL;
-  static constexpr size_t bytes = off_o + sizeof(uint16_t) * TT * D;
-  static constexpr int CPT = TT * (D / 8) / 256;      // 16-byte input chunks per thread and tile
-  static constexpr int CPW = D / 8 / 4;               // 8-column output tiles per warp
-  static constexpr int KC = D / 16;                   // 16-wide k-chunks
+  static constexpr int LD = D + 4;                    // float64 row stride of L (conflict-free fragments)
+  static constexpr int RS = D + 8;                    // bf16 row stride of a staged tile
+  static constexpr int TOK = 16;                      // tokens per warp tile
+  static constexpr int WTILE = TOK * RS;              // bf16 elements per staged tile
+  static constexpr size_t off_x = sizeof(double) * D * LD;
+  static constexpr size_t bytes = off_x + sizeof(uint16_t) * 8 * 2 * WTILE;
+  static constexpr int CT = D / 8, KC = D / 16;
+  static constexpr int CH = TOK * (D / 8) / 32;       // 16-byte chunks per lane and tile
 };
+
+__device__ __forceinline__ uint32_t bf16_of_quotient(double u, double r, double rinv) {
+  const double qv = u * rinv;
+  const unsigned long long bits = (unsigned long long)__double_as_longlong(qv);
+  const long long low = (long long)(bits & ((1ull << 45) - 1));
+  const long long dist = low - (1ll << 44);
+  const unsigned long long top = (bits >> 45) + (dist > 0 ? 1ull : 0ull);   // sign | exp11 | mant7
+  const int e = (int)((top >> 7) & 0x7ff) - 896;                            // bf16 biased exponent
+  if (dist > 8 || dist < -8) {
+    if (e >= 1 && e <= 254) return (uint32_t)(((top >> 18) << 15) | ((unsigned)e << 7) | (top & 0x7f));
+    return (uint32_t)__bfloat16_as_ushort(__double2bfloat16(qv));
+  }
+  return (uint32_t)__bfloat16_as_ushort(__double2bfloat16(u / r));
+}
 
 template <int D>
 __global__ void __launch_bounds__(256, 1)
 normalize64_kernel(const uint16_t* __restrict__ X, const double* __restrict__ Lall, int N, int BH,
                    uint16_t* __restrict__ uhat) {
   using SM = NormSmem<D>;
-  constexpr int TT = SM::TT, LD = SM::LD, CPW = SM::CPW;
+  constexpr int LD = SM::LD, RS = SM::RS, TOK = SM::TOK, CT = SM::CT, KC = SM::KC;
   extern __shared__ __align__(16) unsigned char nsm_raw[];
   double* Ls = reinterpret_cast<double*>(nsm_raw);
-  double* Xs = reinterpret_cast<double*>(nsm_raw + SM::off_x);
-  uint16_t* Os = reinterpret_cast<uint16_t*>(nsm_raw + SM::off_o);
-  __shared__ double nsq[2][4][16];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
-  const int m = warp >> 2, q = warp & 3;
-  const int tpb = N / TT;
-  const long items = (long)BH * tpb;
-  const long per = (items + gridDim.x - 1) / gridDim.x;
-  const long it0 = (long)blockIdx.x * per, it1 = min(items, it0 + per);
-  if (it0 >= it1) return;
-  int cs[CPW];
-#pragma unroll
-  for (int j = 0; j < CPW; ++j) cs[j] = 8 * (j >> 1) + ((j & 1) ? 7 - q : q);
-
-  uint4 pre[SM::CPT];
-  auto fetch = [&](long it) {
-    const int bh = (int)(it / tpb), t0 = (int)(it % tpb) * TT;
-#pragma unroll
-    for (int i = 0; i < SM::CPT; ++i) {
-      const int c = tid + 256 * i, r = c / (D / 8), ch = c % (D / 8);
-      pre[i] = __ldg(reinterpret_cast<const uint4*>(X + ((size_t)bh * N + t0 + r) * D + ch * 8));
-    }
-  };
-  auto stash = [&](int buf) {
-#pragma unroll
-    for (int i = 0; i < SM::CPT; ++i) {
-      const int c = tid + 256 * i, r = c / (D / 8), ch = c % (D / 8);
-      bf8_to_f64(pre[i], Xs + buf * SM::X_DBL + r * LD + ch * 8);
-    }
-  };
-
-  int cur_bh = -1;
-  fetch(it0);
-  stash(0);
-  for (long it = it0; it < it1; ++it) {
-    const int buf = (int)((it - it0) & 1);
-    const int bh = (int)(it / tpb), t0 = (int)(it % tpb) * TT;
-    if (bh != cur_bh) {
-      // a new head's factor (every warp is past the previous tile's MMAs:
-      // the barrier at the end of the last iteration)
+  uint16_t* Xw = reinterpret_cast<uint16_t*>(nsm_raw + SM::off_x) + warp * 2 * SM::WTILE;
+  const int ntile = N / TOK;
+  const long items = (long)BH * ntile;
+  const long i0 = items * blockIdx.x / gridDim.x, i1 = items * (blockIdx.x + 1) / gridDim.x;
+  for (long seg = i0; seg < i1;) {
+    const int bh = (int)(seg / ntile);
+    const int c0 = (int)(seg - (long)bh * ntile);
+    const int c1 = (int)min((long)ntile, (long)c0 + (i1 - seg));
+    seg += c1 - c0;
+    __syncthreads();                                   // every warp is done with the previous head's L
+    {
       const double2* Lg = reinterpret_cast<const double2*>(Lall + (size_t)bh * D * D);
       for (int e = tid; e < D * D / 2; e += 256) {
         const int i = (2 * e) / D, j = (2 * e) % D;
         *reinterpret_cast<double2*>(Ls + i * LD + j) = Lg[e];
       }
-      cur_bh = bh;
     }
-    __syncthreads();                                    // tile `buf` and L are in place
-    if (it + 1 < it1) fetch(it + 1);
-    const double* xs = Xs + buf * SM::X_DBL + (16 * m) * LD;
-    double acc[CPW][4];
+    __syncthreads();
+    const uint16_t* Xh = X + (size_t)bh * N * D;
+    uint16_t* Uh = uhat + (size_t)bh * N * D;
+    auto load = [&](int t, int buf) {
 #pragma unroll
-    for (int j = 0; j < CPW; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[j][e] = 0.0;
-#pragma unroll
-    for (int kc = 0; kc < SM::KC; ++kc) {
-      // A = this m-tile's tokens x dims 16 kc..: a[i] = x[g + 8 (i % 2)][16 kc + t + 4 (i / 2)]
-      double a[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) a[i] = xs[(g + 8 * (i % 2)) * LD + 16 * kc + t4 + 4 * (i / 2)];
-#pragma unroll
-      for (int j = 0; j < CPW; ++j) {
-        if (kc < (cs[j] >> 1)) continue;               // L is zero above its diagonal (warp-uniform)
-        double b[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) b[i] = Ls[(16 * kc + t4 + 4 * i) * LD + 8 * cs[j] + g];
-        dmma16816(acc[j], a, b);
+      for (int i = 0; i < SM::CH; ++i) {
+        const int c = lane + 32 * i, r = c / (D / 8), ch = c % (D / 8);
+        cp_async16(Xw + buf * SM::WTILE + r * RS + ch * 8, Xh + ((size_t)t * TOK + r) * D + ch * 8);
       }
-    }
-    // |u|^2 of tokens g and g + 8 of the m-tile: this warp's columns, then the quarters
-    double s0 = 0.0, s1 = 0.0;
-#pragma unroll
-    for (int j = 0; j < CPW; ++j) {
-      s0 = fma(acc[j][0], acc[j][0], s0);
-      s0 = fma(acc[j][1], acc[j][1], s0);
-      s1 = fma(acc[j][2], acc[j][2], s1);
-      s1 = fma(acc[j][3], acc[j][3], s1);
-    }
-    s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
-    s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
-    s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
-    s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
-    if (t4 == 0) {
-      nsq[m][q][g] = s0;
-      nsq[m][q][g + 8] = s1;
-    }
-    __syncthreads();
-    const double n0 = (nsq[m][0][g] + nsq[m][1][g]) + (nsq[m][2][g] + nsq[m][3][g]);
-    const double n1 = (nsq[m][0][g + 8] + nsq[m][1][g + 8]) + (nsq[m][2][g + 8] + nsq[m][3][g + 8]);
-    const double r0 = sqrt(n0), r1 = sqrt(n1);
-    auto q2 = [](double u, double r) -> uint32_t {
-      return r > 0.0 ? (uint32_t)__bfloat16_as_ushort(__double2bfloat16(u / r)) : 0u;
     };
+    int t = c0 + warp, buf = 0;
+    if (t < c1) load(t, 0);
+    cp_async_commit();
+    for (; t < c1; t += 8, buf ^= 1) {
+      if (t + 8 < c1) load(t + 8, buf ^ 1);
+      cp_async_commit();
+      cp_async_wait<1>();
+      __syncwarp();
+      const uint16_t* xs = Xw + buf * SM::WTILE;
+      double acc[CT][4];
 #pragma unroll
-    for (int j = 0; j < CPW; ++j) {
-      const int col = 8 * cs[j] + 2 * t4;
-      *reinterpret_cast<uint32_t*>(Os + (16 * m + g) * D + col) = q2(acc[j][0], r0) | (q2(acc[j][1], r0) << 16);
-      *reinterpret_cast<uint32_t*>(Os + (16 * m + g + 8) * D + col) = q2(acc[j][2], r1) | (q2(acc[j][3], r1) << 16);
+      for (int c = 0; c < CT; ++c)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[c][e] = 0.0;
+#pragma unroll
+      for (int kc = 0; kc < KC; ++kc) {
+        // A = the tile's tokens x dims 16 kc..: a[i] = x[g + 8 (i % 2)][16 kc + t + 4 (i / 2)]
+        double a[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] = (double)bf2f(xs[(g + 8 * (i % 2)) * RS + 16 * kc + t4 + 4 * (i / 2)]);
+#pragma unroll
+        for (int c = 0; c < CT; ++c) {
+          if (kc < (c >> 1)) continue;                   // L is zero above its diagonal
+          double b[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) b[i] = Ls[(16 * kc + t4 + 4 * i) * LD + 8 * c + g];
+          dmma16816(acc[c], a, b);
+        }
+      }
+      // |u|^2 of tokens g and g + 8: this lane's columns, then the 4 lanes of the row
+      double s0 = 0.0, s1 = 0.0;
+#pragma unroll
+      for (int c = 0; c < CT; ++c) {
+        s0 = fma(acc[c][0], acc[c][0], s0);
+        s0 = fma(acc[c][1], acc[c][1], s0);
+        s1 = fma(acc[c][2], acc[c][2], s1);
+        s1 = fma(acc[c][3], acc[c][3], s1);
+      }
+      s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+      s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+      s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+      s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+      const double r0 = sqrt(s0), r1 = sqrt(s1);
+      const double i0 = r0 > 0.0 ? 1.0 / r0 : 0.0, i1 = r1 > 0.0 ? 1.0 / r1 : 0.0;
+      __syncwarp();                                      // every lane is done reading the staged rows
+      uint16_t* os = Xw + buf * SM::WTILE;
+#pragma unroll
+      for (int c = 0; c < CT; ++c) {
+        const int col = 8 * c + 2 * t4;
+        const uint32_t w0 = r0 > 0.0 ? bf16_of_quotient(acc[c][0], r0, i0) | (bf16_of_quotient(acc[c][1], r0, i0) << 16) : 0u;
+        const uint32_t w1 = r1 > 0.0 ? bf16_of_quotient(acc[c][2], r1, i1) | (bf16_of_quotient(acc[c][3], r1, i1) << 16) : 0u;
+        *reinterpret_cast<uint32_t*>(os + g * RS + col) = w0;
+        *reinterpret_cast<uint32_t*>(os + (g + 8) * RS + col) = w1;
+      }
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < SM::CH; ++i) {
+        const int c = lane + 32 * i, r = c / (D / 8), ch = c % (D / 8);
+        *reinterpret_cast<uint4*>(Uh + ((size_t)t * TOK + r) * D + ch * 8) =
+            *reinterpret_cast<const uint4*>(os + r * RS + ch * 8);
+      }
+      __syncwarp();                                      // the buffer is refilled two tiles on
     }
-    if (it + 1 < it1) stash(buf ^ 1);
-    __syncthreads();
-    for (int c = tid; c < TT * (D / 8); c += 256) {
-      const int r = c / (D / 8), ch = c % (D / 8);
-      *reinterpret_cast<uint4*>(uhat + ((size_t)bh * N + t0 + r) * D + ch * 8) =
-          *reinterpret_cast<const uint4*>(Os + r * D + ch * 8);
-    }
+    cp_async_wait<0>();
   }
 }
 
@@ -1227,12 +1234,11 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
     int sms = 148;
     int dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const long items = (long)pl.BH * (pl.N / NormSmem<D>::TT);
-    const int grid = (int)std::min<long>(items, sms);
+    const long items = (long)pl.BH * (pl.N / NormSmem<D>::TOK);
     e = cudaFuncSetAttribute(normalize64_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)NormSmem<D>::bytes);
     if (e != cudaSuccess) return e;
-    normalize64_kernel<D><<<grid, 256, NormSmem<D>::bytes, s>>>(x, L, pl.N, pl.BH, uhat);
+    normalize64_kernel<D><<<(int)std::min<long>(items, sms), 256, NormSmem<D>::bytes, s>>>(x, L, pl.N, pl.BH, uhat);
   }
 
   tree_build_kernel<<<1, 1, 0, s>>>(pl.nb, nodes);

@@ -387,22 +387,13 @@ def joint_attention(q, k, v, perm, sel, kt, vt, beta, qc, kc, vc, rows=None, tai
         den = e_exact.sum(axis=1) + e_comp.sum(axis=1)
         out[qrow] = (e_exact @ vals + e_comp @ vt[~chosen]) / den[:, None]
         lse[qrow] = m + np.log(den)
-    outc, lsec = dense_attention_lse(qc, np.concatenate([k, kc]), np.concatenate([v, vc]))
+    outc, lsec = dense_attention(qc, np.concatenate([k, kc]), np.concatenate([v, vc]))
     return out, lse, outc, lsec
 
 
-def dense_attention_lse(q, k, v):
-    """Plain softmax attention with its natural-log denominators."""
-    q = np.asarray(q, dtype=np.float64)
-    s = q @ np.asarray(k, dtype=np.float64).T / math.sqrt(q.shape[1])
-    m = s.max(axis=1, keepdims=True)
-    e = np.exp(s - m)
-    den = e.sum(axis=1, keepdims=True)
-    return e @ np.asarray(v, dtype=np.float64) / den, (m + np.log(den))[:, 0]
-
-
 def dense_attention(q, k, v):
-    """Plain softmax attention, the density-1.0 limit of the method."""
+    """Plain softmax attention (the density-1.0 limit of the method) and its
+    natural-log denominators (lse)."""
     q = np.asarray(q, dtype=np.float64)
     s = q @ np.asarray(k, dtype=np.float64).T / math.sqrt(q.shape[1])
     m = s.max(axis=1, keepdims=True)
@@ -454,17 +445,19 @@ def forward_head(q, k, v, ratio=0.2, topk_blocks=0, layout="q_reuse_k",
 # --------------------------------------------------------------------------
 # statistics the pages name (oracle only)
 
-def mass_recall(q, k, perm, sel, rows):
+def mass_recall(q, k, perm, sel, rows, perm_k=None):
     """R12: attention-mass recall ([P2] "+12.88 points of attention-mass
     recall"): for each sampled query, the share (in percent) of its dense
     softmax mass that falls on keys of its selected blocks. rows: permuted
-    query blocks to sample. Returns the mean over their queries."""
+    query blocks to sample; perm_k: the key permutation (default perm; the
+    separate layout's key blocks, R16). Returns the mean over their queries."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
+    perm_k = perm if perm_k is None else perm_k
     N, d = q.shape
     nb = N // BLOCK
     blk = np.empty(N, dtype=np.int64)
-    blk[perm] = np.arange(N) // BLOCK
+    blk[perm_k] = np.arange(N) // BLOCK
     vals = []
     for a in rows:
         Qa = q[perm[a * BLOCK:(a + 1) * BLOCK]]
@@ -476,16 +469,19 @@ def mass_recall(q, k, perm, sel, rows):
     return float(np.concatenate(vals).mean())
 
 
-def log_mass_error(q, k, perm, sel, kt, beta, rows):
+def log_mass_error(q, k, perm, sel, kt, beta, rows, perm_k=None):
     """R12: absolute log-mass error ([P2] "-28% absolute log-mass error"):
-    mean over sampled queries i and unselected blocks b of
-    |(q_i . k~_b / sqrt(d) + beta_b) - ln sum_{j in b} exp(q_i . k_j / sqrt(d))|."""
+    the plain (unweighted) mean over sampled queries i and unselected blocks b
+    of |(q_i . k~_b / sqrt(d) + beta_b) - ln sum_{j in b} exp(q_i . k_j / sqrt(d))|.
+    Key block b is block b of perm_k (default perm; the separate layout's key
+    permutation, R16)."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
+    perm_k = perm if perm_k is None else perm_k
     N, d = q.shape
     nb = N // BLOCK
     scale = 1.0 / math.sqrt(d)
-    Kb = k[perm].reshape(nb, BLOCK, d)
+    Kb = k[perm_k].reshape(nb, BLOCK, d)
     errs = []
     for a in rows:
         Qa = q[perm[a * BLOCK:(a + 1) * BLOCK]]

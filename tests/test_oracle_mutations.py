@@ -11,7 +11,7 @@ from oracle import spark_oracle as so
 
 _orig = {name: getattr(so, name) for name in
          ("summaries", "whitening_factor", "split_direction", "select", "attention",
-          "split_group", "round_bf16", "block_means", "dense_attention_lse")}
+          "split_group", "round_bf16", "block_means", "dense_attention", "log_mass_error")}
 
 
 def _beta_without_anchor_term(k, v, perm, qbar, mode="reweight"):
@@ -58,12 +58,40 @@ def _block_tail_from_head_anchor(q, k, v, perm, sel, kt, vt, beta, rows=None, ta
 
 def _context_rows_without_context_keys(q, k, v):
     # context queries that only see the video keys (the context segment dropped)
-    return _orig["dense_attention_lse"](q, k[: len(k) - len(k) % 64], v[: len(v) - len(v) % 64])
+    return _orig["dense_attention"](q, k[: len(k) - len(k) % 64], v[: len(v) - len(v) % 64])
 
 
 def _keys_through_query_perm(q, k, v, perm, sel, kt, vt, beta, rows=None, perm_k=None, **kw):
     # separate layout: key blocks looked up through the query permutation
     return _orig["attention"](q, k, v, perm, sel, kt, vt, beta, rows, perm_k=perm, **kw)
+
+
+def _signed_log_mass_error(q, k, perm, sel, kt, beta, rows, perm_k=None):
+    # the error without its absolute value (signed deviations cancel)
+    d = q.shape[1]
+    out = []
+    for a in rows:
+        Qa = q[perm[64 * a:64 * (a + 1)]]
+        for b in np.setdiff1d(np.arange(len(q) // 64), sel[a]):
+            s = Qa @ k[(perm if perm_k is None else perm_k)[64 * b:64 * (b + 1)]].T / math.sqrt(d)
+            true = np.log(np.exp(s).sum(axis=1))
+            out.append(Qa @ kt[b] / math.sqrt(d) + beta[b] - true)
+    return float(np.concatenate(out).mean())
+
+
+def _mass_weighted_log_mass_error(q, k, perm, sel, kt, beta, rows, perm_k=None):
+    # the error averaged with each (query, block)'s true softmax mass as weight
+    d = q.shape[1]
+    num = den = 0.0
+    for a in rows:
+        Qa = q[perm[64 * a:64 * (a + 1)]]
+        for b in np.setdiff1d(np.arange(len(q) // 64), sel[a]):
+            s = Qa @ k[(perm if perm_k is None else perm_k)[64 * b:64 * (b + 1)]].T / math.sqrt(d)
+            true = np.log(np.exp(s).sum(axis=1))
+            w = np.exp(true)
+            num += float((w * np.abs(Qa @ kt[b] / math.sqrt(d) + beta[b] - true)).sum())
+            den += float(w.sum())
+    return num / den
 
 
 def _truncating_round(x):
@@ -93,11 +121,13 @@ MUTANTS = [
     ("attention", _attention_unscaled, [pins.test_density_one_is_dense_attention]),
     ("attention", _block_tail_from_head_anchor,
      [lambda: pins.test_block_tail_matches_brute_force(256, 8, 0.25, "reweight")]),
-    ("dense_attention_lse", _context_rows_without_context_keys,
+    ("dense_attention", _context_rows_without_context_keys,
      [lambda: pins.test_joint_attention_matches_brute_force(128, 8, 0.5, 7)]),
     ("attention", _keys_through_query_perm,
      [lambda: pins.test_separate_layout_matches_brute_force(256, 8, 0.25, "reweight")]),
     ("round_bf16", _truncating_round, [pins.test_round_bf16_matches_bit_rounding]),
+    ("log_mass_error", _signed_log_mass_error, [pins.test_log_mass_error_brute_force]),
+    ("log_mass_error", _mass_weighted_log_mass_error, [pins.test_log_mass_error_brute_force]),
     ("split_group", _split_ceil_left, [pins.test_split_group_orientation_and_capacity]),
 ]
 

@@ -544,11 +544,11 @@ def test_joint_attention_lse_merge():
     res = so.forward_head(q, k, v, ratio=0.25)
     out, lse, _, _ = so.joint_attention(q, k, v, res["perm"], res["sel"], res["kt"], res["vt"], res["beta"],
                                         qc, kc, vc)
-    _, lse_ctx = so.dense_attention_lse(q, kc, vc)
+    _, lse_ctx = so.dense_attention(q, kc, vc)
     merged = np.logaddexp(res["lse"], lse_ctx)
     assert np.allclose(lse, merged, rtol=1e-12, atol=1e-12)
     # and the output is the matching convex combination of the two partial outputs
-    o_ctx, _ = so.dense_attention_lse(q, kc, vc)
+    o_ctx, _ = so.dense_attention(q, kc, vc)
     w = np.exp(res["lse"] - lse)[:, None]
     assert np.allclose(out, w * res["out"] + (1 - w) * o_ctx, rtol=1e-10, atol=1e-12)
 
@@ -606,6 +606,54 @@ def test_log_mass_error_zero_for_identical_keys():
     res = _run(q, kb, r.standard_normal((64 * nb, d)), 0.25, np.arange(64 * nb))
     e = so.log_mass_error(q, kb, res["perm"], res["sel"], res["kt"], res["beta"], range(nb))
     assert e < 1e-12
+
+
+def test_log_mass_error_brute_force():
+    """Every (query, unselected block) pair spelled out with math.fsum over
+    the 64 exponentials and math.log, then the plain mean of the absolute
+    differences ([P2] "absolute log-mass error")."""
+    q, k, v = rand_qkv(256, 8, seed=31, scale=2)
+    r = _run(q, k, v, 0.25)
+    perm, sel, kt, beta = r["perm"], r["sel"], r["kt"], r["beta"]
+    rows = [0, 2, 3]
+    errs = []
+    for a in rows:
+        for i in perm[64 * a:64 * (a + 1)]:
+            for b in range(4):
+                if b in set(sel[a].tolist()):
+                    continue
+                keys = perm[64 * b:64 * (b + 1)]
+                true = math.log(math.fsum(math.exp(float(q[i] @ k[j]) / math.sqrt(8)) for j in keys))
+                pooled = float(q[i] @ kt[b]) / math.sqrt(8) + float(beta[b])
+                errs.append(abs(pooled - true))
+    assert len(errs) == 3 * 64 * 3
+    assert so.log_mass_error(q, k, perm, sel, kt, beta, rows) == pytest.approx(math.fsum(errs) / len(errs),
+                                                                              rel=1e-12)
+
+
+def test_statistics_take_the_key_permutation():
+    """Separate layout (R16): key block b is block b of the key permutation,
+    for both statistics."""
+    q, k, v = rand_qkv(256, 8, seed=32, scale=2)
+    r = so.forward_head(q, k, v, ratio=0.25, layout="separate")
+    pq, pk = r["perm"], r["perm_k"]
+    assert not np.array_equal(pq, pk)
+    rows = [0, 1]
+    s = q @ k.T / math.sqrt(8)
+    P = np.exp(s - s.max(axis=1, keepdims=True))
+    P /= P.sum(axis=1, keepdims=True)
+    kblk = np.empty(256, dtype=int)
+    kblk[pk] = np.arange(256) // 64
+    rec = [100 * P[i, np.isin(kblk, r["sel"][a])].sum() for a in rows for i in pq[64 * a:64 * (a + 1)]]
+    assert so.mass_recall(q, k, pq, r["sel"], rows, perm_k=pk) == pytest.approx(np.mean(rec), rel=1e-12)
+    errs = []
+    for a in rows:
+        for i in pq[64 * a:64 * (a + 1)]:
+            for b in sorted(set(range(4)) - set(r["sel"][a].tolist())):
+                true = math.log(math.fsum(math.exp(float(q[i] @ k[j]) / math.sqrt(8)) for j in pk[64 * b:64 * (b + 1)]))
+                errs.append(abs(float(q[i] @ r["kt"][b]) / math.sqrt(8) + float(r["beta"][b]) - true))
+    got = so.log_mass_error(q, k, pq, r["sel"], r["kt"], r["beta"], rows, perm_k=pk)
+    assert got == pytest.approx(math.fsum(errs) / len(errs), rel=1e-12)
 
 
 @pytest.mark.parametrize("summary", ["reweight", "meanpool"])

@@ -14,7 +14,7 @@ import os
 __all__ = ["SparkError", "Params", "lib", "params", "num_selected", "workspace_size",
            "host_workspace_size", "workspace_region", "alloc_workspace", "moments", "reblock",
            "positional_perm", "select", "attn_fwd", "attn_fwd_joint", "forward", "forward_joint",
-           "forward_host", "get_status",
+           "forward_host", "get_status", "selftest_wait",
            "LAYOUTS", "SUMMARIES", "TAILS", "WS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -74,6 +74,7 @@ _SIGS = {
                                    _vp]),
     "spark_forward_host": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "spark_get_status": (_i32, [_vp]),
+    "spark_selftest_wait": (_i32, [ctypes.c_int64, _vp]),
     "spark_strerror": (ctypes.c_char_p, [_i32]),
 }
 
@@ -316,6 +317,12 @@ def forward_host(p: Params, q_host, k_host, v_host, out_host, ws, lse_host=None)
                                     _ptr(out_host), _ptr(lse_host), _ptr(ws), ws.numel(),
                                     _stream()), "spark_forward_host")
     return out_host
+
+
+def selftest_wait(limit_ns: int):
+    """Launch the bounded-wait diagnostic (see include/spark.h); the timeout
+    shows up in the next get_status()."""
+    _check(lib().spark_selftest_wait(int(limit_ns), _stream()), "spark_selftest_wait")
 
 
 def get_status():

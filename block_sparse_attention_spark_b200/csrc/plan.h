@@ -71,6 +71,8 @@ cudaError_t launch_positional(const Plan& pl, int F, int Hl, int Wl, int32_t* pe
 cudaError_t launch_select(const Plan& pl, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                           const int32_t* perm, const double* qmean, int32_t* sel, int summary,
                           void* ws, int* status, cudaStream_t s);
+// Diagnostic: a bounded wait that expires (see spark_selftest_wait).
+cudaError_t launch_selftest_wait(unsigned long long limit_ns, int* status, cudaStream_t s);
 // Context segment of joint attention: qc, kc, vc [BH, C, d] bf16 (C >= 1);
 // outc [BH, C, d] bf16, lsec [BH, C] float32 or null.
 struct JointContext {

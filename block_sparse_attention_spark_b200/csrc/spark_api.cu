@@ -427,13 +427,23 @@ spark_status spark_forward_host(const spark_params* p, const void* q_host, const
   const size_t head_bytes = (size_t)pl.N * pl.d * 2;   // one head of q, k, v or out
   const int nch = std::min(pl.BH, HOST_CHUNKS);
 
+  // every chunk is a problem of its own (B = 1, H = its heads) run in this
+  // workspace: check them all before anything is queued
+  auto head0 = [&](int c) { return (int)(((long)pl.BH * c) / nch); };
+  for (int c = 0; c < nch; ++c) {
+    spark_params pc = *p;
+    pc.B = 1;
+    pc.H = head0(c + 1) - head0(c);
+    Plan plc;
+    if (validate(&pc) != SPARK_OK || !make_plan(&pc, &plc)) return SPARK_ERR_INVALID_ARG;
+    if (plc.total > pl.total) return SPARK_ERR_WORKSPACE;
+  }
   std::lock_guard<std::mutex> guard(g_host_mu);
   HostPipe* hp = host_pipe();
   if (hp == nullptr) return SPARK_ERR_CUDA;
   if (cudaEventRecord(hp->entry, stream) != cudaSuccess) return SPARK_ERR_CUDA;
   if (cudaStreamWaitEvent(hp->h2d, hp->entry, 0) != cudaSuccess) return SPARK_ERR_CUDA;
   if (cudaStreamWaitEvent(hp->d2h, hp->entry, 0) != cudaSuccess) return SPARK_ERR_CUDA;
-  auto head0 = [&](int c) { return (int)(((long)pl.BH * c) / nch); };
   for (int c = 0; c < nch; ++c) {
     const size_t off = (size_t)head0(c) * head_bytes, len = (size_t)(head0(c + 1) - head0(c)) * head_bytes;
     if (cudaMemcpyAsync(dq + off, (const char*)q_host + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
@@ -489,6 +499,11 @@ size_t spark_workspace_region(const spark_params* p, int32_t region, size_t* byt
   }
   if (bytes) *bytes = sz;
   return off;
+}
+
+spark_status spark_selftest_wait(int64_t limit_ns, cudaStream_t stream) {
+  if (limit_ns < 1 || limit_ns > 2000000000ll) return SPARK_ERR_INVALID_ARG;
+  return cuda_status(launch_selftest_wait((unsigned long long)limit_ns, status_ptr(), stream));
 }
 
 spark_status spark_get_status(cudaStream_t stream) {

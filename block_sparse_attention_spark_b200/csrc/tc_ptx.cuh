@@ -48,17 +48,22 @@ __device__ __forceinline__ bool mbar_probe(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait; false (and a timeout bit in *status) if the phase never came.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* status) {
+// Bounded wait; false (and a timeout bit in *status) if the phase did not
+// come within limit_ns.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, int* status,
+                                              unsigned long long limit_ns) {
   if (mbar_test(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   while (!mbar_test(bar, parity)) {
-    if (globaltimer() - t0 > WAIT_NS) {
+    if (globaltimer() - t0 > limit_ns) {
       set_status(status, STATUS_TIMEOUT);
       return false;
     }
   }
   return true;
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* status) {
+  return mbar_wait_for(bar, parity, status, WAIT_NS);
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
   asm volatile(

@@ -295,6 +295,17 @@ enum {
 };
 size_t spark_workspace_region(const spark_params* p, int32_t region, size_t* bytes);
 
+/* Diagnostic (the pages have no counterpart): checks that a device-side
+ * timeout surfaces as an error and leaves the context usable. One warp
+ * allocates tensor memory, waits through the bounded-wait routine every
+ * kernel here uses on a barrier phase that nothing completes, gives up after
+ * limit_ns, sets the device status word, frees its tensor memory and
+ * returns; the next spark_get_status() reports SPARK_ERR_TIMEOUT and clears
+ * it. No fault, trap or endless loop is involved.
+ *   limit_ns : 1 .. 2e9 (the kernels' own limit is 2 s); outside that range
+ *              SPARK_ERR_INVALID_ARG, nothing launched. */
+spark_status spark_selftest_wait(int64_t limit_ns, cudaStream_t stream);
+
 /* Synchronises the stream, reads and clears the device status word:
  * SPARK_OK, SPARK_ERR_TIMEOUT (a bounded wait expired) or SPARK_ERR_CUDA. */
 spark_status spark_get_status(cudaStream_t stream);

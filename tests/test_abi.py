@@ -108,6 +108,11 @@ def test_entry_points_reject_null_and_small_workspace_without_launching():
     assert L.spark_moments(ctypes.byref(p), None, fake, fake, fake, fake, fake, n, None) == 1
     assert L.spark_moments(ctypes.byref(p), fake, fake, fake, fake, fake, fake, n - 1, None) == 3
     assert L.spark_reblock(ctypes.byref(p), fake, fake, fake, fake, None, fake, n, None) == 1
+    # q_reuse_k whitens the queries with M_K: M_K is required, M_Q is not read
+    assert L.spark_reblock(ctypes.byref(p), fake, fake, fake, None, fake, fake, n, None) == 1
+    # the bounded-wait diagnostic checks its limit before launching
+    assert L.spark_selftest_wait(0, None) == 1
+    assert L.spark_selftest_wait(3_000_000_000, None) == 1
     assert L.spark_select(ctypes.byref(p), fake, fake, fake, fake, fake, None, fake, n, None) == 1
     assert L.spark_attn_fwd(ctypes.byref(p), fake, fake, fake, None, None, n, None) == 1
     assert L.spark_attn_fwd(ctypes.byref(p), fake, fake, fake, None, fake, 16, None) == 3

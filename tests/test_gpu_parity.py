@@ -57,6 +57,23 @@ def run_stages(w, ratio=None, layout="q_reuse_k", summary="reweight", topk_block
     return res
 
 
+def check_beta(gk, gb, kt, beta, qbar, summary):
+    """The log-mass bias. Reweight ("Spark-H3" news post, Spark-Reweight
+    figure: the exp of the biased pooled logit is the block's E[exp x] at the
+    anchor) makes qbar . k~_b / sqrt(d) + beta_b = ln sum_{j in b} exp(x_j).
+    The GPU keeps that identity for the bf16 k~ it stores (and attention
+    reads), so its beta differs from the oracle's, formed with the unrounded
+    k~, by qbar . (rounding of k~) / sqrt(d); the identity itself is compared.
+    Mean pooling: beta = ln 64."""
+    d = gk.shape[1]
+    if summary == "meanpool":
+        assert np.abs(gb - beta).max() <= 1e-6
+        return
+    lnz_ref = kt @ qbar / math.sqrt(d) + beta
+    lnz_gpu = gk @ qbar / math.sqrt(d) + gb
+    assert np.abs(lnz_gpu - lnz_ref).max() <= 1e-4 * (1 + np.abs(lnz_ref).max())
+
+
 def check_head(r, b, h, layout="q_reuse_k", summary="reweight", rows=None, check_perm=True,
                report=None, tail="query", power_iters=so.POWER_ITERS):
     q = bf16_bits_to_f64(r["q"][b, h])
@@ -110,7 +127,7 @@ def check_head(r, b, h, layout="q_reuse_k", summary="reweight", rows=None, check
     gk, gv, gb = r["kt"][b, h, :nb], r["vt"][b, h, :nb], r["beta"][b, h, :nb]
     assert np.all(np.abs(gk - kt) <= 2 ** -8 * np.abs(kt) + 1e-6 * np.abs(kt).max())
     assert np.all(np.abs(gv - vt) <= 2 ** -8 * np.abs(vt) + 1e-6 * np.abs(vt).max())
-    assert np.abs(gb - beta).max() <= 1e-4 * (1 + np.abs(beta).max())
+    check_beta(gk, gb, kt, beta, qbar, summary)
     assert np.all(r["kt"][b, h, nb:] == 0) and np.all(r["beta"][b, h, nb:] == 0)
     # a4 selection, given the CUDA permutation
     ksel = spark.num_selected(p)
@@ -247,6 +264,65 @@ def test_joint_attention_context_segment(C):
     assert np.array_equal(bf16_to_f64(o2), out) and np.array_equal(bf16_to_f64(oc2), outc)
 
 
+def test_reweight_with_an_offset_anchor():
+    """Spark-Reweight with a mean query far from zero ("Spark-H3" news post,
+    What Spark-Attn changed, Spark-Reweight bullet and figure: the bias
+    restores E[exp x], which mean pooling replaces by exp E[x]). A common
+    offset c is added to every query so that the anchor logits qbar . k_j /
+    sqrt(d) spread by about three units inside a block; the GPU's k~, v~,
+    beta and outputs must match the oracle, and they must be far from what
+    mean pooling gives (a GPU that mean-pooled would fail here)."""
+    from spark_gen import f32_to_bf16_bits
+    w = tiny_workload("anchor", 2, (2, 16, 64), 128, 0.2, seed_index=1100)
+    q, k, v = make_inputs(w)
+    d = w.d
+    rng = np.random.default_rng(77)
+    for h in range(w.H):
+        kf, qf = bf16_bits_to_f64(k[0, h]), bf16_bits_to_f64(q[0, h])
+        u = rng.standard_normal(d)
+        u /= np.linalg.norm(u)
+        alpha = 3.0 * math.sqrt(d) / float(np.std(kf @ u))
+        q[0, h] = f32_to_bf16_bits((qf + alpha * u).astype(np.float32))
+    r = run_stages(w, qkv=(q, k, v))
+    nb = w.nb
+    for h in range(w.H):
+        check_head(r, 0, h)
+        qf, kf, vf = (bf16_bits_to_f64(x[0, h]) for x in (q, k, v))
+        perm = r["perm"][0, h].astype(np.int64)
+        qbar = so.anchor(qf)
+        x = (kf @ qbar) / math.sqrt(d)
+        spread = float(np.median([np.std(x[perm[64 * b:64 * (b + 1)]]) for b in range(nb)]))
+        assert spread > 1.5, spread
+        gk, gb = r["kt"][0, h, :nb], r["beta"][0, h, :nb]
+        kmean, _, bmean = so.summaries(kf, vf, perm, qbar, "meanpool")
+        beta_tol = 1e-4 * (1 + np.abs(gb).max())
+        assert np.abs(gb - bmean).max() > 100 * beta_tol           # beta far from ln 64
+        k_tol = 2 ** -8 * np.abs(gk) + 1e-6 * np.abs(gk).max()
+        assert (np.abs(gk - kmean) / k_tol).max() > 100             # k~ far from the block mean
+
+
+def test_forward_host_uneven_chunks_with_lse():
+    """spark_forward_host with B = 2, H = 5 (ten heads in four uneven chunks,
+    batch items flattened) and lse requested: out and lse equal
+    spark_forward's bit for bit."""
+    import torch
+    w = tiny_workload("hostchunks", 5, (2, 16, 32), 128, 0.2, seed_index=1200, B=2)
+    q, k, v = make_inputs(w)
+    p = spark.params(2, 5, w.N, w.d, w.ratio)
+    ws = spark.alloc_workspace(p)
+    lse = torch.empty(2, 5, w.N, dtype=torch.float32, device="cuda")
+    out = spark.forward(p, to_dev(q), to_dev(k), to_dev(v), ws=ws, lse=lse)
+    assert spark.get_status() == 0
+    hws = spark.alloc_workspace(p, host=True)
+    qh, kh, vh = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in (q, k, v))
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty(2, 5, w.N, dtype=torch.float32).pin_memory()
+    spark.forward_host(p, qh, kh, vh, oh, hws, lse_host=lh)
+    assert spark.get_status() == 0
+    assert torch.equal(oh, out.cpu())
+    assert torch.equal(lh, lse.cpu())
+
+
 def test_lite_reblock_power_iters():
     """The Lite reblock reading: 4 power iterations per split; every split is
     replayed by the oracle with the same count."""
@@ -372,7 +448,7 @@ def sampled_workload_check(w, ratio, pairs, rows_per_head=12, seed=7, qkv=None):
         gb = beta[b, h, :nb].cpu().numpy().astype(np.float64)
         assert np.all(np.abs(gk - rkt) <= 2 ** -8 * np.abs(rkt) + 1e-6 * np.abs(rkt).max())
         assert np.all(np.abs(gv - rvt) <= 2 ** -8 * np.abs(rvt) + 1e-6 * np.abs(rvt).max())
-        assert np.abs(gb - rbeta).max() <= 1e-4 * (1 + np.abs(rbeta).max())
+        check_beta(gk, gb, rkt, rbeta, qbar, "reweight")
         rows = sorted(rng.choice(nb, rows_per_head, replace=False).tolist()) + [nb - 1]
         ref, _ = so.attention(q, k, v, pm, sh, rkt, rvt, rbeta, rows=rows)
         mask = ~np.isnan(ref[:, 0])

@@ -17,7 +17,7 @@
 //                  float64 quotient (the plain definition's value)
 //   tree_build   : node table (first block, g) per level; depends on nb only
 //   init_idx     : identity token order
-//   big_gram / big_solve / big_project / big_select, per level above the
+//   big_gram / big_reduce / big_solve / big_project / big_select, per level above the
 //                  subtree level - chunked Gram sums of the groups (tcgen05
 //                  for d = 128, mma.sync for d = 64; float64 flush; right
 //                  halves derived from the parent level),
@@ -673,6 +673,24 @@ big_gram_tc_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restr
   tc::gram_tc_body<false>(X, [=](int tt, int r) { return ids[tt * BLK + r]; }, max(0, t1 - t0), out, status);
 }
 
+// The chunk partials of each group that has them, summed in chunk order
+// (c = 0, 1, ...) into chunk 0's slot: grid (entry slices, groups, heads),
+// every entry owned by one thread, so the reads and the in-place write do
+// not meet. big_solve then reads one Gram sum per group.
+template <int D>
+__global__ void __launch_bounds__(256)
+big_reduce_kernel(const int2* __restrict__ nodes, int nnodes, int chunks, int kstep, double* __restrict__ part) {
+  const int k = blockIdx.y * kstep, bh = blockIdx.z;
+  const int used = (nodes[k].y + BIG_CHUNK_TILES - 1) / BIG_CHUNK_TILES;
+  if (used <= 1) return;
+  double* src = part + (size_t)(bh * nnodes + k) * chunks * (size_t)(D * D + D);
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < D * D + D; e += gridDim.x * blockDim.x) {
+    double t = 0.0;
+    for (int c = 0; c < used; ++c) t += src[(size_t)c * (D * D + D) + e];
+    src[e] = t;
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(256, 1)
 big_solve_kernel(const int2* __restrict__ nodes, int nnodes, int chunks, const double* __restrict__ part,
@@ -690,7 +708,7 @@ big_solve_kernel(const int2* __restrict__ nodes, int nnodes, int chunks, const d
   const int n = node.y * BLK;
   const int ks = derive ? (k & ~1) : k;                    // node whose partials exist
   const bool right = derive && (k & 1);
-  const int used = (nodes[ks].y + BIG_CHUNK_TILES - 1) / BIG_CHUNK_TILES;
+  const int used = 1;                                      // big_reduce left the sum in chunk 0
   const double* src = part + (size_t)(bh * nnodes + ks) * chunks * (size_t)(D * D + D);
   const double* par = right ? gpar + (size_t)(bh * npar + (k >> 1)) * (size_t)(D * D + D) : nullptr;
   double* gsave = gout ? gout + (size_t)(bh * nnodes + k) * (size_t)(D * D + D) : nullptr;
@@ -1281,6 +1299,9 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
           uhat, pl.N, nd, cnt, ch, kstep, idx, bpart, status);
     else
       big_gram_kernel<D><<<dim3(ch, cnt / kstep, pl.BH), 256, smem_s, s>>>(uhat, pl.N, nd, cnt, ch, kstep, idx, bpart);
+    if (ch > 1)
+      big_reduce_kernel<D><<<dim3(std::min(16, (D * D + D + 255) / 256), cnt / kstep, pl.BH), 256, 0, s>>>(
+          nd, cnt, ch, kstep, bpart);
     big_solve_kernel<D><<<dim3(cnt, pl.BH), 256, smem_solve, s>>>(nd, cnt, ch, bpart, binfo, derive, gpar,
                                                                    derive ? pl.level_count[lv - 1] : 0, gout,
                                                                    pl.power_iters);

@@ -195,13 +195,17 @@ size_t spark_workspace_size(const spark_params* p) {
 int32_t spark_forward_launches(const spark_params* p) {
   Plan pl;
   if (!make_plan(p, &pl)) return -1;
-  // moments 2; reblock: whiten, normalise, tree, init, split levels, subtree, leaves;
-  // select: block statistics, then scores + top-K per chunk of heads; attention 1
+  // moments: one Gram per moment the layout uses, the anchor's column sums
+  // when the query moment is not formed, the reduce; reblock: whiten,
+  // normalise, tree, init, per split level Gram (+ reduce of chunk partials),
+  // solve, project, select, then subtree and leaves; select: block
+  // statistics, then scores + top-K per chunk of heads; attention 1
+  const int moments = (pl.layout == SPARK_LAYOUT_K_REUSE_Q) ? 2 : 3;
   int split_launches = 0;
-  for (int lv = 0; lv < pl.sub_level; ++lv) split_launches += 4;
+  for (int lv = 0; lv < pl.sub_level; ++lv) split_launches += 4 + (pl.level_chunks[lv] > 1 ? 1 : 0);
   const int reblock = pl.nperm * (4 + split_launches + (pl.sub_level < pl.nlevels ? 1 : 0) + 1);
   const int select = 1 + 2 * ((pl.BH + pl.score_heads - 1) / pl.score_heads) + (pl.tail == SPARK_TAIL_BLOCK ? 1 : 0);
-  return 2 + reblock + select + 1;
+  return moments + reblock + select + 1;
 }
 
 size_t spark_host_workspace_size(const spark_params* p) {

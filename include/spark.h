@@ -252,10 +252,12 @@ spark_status spark_forward(const spark_params* p, const void* q, const void* k, 
                            void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Number of kernel launches one spark_forward call makes for these params
- * (moments 2; reblock 5, plus 1 per tree level above the first level whose
- * groups all have at most 9 blocks - 4 for a level of few large groups that
- * are spread over chunk CTAs - plus 1 for the subtree pass; select 2;
- * attention 1); -1 if invalid. */
+ * (moments 2 or 3: a Gram per moment the layout uses, column sums for the
+ * anchor when M_Q is not formed, a reduce; per partition, reblock 6 - whiten,
+ * normalise, tree, init, subtree, leaves - plus 4 per tree level above the
+ * first level whose groups all have at most 9 blocks, 5 when that level's
+ * groups span several chunk CTAs; select 1 + 2 per chunk of heads (+1 for
+ * the block tail); attention 1); -1 if invalid. */
 int32_t spark_forward_launches(const spark_params* p);
 
 /* Device bytes spark_forward_host needs: spark_workspace_size() plus room

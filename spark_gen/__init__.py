@@ -161,6 +161,9 @@ def make_inputs(w: Workload, heads=None, procs: int = 1):
     are always all drawn. procs > 1 draws the heads in a pool of that many
     fresh ("spawn") processes, which is safe after CUDA has been initialised
     in this process; every head has its own seed, so the result is the same.
+    A spawned worker imports the calling program's main module again, so a
+    script that calls this with procs > 1 must keep its top-level work under
+    `if __name__ == "__main__":` (pytest's and bench.py's entry points do).
     """
     hs = list(range(w.H)) if heads is None else list(heads)
     shape = (w.B, len(hs), w.N, w.d)

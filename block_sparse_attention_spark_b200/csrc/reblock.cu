@@ -254,18 +254,30 @@ normalize64_kernel(const uint16_t* __restrict__ X, const double* __restrict__ La
 // Nodes that split, level by level: (first block, g blocks). Same recursion
 // as the host side make_plan() uses for the counts.
 __global__ void tree_build_kernel(int nb, int2* nodes) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  // one warp: each level's nodes in rounds of 32, every lane emitting the
+  // children (0, 1 or 2) of one node, placed in node order by ballot counts
+  if (blockIdx.x != 0 || threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
+  if (lane == 0) nodes[0] = make_int2(0, nb);
+  __syncwarp();
   int count = 1, off = 0;
-  nodes[0] = make_int2(0, nb);
   while (count > 0) {
-    int nxt = 0;
     const int base = off + count;
-    for (int i = 0; i < count; ++i) {
-      const int2 nd = nodes[off + i];
+    int nxt = 0;
+    for (int i0 = 0; i0 < count; i0 += 32) {
+      const int i = i0 + lane;
+      int2 nd = make_int2(0, 0);
+      if (i < count) nd = nodes[off + i];
       const int gl = nd.y / 2, gr = nd.y - nd.y / 2;
-      if (gl >= 2) nodes[base + nxt++] = make_int2(nd.x, gl);
-      if (gr >= 2) nodes[base + nxt++] = make_int2(nd.x + gl, gr);
+      const bool el = i < count && gl >= 2, er = i < count && gr >= 2;
+      const unsigned bl = __ballot_sync(0xffffffffu, el), br = __ballot_sync(0xffffffffu, er);
+      const unsigned below = (1u << lane) - 1u;
+      int pos = base + nxt + __popc(bl & below) + __popc(br & below);
+      if (el) nodes[pos++] = make_int2(nd.x, gl);
+      if (er) nodes[pos] = make_int2(nd.x + gl, gr);
+      nxt += __popc(bl) + __popc(br);
     }
+    __syncwarp();
     off = base;
     count = nxt;
   }
@@ -1259,7 +1271,7 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
     normalize64_kernel<D><<<(int)std::min<long>(items, sms), 256, NormSmem<D>::bytes, s>>>(x, L, pl.N, pl.BH, uhat);
   }
 
-  tree_build_kernel<<<1, 1, 0, s>>>(pl.nb, nodes);
+  tree_build_kernel<<<1, 32, 0, s>>>(pl.nb, nodes);
   const long total = (long)pl.BH * pl.N;
   init_idx_kernel<<<(int)std::min<long>((total + 255) / 256, 4096), 256, 0, s>>>(idx, pl.N, total);
 

@@ -984,27 +984,34 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
     }
   }
   __syncthreads();
-  // S = G / n - mu mu^T on this thread's fragment entries (float64)
+  // S = G / n - mu mu^T on this thread's fragment entries, formed in float64
+  // and kept in float32: a subtree's groups are small and its Gram sums are
+  // float32 already, and float32 steps halve the latency-bound iteration
+  // (the direction is scale-free, so rescaling v by an approximate norm every
+  // NORM_EVERY_F32 steps changes nothing; two unscaled float32 steps stay far
+  // from underflow for any nonzero covariance of distinct bf16 unit vectors).
+  constexpr int NORM_EVERY_F32 = 2;
   const double invn = 1.0 / (double)nn;
-  double S[G::ACC];
+  float S[G::ACC];
 #pragma unroll
   for (int j = 0; j < G::ACC; ++j) {
     int row, col;
     G::coord(j, warp, lane, row, col);
-    S[j] = (double)acc[j] * invn - mus[row] * mus[col];
+    S[j] = (float)((double)acc[j] * invn - mus[row] * mus[col]);
   }
   // power iteration in the fragment layout: rows m0 + mt*16 + lane/4 + 8h,
   // columns n0 + nt*8 + 2 (lane % 4) + e
-  double vl[G::NT * 2];
+  float vl[G::NT * 2];
 #pragma unroll
-  for (int j = 0; j < G::NT * 2; ++j) vl[j] = 1.0 / sqrt((double)D);
+  for (int j = 0; j < G::NT * 2; ++j) vl[j] = 1.0f;
   bool zero_dir = false;
+  float* zpf = reinterpret_cast<float*>(zp);
   for (int iter = 0; iter < iters; ++iter) {
-    double* z = zp + (iter & 1) * 2 * D;        // [wn][row]: the two column halves' partial sums
-    const bool norm_step = (iter % NORM_EVERY) == NORM_EVERY - 1 || iter == iters - 1;
-    double zr[G::MT][2];
+    float* z = zpf + (iter & 1) * 2 * D;         // [wn][row]: the two column halves' partial sums
+    const bool norm_step = (iter % NORM_EVERY_F32) == NORM_EVERY_F32 - 1 || iter == iters - 1;
+    float zr[G::MT][2];
 #pragma unroll
-    for (int mt = 0; mt < G::MT; ++mt) { zr[mt][0] = 0.0; zr[mt][1] = 0.0; }
+    for (int mt = 0; mt < G::MT; ++mt) { zr[mt][0] = 0.f; zr[mt][1] = 0.f; }
 #pragma unroll
     for (int nt = 0; nt < G::NT; ++nt)
 #pragma unroll
@@ -1012,7 +1019,7 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
 #pragma unroll
         for (int mt = 0; mt < G::MT; ++mt)
 #pragma unroll
-          for (int h = 0; h < 2; ++h) zr[mt][h] = fma(S[(mt * G::NT + nt) * 4 + 2 * h + e], vl[nt * 2 + e], zr[mt][h]);
+          for (int h = 0; h < 2; ++h) zr[mt][h] = fmaf(S[(mt * G::NT + nt) * 4 + 2 * h + e], vl[nt * 2 + e], zr[mt][h]);
 #pragma unroll
     for (int o = 1; o <= 2; o <<= 1)
 #pragma unroll
@@ -1026,33 +1033,33 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
         for (int h = 0; h < 2; ++h) z[wn * D + m0 + mt * 16 + (lane >> 2) + 8 * h] = zr[mt][h];
     }
     __syncthreads();
-    double inv = 1.0;
+    float inv = 1.f;
     if (norm_step) {
       // every warp forms |z|^2 itself, in the same order: no second barrier
-      double sq = 0.0;
+      float sq = 0.f;
 #pragma unroll
       for (int k = 0; k < D / 32; ++k) {
-        const double zz = z[lane + 32 * k] + z[D + lane + 32 * k];
-        sq = fma(zz, zz, sq);
+        const float zz = z[lane + 32 * k] + z[D + lane + 32 * k];
+        sq = fmaf(zz, zz, sq);
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-      if (sq == 0.0) { zero_dir = true; break; }
-      inv = rsqrt(sq);
+      if (sq == 0.f) { zero_dir = true; break; }
+      inv = rsqrtf(sq);
     }
 #pragma unroll
-    for (int nt = 0; nt < G::NT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int col = n0 + nt * 8 + 2 * (lane & 3) + e;
-        vl[nt * 2 + e] = (z[col] + z[D + col]) * inv;
-      }
+    for (int nt = 0; nt < G::NT; ++nt) {
+      const float2 za = *reinterpret_cast<const float2*>(z + n0 + nt * 8 + 2 * (lane & 3));
+      const float2 zb = *reinterpret_cast<const float2*>(z + D + n0 + nt * 8 + 2 * (lane & 3));
+      vl[nt * 2] = (za.x + zb.x) * inv;
+      vl[nt * 2 + 1] = (za.y + zb.y) * inv;
+    }
   }
   if (wm == 0 && lane < 4) {
 #pragma unroll
     for (int nt = 0; nt < G::NT; ++nt)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) vs[n0 + nt * 8 + 2 * lane + e] = zero_dir ? 0.0 : vl[nt * 2 + e];
+      for (int e = 0; e < 2; ++e) vs[n0 + nt * 8 + 2 * lane + e] = zero_dir ? 0.0 : (double)vl[nt * 2 + e];
   }
   __syncthreads();
   // projections p_t = v . (u_t - mu), float64; best |p| (lowest index on ties)

@@ -1,8 +1,12 @@
 // Steps a5-a7 on the sm_100a tensor cores: exact branch, compressed branch,
 // merge and un-permute in one kernel (tcgen05.mma + TMEM + TMA).
 //
-// Work unit: a pair of adjacent query blocks (2p, 2p+1) of one head = 128
-// query rows, the M of one tcgen05 MMA. The exact branch ("Spark-H3" news
+// Work unit: a pair of query blocks of one head = 128 query rows, the M of
+// one tcgen05 MMA. The pairs come from pair_kernel: inside windows of 64
+// consecutive (permuted) query blocks, blocks are matched greedily by the
+// number of selected key blocks they share, so that the union each unit
+// walks is small (each row's result does not depend on its partner: the
+// partner's blocks carry zero weight for it). The exact branch ("Spark-H3" news
 // post, "What Spark-Attn changed": the exact branch fully computes the
 // top-ranked key/value blocks) runs over the UNION of the two blocks'
 // selected key blocks in ascending order, one 64-key block per tile; the
@@ -44,6 +48,75 @@
 #include "tc_ptx.cuh"
 
 namespace spark {
+
+// ------------------------------------------------------------------ query-block pairs
+// grid (windows of PAIR_WIN query blocks, B*H), 256 threads. The window's
+// selection bitmasks in shared memory, the shared-block count of every pair
+// of its blocks, then PAIR_WIN / 2 rounds of: take the free pair with the
+// largest count (ties to the lower pair index). Unit w * PAIR_WIN / 2 + k of
+// the head is the k-th pair taken; an odd window ends with its last free
+// block alone (partner -1). Out-of-range selection entries are skipped (the
+// attention kernel reports them).
+constexpr int PAIR_WIN = 64;
+
+__global__ void __launch_bounds__(256) pair_kernel(const int32_t* __restrict__ sel, int nb, int ksel,
+                                                   int2* __restrict__ pairs) {
+  extern __shared__ uint32_t pm[];                     // [PAIR_WIN][nwords] selection masks
+  __shared__ int ov[PAIR_WIN * PAIR_WIN];              // shared-block counts, i < j
+  __shared__ int used[PAIR_WIN];
+  __shared__ unsigned best_w[8];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int w = blockIdx.x, bh = blockIdx.y;
+  const int b0 = w * PAIR_WIN, m = min(PAIR_WIN, nb - b0);
+  const int nwords = (nb + 31) >> 5;
+  const int npairs = (nb + 1) >> 1;
+  for (int i = tid; i < m * nwords; i += 256) pm[i] = 0u;
+  for (int i = tid; i < PAIR_WIN; i += 256) used[i] = 0;
+  __syncthreads();
+  for (int i = tid; i < m * ksel; i += 256) {
+    const int r = i / ksel;
+    const int b = sel[((size_t)bh * nb + b0 + r) * ksel + (i - r * ksel)];
+    if ((unsigned)b < (unsigned)nb) atomicOr(&pm[r * nwords + (b >> 5)], 1u << (b & 31));
+  }
+  __syncthreads();
+  for (int q = tid; q < m * m; q += 256) {
+    const int i = q / m, j = q - (q / m) * m;
+    if (i >= j) continue;
+    int c = 0;
+    for (int x = 0; x < nwords; ++x) c += __popc(pm[i * nwords + x] & pm[j * nwords + x]);
+    ov[i * PAIR_WIN + j] = c;
+  }
+  __syncthreads();
+  int2* out = pairs + (size_t)bh * npairs + (size_t)w * (PAIR_WIN / 2);
+  for (int k = 0; k < m / 2; ++k) {
+    // key: count, then the lower pair index (i * PAIR_WIN + j) wins
+    unsigned best = 0u;
+    for (int q = tid; q < m * m; q += 256) {
+      const int i = q / m, j = q - (q / m) * m;
+      if (i >= j || used[i] || used[j]) continue;
+      const unsigned key = ((unsigned)ov[i * PAIR_WIN + j] << 13) | (unsigned)(8191 - (i * PAIR_WIN + j)) | (1u << 31);
+      best = max(best, key);
+    }
+    for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+    if (lane == 0) best_w[warp] = best;
+    __syncthreads();
+    if (tid == 0) {
+      unsigned b = 0u;
+      for (int x = 0; x < 8; ++x) b = max(b, best_w[x]);
+      const int pq = 8191 - (int)(b & 8191u);
+      const int i = pq / PAIR_WIN, j = pq % PAIR_WIN;
+      used[i] = 1;
+      used[j] = 1;
+      out[k] = make_int2(b0 + i, b0 + j);
+    }
+    __syncthreads();
+  }
+  if ((m & 1) && tid == 0) {
+    for (int i = 0; i < m; ++i)
+      if (!used[i]) out[m / 2] = make_int2(b0 + i, -1);
+  }
+}
+
 namespace tc {
 
 constexpr int ROWS = 128;
@@ -127,7 +200,7 @@ __device__ __forceinline__ int next_block(const uint32_t* um, int from, int nwor
 }
 
 struct Maps {
-  CUtensorMap q, k, v, kt, vt;
+  CUtensorMap q, k, v, kt, vt;  // q: 64-row boxes (the two query blocks of a unit load separately)
   CUtensorMap qc, kc, vc;      // context segment (joint attention); copies of q, k, v when absent
 };
 
@@ -136,9 +209,9 @@ struct Maps {
 template <int D, bool EXT>
 __global__ void __launch_bounds__(THREADS, 1)
 attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta, const float* __restrict__ ttab,
-               const int32_t* __restrict__ perm, const int32_t* __restrict__ sel, int N, int nb,
-               int nb_pad, int ksel, uint16_t* __restrict__ out, float* __restrict__ lse, int C, int nvid,
-               uint16_t* __restrict__ outc, float* __restrict__ lsec, int* status) {
+               const int32_t* __restrict__ perm, const int32_t* __restrict__ sel, const int2* __restrict__ pairs,
+               int N, int nb, int nb_pad, int ksel, uint16_t* __restrict__ out, float* __restrict__ lse, int C,
+               int nvid, uint16_t* __restrict__ outc, float* __restrict__ lsec, int* status) {
   using L = Layout<D>;
   constexpr int NBAR = 16;                             // barriers per slot
   extern __shared__ unsigned char smem_raw[];
@@ -193,9 +266,18 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   __syncthreads();
+  // the unit's two query blocks (video CTAs; context CTAs have no pairs)
+  static_assert(SLOTS == 2, "two units per CTA");
+  auto load_unit = [&](int s) -> int2 {
+    const int u = SLOTS * blockIdx.x + s;
+    return ((int)blockIdx.x < nvid && u < npairs) ? pairs[(size_t)bh * npairs + u] : make_int2(-1, -1);
+  };
+  const int2 unit0 = load_unit(0), unit1 = load_unit(1);
+  auto unit_of = [&](int s) -> int2 { return s == 0 ? unit0 : unit1; };
   for (int qb = 0; qb < 2 * SLOTS; ++qb) {
-    const int blk = 2 * SLOTS * blockIdx.x + qb;
-    if (blk >= nb) break;
+    const int2 un = unit_of(qb >> 1);
+    const int blk = (qb & 1) ? un.y : un.x;
+    if ((unsigned)blk >= (unsigned)nb) continue;
     const int32_t* sp = sel + ((size_t)bh * nb + blk) * ksel;
     uint32_t* m = selm[qb >> 1][qb & 1];
     for (int i = tid; i < ksel; i += THREADS) {
@@ -256,13 +338,13 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
     const int s = warp >> 2;
     const int Ts = T[s], TEs = TE[s], TXs = TX[s];
     if (Ts > 0) {
-      const int a0 = 2 * (SLOTS * blockIdx.x + s);
       const int crow0 = (SLOTS * ((int)blockIdx.x - nvid) + s) * ROWS;   // context CTAs
       const int r = (warp & 3) * 32 + lane;              // query row 0..127 of the pair
       const int qh = r >> 6;                             // which of the two query blocks
+      const int qa = qh ? unit_of(s).y : unit_of(s).x;   // that query block (-1: none)
       // uniform per warp (C - crow0 is a multiple of 32 only at whole warps; rows
       // of a partial warp past C still take part, their results are not written)
-      const bool row_valid = ctx_cta ? (crow0 + (warp & 3) * 32 < C) : (qh == 0 || a0 + 1 < nb);
+      const bool row_valid = ctx_cta ? (crow0 + (warp & 3) * 32 < C) : ((unsigned)qa < (unsigned)nb);
       const uint32_t* mymask = selm[s][qh];
       const uint32_t* um = unionm[s];
       const uint32_t tbase = tmem + ((uint32_t)((warp & 3) * 32) << 16) + SLOT_COLS * (uint32_t)s;
@@ -329,7 +411,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
             // context keys: s / sqrt(d), -inf past the end of the segment
             const bool tab = EXT && kind == 1 && ttab != nullptr;
             const float* brow = (EXT && kind == 2) ? nullptr
-                                : tab    ? ttab + ((size_t)bh * nb + a0 + qh) * nb_pad + c0
+                                : tab    ? ttab + ((size_t)bh * nb + qa) * nb_pad + c0
                                          : beta + (size_t)bh * nb_pad + c0;
 #pragma unroll
             for (int c4 = 0; c4 < 16; ++c4) {
@@ -416,7 +498,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
         size_t orow;
         bool dst_ok;
         if (!ctx_cta) {
-          const int orig = perm[(size_t)bh * N + a0 * BLK + r];
+          const int orig = perm[(size_t)bh * N + qa * BLK + (r & (BLK - 1))];
           dst_ok = (unsigned)orig < (unsigned)N;
           if (!dst_ok) set_status(status, STATUS_BAD_INPUT);
           orow = (size_t)bh * N + (dst_ok ? orig : 0);
@@ -452,13 +534,19 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
     // ------------------------------------------------ TMA producer of slot warp - 8
     const int s = warp - 8;
     if (lane == 0 && T[s] > 0) {
-      const int a0 = 2 * (SLOTS * blockIdx.x + s);
       const int crow0 = (SLOTS * ((int)blockIdx.x - nvid) + s) * ROWS;   // context CTAs
       mbar_arrive_tx(q_full(s), L::Q_BYTES);
+      // video unit: the two query blocks' 64 rows each (a lone block fills both halves)
+      const int2 un = unit_of(s);
+      const int qa0 = un.x, qa1 = un.y >= 0 ? un.y : un.x;
 #pragma unroll
       for (int a = 0; a < L::KATOMS; ++a) {
-        if (!ctx_cta) tma_load_2d(sQ(s) + a * L::Q_ATOM, &maps.q, 64 * a, bh * N + a0 * BLK, q_full(s));
-        else tma_load_2d(sQ(s) + a * L::Q_ATOM, &maps.qc, 64 * a, bh * C + crow0, q_full(s));
+        if (!ctx_cta) {
+          tma_load_2d(sQ(s) + a * L::Q_ATOM, &maps.q, 64 * a, bh * N + qa0 * BLK, q_full(s));
+          tma_load_2d(sQ(s) + a * L::Q_ATOM + BLK * 128, &maps.q, 64 * a, bh * N + qa1 * BLK, q_full(s));
+        } else {
+          tma_load_2d(sQ(s) + a * L::Q_ATOM, &maps.qc, 64 * a, bh * C + crow0, q_full(s));
+        }
       }
       const uint32_t* um = unionm[s];
       int cur = ctx_cta ? 0 : next_block(um, 0, nwords);
@@ -637,7 +725,7 @@ static cudaError_t run(const Plan& pl, const int32_t* perm, const int32_t* sel, 
   Maps maps;
   const uint64_t rows = (uint64_t)pl.BH * pl.N, srows = (uint64_t)pl.BH * pl.nb_pad;
   if (pl.nb_pad % KEYS != 0) return cudaErrorInvalidValue;
-  if (!make_map(&maps.q, ws_at<void>(ws, pl.off_Qp), rows, D, ROWS) ||
+  if (!make_map(&maps.q, ws_at<void>(ws, pl.off_Qp), rows, D, 64) ||
       !make_map(&maps.k, ws_at<void>(ws, pl.off_Kp), rows, D, 64) ||
       !make_map(&maps.v, ws_at<void>(ws, pl.off_Vp), rows, D, 64) ||
       !make_map(&maps.kt, ws_at<void>(ws, pl.off_kt), srows, D, 64) ||
@@ -662,9 +750,15 @@ static cudaError_t run(const Plan& pl, const int32_t* perm, const int32_t* sel, 
   const int nvid = (npairs + SLOTS - 1) / SLOTS;
   const int nctx = C > 0 ? ((C + ROWS - 1) / ROWS + SLOTS - 1) / SLOTS : 0;   // context query chunks, two per CTA
   const float* ttab = pl.tail == SPARK_TAIL_BLOCK ? ws_at<float>(ws, pl.off_tail) : nullptr;
+  int2* pairs = ws_at<int2>(ws, pl.off_pairs);
+  const int nwin = (pl.nb + PAIR_WIN - 1) / PAIR_WIN;
+  const size_t pair_smem = sizeof(uint32_t) * PAIR_WIN * (size_t)((pl.nb + 31) / 32);
+  e = cudaFuncSetAttribute(pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pair_smem);
+  if (e != cudaSuccess) return e;
+  pair_kernel<<<dim3(nwin, pl.BH), 256, pair_smem, s>>>(sel, pl.nb, pl.ksel, pairs);
   kern<<<dim3(nvid + nctx, pl.BH), THREADS, Lay::SMEM, s>>>(
-      maps, ws_at<float>(ws, pl.off_beta), ttab, perm, sel, pl.N, pl.nb, pl.nb_pad, pl.ksel, out, lse, C, nvid,
-      ctx ? ctx->outc : nullptr, ctx ? ctx->lsec : nullptr, status);
+      maps, ws_at<float>(ws, pl.off_beta), ttab, perm, sel, pairs, pl.N, pl.nb, pl.nb_pad, pl.ksel, out, lse, C,
+      nvid, ctx ? ctx->outc : nullptr, ctx ? ctx->lsec : nullptr, status);
   return cudaGetLastError();
 }
 

@@ -43,6 +43,7 @@ struct Plan {
   size_t off_Qp = 0, off_Kp = 0, off_Vp = 0;
   size_t off_qm = 0, off_km = 0;
   size_t off_kt = 0, off_vt = 0, off_beta = 0;
+  size_t off_pairs = 0;            // query-block pairs of the attention units (int2 [BH][ceil(nb/2)])
   size_t off_scores = 0;           // block-score matrices of score_heads heads (float64 [nb][nb] each)
   size_t off_tail = 0;             // block-tail compressed logits (float32 [BH][nb][nb_pad], log2 units)
   int score_heads = 1;

@@ -142,6 +142,7 @@ bool make_plan(const spark_params* p, Plan* pl) {
   P.off_vt = take(BH * nbp * d * 2);
   P.off_beta = take(BH * nbp * 4);
   P.off_tail = P.tail == SPARK_TAIL_BLOCK ? take(BH * nb * nbp * 4) : 0;
+  P.off_pairs = take(BH * ((nb + 1) / 2) * 8);
   {
     // float64 block-score matrices, a chunk of heads at a time (at most
     // 1 GiB, at least one head)
@@ -199,13 +200,13 @@ int32_t spark_forward_launches(const spark_params* p) {
   // when the query moment is not formed, the reduce; reblock: whiten,
   // normalise, tree, init, per split level Gram (+ reduce of chunk partials),
   // solve, project, select, then subtree and leaves; select: block
-  // statistics, then scores + top-K per chunk of heads; attention 1
+  // statistics, then scores + top-K per chunk of heads; attention 2 (pairs, kernel)
   const int moments = (pl.layout == SPARK_LAYOUT_K_REUSE_Q) ? 2 : 3;
   int split_launches = 0;
   for (int lv = 0; lv < pl.sub_level; ++lv) split_launches += 4 + (pl.level_chunks[lv] > 1 ? 1 : 0);
   const int reblock = pl.nperm * (4 + split_launches + (pl.sub_level < pl.nlevels ? 1 : 0) + 1);
   const int select = 1 + 2 * ((pl.BH + pl.score_heads - 1) / pl.score_heads) + (pl.tail == SPARK_TAIL_BLOCK ? 1 : 0);
-  return moments + reblock + select + 1;
+  return moments + reblock + select + 2;
 }
 
 size_t spark_host_workspace_size(const spark_params* p) {

@@ -257,7 +257,8 @@ spark_status spark_forward(const spark_params* p, const void* q, const void* k, 
  * normalise, tree, init, subtree, leaves - plus 4 per tree level above the
  * first level whose groups all have at most 9 blocks, 5 when that level's
  * groups span several chunk CTAs; select 1 + 2 per chunk of heads (+1 for
- * the block tail); attention 1); -1 if invalid. */
+ * the block tail); attention 2: query-block pairing, then the kernel); -1 if
+ * invalid. */
 int32_t spark_forward_launches(const spark_params* p);
 
 /* Device bytes spark_forward_host needs: spark_workspace_size() plus room

@@ -52,26 +52,26 @@ namespace spark {
 // ------------------------------------------------------------------ query-block pairs
 // grid (windows of PAIR_WIN query blocks, B*H), 256 threads. The window's
 // selection bitmasks in shared memory, the shared-block count of every pair
-// of its blocks, then PAIR_WIN / 2 rounds of: take the free pair with the
-// largest count (ties to the lower pair index). Unit w * PAIR_WIN / 2 + k of
+// of its blocks (each thread keeps its 16 candidates in registers), then
+// PAIR_WIN / 2 rounds of: take the free pair with the largest count (ties to
+// the lower pair index), the used blocks one 64-bit mask. Unit w * PAIR_WIN / 2 + k of
 // the head is the k-th pair taken; an odd window ends with its last free
 // block alone (partner -1). Out-of-range selection entries are skipped (the
 // attention kernel reports them).
 constexpr int PAIR_WIN = 64;
 
-__global__ void __launch_bounds__(256) pair_kernel(const int32_t* __restrict__ sel, int nb, int ksel,
+__global__ void __launch_bounds__(256, 1) pair_kernel(const int32_t* __restrict__ sel, int nb, int ksel,
                                                    int2* __restrict__ pairs) {
+  static_assert(PAIR_WIN == 64, "pair (i, j) is coded as i * 64 + j; the used set is one 64-bit mask");
+  constexpr int KPT = PAIR_WIN * PAIR_WIN / 256;       // candidate pairs per thread
   extern __shared__ uint32_t pm[];                     // [PAIR_WIN][nwords] selection masks
-  __shared__ int ov[PAIR_WIN * PAIR_WIN];              // shared-block counts, i < j
-  __shared__ int used[PAIR_WIN];
-  __shared__ unsigned best_w[8];
+  __shared__ unsigned best_w[2][8];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int w = blockIdx.x, bh = blockIdx.y;
   const int b0 = w * PAIR_WIN, m = min(PAIR_WIN, nb - b0);
   const int nwords = (nb + 31) >> 5;
   const int npairs = (nb + 1) >> 1;
   for (int i = tid; i < m * nwords; i += 256) pm[i] = 0u;
-  for (int i = tid; i < PAIR_WIN; i += 256) used[i] = 0;
   __syncthreads();
   for (int i = tid; i < m * ksel; i += 256) {
     const int r = i / ksel;
@@ -79,41 +79,43 @@ __global__ void __launch_bounds__(256) pair_kernel(const int32_t* __restrict__ s
     if ((unsigned)b < (unsigned)nb) atomicOr(&pm[r * nwords + (b >> 5)], 1u << (b & 31));
   }
   __syncthreads();
-  for (int q = tid; q < m * m; q += 256) {
-    const int i = q / m, j = q - (q / m) * m;
-    if (i >= j) continue;
-    int c = 0;
-    for (int x = 0; x < nwords; ++x) c += __popc(pm[i * nwords + x] & pm[j * nwords + x]);
-    ov[i * PAIR_WIN + j] = c;
+  // this thread's candidates q = tid + 256 s, q = i * 64 + j: key = shared
+  // count, then the lower q; 0 = not a pair of the window
+  unsigned key[KPT];
+#pragma unroll
+  for (int s = 0; s < KPT; ++s) {
+    const int q = tid + 256 * s, i = q >> 6, j = q & 63;
+    key[s] = 0u;
+    if (i < j && j < m) {
+      int c = 0;
+      for (int x = 0; x < nwords; ++x) c += __popc(pm[i * nwords + x] & pm[j * nwords + x]);
+      key[s] = (1u << 31) | ((unsigned)c << 12) | (unsigned)(4095 - q);
+    }
   }
-  __syncthreads();
   int2* out = pairs + (size_t)bh * npairs + (size_t)w * (PAIR_WIN / 2);
+  unsigned long long usedm = 0ull;
   for (int k = 0; k < m / 2; ++k) {
-    // key: count, then the lower pair index (i * PAIR_WIN + j) wins
     unsigned best = 0u;
-    for (int q = tid; q < m * m; q += 256) {
-      const int i = q / m, j = q - (q / m) * m;
-      if (i >= j || used[i] || used[j]) continue;
-      const unsigned key = ((unsigned)ov[i * PAIR_WIN + j] << 13) | (unsigned)(8191 - (i * PAIR_WIN + j)) | (1u << 31);
-      best = max(best, key);
+#pragma unroll
+    for (int s = 0; s < KPT; ++s) {
+      const int q = tid + 256 * s;
+      const bool free = !((usedm >> (q >> 6)) & 1ull) && !((usedm >> (q & 63)) & 1ull);
+      if (free) best = max(best, key[s]);
     }
     for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
-    if (lane == 0) best_w[warp] = best;
-    __syncthreads();
-    if (tid == 0) {
-      unsigned b = 0u;
-      for (int x = 0; x < 8; ++x) b = max(b, best_w[x]);
-      const int pq = 8191 - (int)(b & 8191u);
-      const int i = pq / PAIR_WIN, j = pq % PAIR_WIN;
-      used[i] = 1;
-      used[j] = 1;
-      out[k] = make_int2(b0 + i, b0 + j);
-    }
-    __syncthreads();
+    if (lane == 0) best_w[k & 1][warp] = best;
+    __syncthreads();                                   // best_w[k & 1] is rewritten two rounds on
+    unsigned b = 0u;
+#pragma unroll
+    for (int x = 0; x < 8; ++x) b = max(b, best_w[k & 1][x]);
+    const int pq = 4095 - (int)(b & 4095u);
+    const int i = pq >> 6, j = pq & 63;
+    usedm |= (1ull << i) | (1ull << j);
+    if (tid == 0) out[k] = make_int2(b0 + i, b0 + j);
   }
   if ((m & 1) && tid == 0) {
     for (int i = 0; i < m; ++i)
-      if (!used[i]) out[m / 2] = make_int2(b0 + i, -1);
+      if (!((usedm >> i) & 1ull)) out[m / 2] = make_int2(b0 + i, -1);
   }
 }
 

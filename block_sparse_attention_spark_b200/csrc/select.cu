@@ -16,6 +16,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "dmma.cuh"
 #include "plan.h"
 
 namespace spark {
@@ -140,76 +141,85 @@ blockstats_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k
 
 // ------------------------------------------------------------------ selection
 // score_kernel: the block-score matrix of one chunk of heads,
-//   sc[h][a][b] = (Qbar_a . Kbar_b) / sqrt(d) in float64, as a register-tiled
-//   GEMM: a CTA computes a 128 x 128 tile, each thread an 8 x 8 sub-tile
-//   (rows and columns in pairs 32 apart),
-//   with the d dimension staged through shared memory 8 at a time.
-constexpr int SC_TILE = 128, SC_KSTEP = 8;
+//   sc[h][a][b] = (Qbar_a . Kbar_b) / sqrt(d) in float64, on the float64
+//   tensor cores (mma.sync m16n8k16, dmma.cuh): a CTA computes a 128 x 128
+//   tile; warp w owns rows 32 (w % 4).. and columns 64 (w / 4)..: two 16-row
+//   by eight 8-column MMA tiles. The d dimension is staged 16 at a time
+//   through a cp.async double buffer of float64 rows (stride 20 doubles: the
+//   fragments' half-warps hit distinct bank pairs); rows past nb are zero.
+constexpr int SC_TILE = 128, SC_KSTEP = 16, SC_LD = SC_KSTEP + 4;
+constexpr int SC_SMEM = (int)sizeof(double) * 4 * SC_TILE * SC_LD;   // two buffers of each operand
 
 template <int D>
 __global__ void __launch_bounds__(256)
 score_kernel(const double* __restrict__ qm, const double* __restrict__ km, int nb, int h0,
              double* __restrict__ sc) {
-  __shared__ __align__(16) double qs[2][SC_KSTEP][SC_TILE];   // [k][a]
-  __shared__ __align__(16) double ks[2][SC_KSTEP][SC_TILE];   // [k][b]
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  extern __shared__ __align__(16) double scs[];       // qs [2][a][k], then ks [2][b][k]
+  auto qs = [&](int buf) { return scs + buf * (SC_TILE * SC_LD); };
+  auto ks = [&](int buf) { return scs + (2 + buf) * (SC_TILE * SC_LD); };
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
   const int b0 = blockIdx.x * SC_TILE, a0 = blockIdx.y * SC_TILE, h = blockIdx.z;
   const size_t bh = (size_t)(h0 + h);
   const double* Q = qm + bh * nb * D;
   const double* K = km + bh * nb * D;
-  // loader: thread -> (row r = tid / 2, 4 consecutive k of the 8) for Q and K
-  const int lr = tid >> 1, lk = (tid & 1) * 4;
+  const int wr = (warp & 3) * 32, wc = (warp >> 2) * 64;
+  // loader: 128 rows x 16 doubles = 1024 16-byte chunks per operand, 4 per thread
   auto load = [&](int buf, int kc) {
-    const int ra = a0 + lr, rb = b0 + lr;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      qs[buf][lk + e][lr] = ra < nb ? Q[(size_t)ra * D + kc + lk + e] : 0.0;
-      ks[buf][lk + e][lr] = rb < nb ? K[(size_t)rb * D + kc + lk + e] : 0.0;
+    for (int i = 0; i < 4; ++i) {
+      const int c = tid + 256 * i, r = c >> 3, ch = c & 7;
+      double* dq = qs(buf) + r * SC_LD + 2 * ch;
+      double* dk = ks(buf) + r * SC_LD + 2 * ch;
+      if (a0 + r < nb) cp_async16(dq, Q + (size_t)(a0 + r) * D + kc + 2 * ch);
+      else *reinterpret_cast<double2*>(dq) = make_double2(0.0, 0.0);
+      if (b0 + r < nb) cp_async16(dk, K + (size_t)(b0 + r) * D + kc + 2 * ch);
+      else *reinterpret_cast<double2*>(dk) = make_double2(0.0, 0.0);
     }
   };
-  double acc[8][8];
+  double acc[2][8][4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int m = 0; m < 2; ++m)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[m][j][e] = 0.0;
   load(0, 0);
-  __syncthreads();
+  cp_async_commit();
   for (int kc = 0; kc < D; kc += SC_KSTEP) {
     const int buf = (kc / SC_KSTEP) & 1;
     if (kc + SC_KSTEP < D) load(buf ^ 1, kc + SC_KSTEP);
-#pragma unroll
-    for (int kk = 0; kk < SC_KSTEP; ++kk) {
-      // rows ty*2 + 32*ii + {0,1}, columns tx*2 + 32*jj + {0,1}: for each ii / jj
-      // the 16 lanes of a half-warp read consecutive double2 (no bank conflicts)
-      double qa[8], kb[8];
-#pragma unroll
-      for (int ii = 0; ii < 4; ++ii) {
-        const double2 t = *reinterpret_cast<const double2*>(&qs[buf][kk][ty * 2 + 32 * ii]);
-        qa[2 * ii] = t.x;
-        qa[2 * ii + 1] = t.y;
-        const double2 u = *reinterpret_cast<const double2*>(&ks[buf][kk][tx * 2 + 32 * ii]);
-        kb[2 * ii] = u.x;
-        kb[2 * ii + 1] = u.y;
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fma(qa[i], kb[j], acc[i][j]);
-    }
+    cp_async_commit();
+    cp_async_wait<1>();
     __syncthreads();
-  }
-  const double scale = 1.0 / sqrt((double)D);
-  double* out = sc + (size_t)h * nb * nb;
+    const double* qb = qs(buf);
+    const double* kb = ks(buf);
+    double a[2][8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int a = a0 + ty * 2 + 32 * (i >> 1) + (i & 1);
-    if (a >= nb) continue;
+    for (int m = 0; m < 2; ++m)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a[m][i] = qb[(wr + 16 * m + g + 8 * (i % 2)) * SC_LD + t4 + 4 * (i / 2)];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const int b = b0 + tx * 2 + 32 * (j >> 1) + (j & 1);
-      if (b < nb) out[(size_t)a * nb + b] = acc[i][j] * scale;
+      double bf[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) bf[i] = kb[(wc + 8 * j + g) * SC_LD + t4 + 4 * i];
+#pragma unroll
+      for (int m = 0; m < 2; ++m) dmma16816(acc[m][j], a[m], bf);
     }
+    __syncthreads();                                   // the buffer is refilled next step
   }
+  cp_async_wait<0>();
+  const double sd = sqrt((double)D);
+  double* out = sc + (size_t)h * nb * nb;
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int a = a0 + wr + 16 * m + g + 8 * (e >> 1), b = b0 + wc + 8 * j + 2 * t4 + (e & 1);
+        if (a < nb && b < nb) out[(size_t)a * nb + b] = acc[m][j][e] / sd;
+      }
 }
 
 // topk_kernel: one warp per query block a of the chunk: the ksel largest
@@ -369,9 +379,11 @@ static cudaError_t run_select(const Plan& pl, const uint16_t* q, const uint16_t*
         qm, kt, beta, pl.nb, pl.nb_pad, ws_at<float>(ws, pl.off_tail));
   double* sc = ws_at<double>(ws, pl.off_scores);
   const int tiles = (pl.nb + SC_TILE - 1) / SC_TILE;
+  cudaError_t e = cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, SC_SMEM);
+  if (e != cudaSuccess) return e;
   for (int h0 = 0; h0 < pl.BH; h0 += pl.score_heads) {
     const int heads = std::min(pl.score_heads, pl.BH - h0);
-    score_kernel<D><<<dim3(tiles, tiles, heads), 256, 0, s>>>(qm, km, pl.nb, h0, sc);
+    score_kernel<D><<<dim3(tiles, tiles, heads), 256, SC_SMEM, s>>>(qm, km, pl.nb, h0, sc);
     const long rows = (long)heads * pl.nb;
     topk_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(sc, pl.nb, pl.ksel, h0, heads, sel);
   }

@@ -103,14 +103,13 @@ whiten_prep_kernel(const double* __restrict__ M, double* __restrict__ Lout, int*
 // within a float64 rounding of a bf16 midpoint.
 //
 // The quotient: q = u_j * (1 / |u|) is within 3 float64 ulps of the IEEE
-// quotient u_j / |u|, so both round to the same bf16 unless q's 45 bits
-// below the bf16 precision lie within 8 units of the halfway pattern; only
-// then (practically never) is the division carried out. Away from a
-// midpoint, rounding q to nearest keeps its top 19 bits (sign, 11-bit
-// exponent, 7 mantissa bits) plus one when the dropped bits exceed half, the
-// carry running into the exponent; the exponent is then rebased from
-// float64 to bf16. Zero, and magnitudes outside the bf16 normal range, take
-// the library conversion instead.
+// quotient u_j / |u|. q is rounded to nearest float32, f, and f to nearest
+// bf16. Rounding twice differs from rounding q once only when f lands
+// exactly on a bf16 halfway point (low 16 bits 0x8000), and f lands there
+// whenever q (or the IEEE quotient) is within half a float32 ulp of a
+// halfway point, far more than 3 float64 ulps; so when f's low half is not
+// 0x8000, bf16(f) is the bf16 of the IEEE quotient, and otherwise
+// (practically never) the division is carried out and rounded once.
 //
 // Persistent CTAs, one per SM, each take a balanced contiguous range of the
 // layer's (head, 16-token tile) items, in segments of one head: per segment
@@ -133,18 +132,16 @@ struct NormSmem {
   static constexpr int CH = TOK * (D / 8) / 32;       // 16-byte chunks per lane and tile
 };
 
-__device__ __forceinline__ uint32_t bf16_of_quotient(double u, double r, double rinv) {
-  const double qv = u * rinv;
-  const unsigned long long bits = (unsigned long long)__double_as_longlong(qv);
-  const long long low = (long long)(bits & ((1ull << 45) - 1));
-  const long long dist = low - (1ll << 44);
-  const unsigned long long top = (bits >> 45) + (dist > 0 ? 1ull : 0ull);   // sign | exp11 | mant7
-  const int e = (int)((top >> 7) & 0x7ff) - 896;                            // bf16 biased exponent
-  if (dist > 8 || dist < -8) {
-    if (e >= 1 && e <= 254) return (uint32_t)(((top >> 18) << 15) | ((unsigned)e << 7) | (top & 0x7f));
-    return (uint32_t)__bfloat16_as_ushort(__double2bfloat16(qv));
+// bf16 bits of u / r for a pair (u0, u1), low half u0; rinv = 1 / r.
+__device__ __forceinline__ uint32_t bf16x2_of_quotients(double u0, double u1, double r, double rinv) {
+  const float f0 = __double2float_rn(u0 * rinv), f1 = __double2float_rn(u1 * rinv);
+  if (((__float_as_uint(f0) & 0xffffu) == 0x8000u) | ((__float_as_uint(f1) & 0xffffu) == 0x8000u)) {
+    return (uint32_t)__bfloat16_as_ushort(__double2bfloat16(u0 / r)) |
+           ((uint32_t)__bfloat16_as_ushort(__double2bfloat16(u1 / r)) << 16);
   }
-  return (uint32_t)__bfloat16_as_ushort(__double2bfloat16(u / r));
+  uint32_t w;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(f1), "f"(f0));
+  return w;
 }
 
 template <int D>
@@ -232,8 +229,8 @@ normalize64_kernel(const uint16_t* __restrict__ X, const double* __restrict__ La
 #pragma unroll
       for (int c = 0; c < CT; ++c) {
         const int col = 8 * c + 2 * t4;
-        const uint32_t w0 = r0 > 0.0 ? bf16_of_quotient(acc[c][0], r0, i0) | (bf16_of_quotient(acc[c][1], r0, i0) << 16) : 0u;
-        const uint32_t w1 = r1 > 0.0 ? bf16_of_quotient(acc[c][2], r1, i1) | (bf16_of_quotient(acc[c][3], r1, i1) << 16) : 0u;
+        const uint32_t w0 = r0 > 0.0 ? bf16x2_of_quotients(acc[c][0], acc[c][1], r0, i0) : 0u;
+        const uint32_t w1 = r1 > 0.0 ? bf16x2_of_quotients(acc[c][2], acc[c][3], r1, i1) : 0u;
         *reinterpret_cast<uint32_t*>(os + g * RS + col) = w0;
         *reinterpret_cast<uint32_t*>(os + (g + 8) * RS + col) = w1;
       }
@@ -1139,9 +1136,36 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
   // slice, the rest the right child's (order inside a child is irrelevant:
   // it is cut again, and leaves are sorted by index at the end)
   const int nL = BLK * ((nn / BLK) / 2);
-  cut_partition<1>(
-      nn, nL, [&](int t) -> uint64_t { return ordered_key(sgn * pv[t]); }, [&](int t) { return ids[lo[t]]; },
-      [&](int dst, int t) { stok[dst] = lo[t]; }, hist, sh_sel, sh_key, warp_tot, red_i, status);
+  if (nn <= 256) {
+    // at most one member per thread: its rank among the unique (key, index)
+    // pairs is its position, so the nL smallest come first (no select passes)
+    uint64_t* kv = reinterpret_cast<uint64_t*>(pv);
+    int* kid = reinterpret_cast<int*>(zp);
+    uint64_t mykey = 0;
+    int myid = 0;
+    if (tid < nn) {
+      mykey = ordered_key(sgn * pv[tid]);
+      myid = ids[lo[tid]];
+    }
+    __syncthreads();                                   // pv is read as doubles above
+    if (tid < nn) {
+      kv[tid] = mykey;
+      kid[tid] = myid;
+    }
+    __syncthreads();
+    if (tid < nn) {
+      int rank = 0;
+      for (int u = 0; u < nn; ++u) {
+        const uint64_t k = kv[u];
+        rank += (k < mykey) | ((k == mykey) & (kid[u] < myid));
+      }
+      stok[rank] = lo[tid];
+    }
+  } else {
+    cut_partition<1>(
+        nn, nL, [&](int t) -> uint64_t { return ordered_key(sgn * pv[t]); }, [&](int t) { return ids[lo[t]]; },
+        [&](int dst, int t) { stok[dst] = lo[t]; }, hist, sh_sel, sh_key, warp_tot, red_i, status);
+  }
   __syncthreads();
   for (int t = tid; t < nn; t += blockDim.x) loc[s0 + t] = stok[t];
   __syncthreads();

@@ -893,6 +893,7 @@ big_select_kernel(int N, const int2* __restrict__ nodes, int nnodes, int chunks,
 // exact ranks of (projection, index) - the node's slice of the local order
 // is rewritten in ascending rank, so children are contiguous slices.
 constexpr int SUB_BLOCKS = 9;
+constexpr bool SUB_PAIR = true;   // two groups of a level share one power iteration
 
 template <int D>
 struct SubSmem {
@@ -908,11 +909,18 @@ struct SubSmem {
   static constexpr size_t bytes = off_zp + (zp_bytes > sizeof(double) * 256 ? zp_bytes : sizeof(double) * 256);
 };
 
+// One split of a subtree group, in three phases so that two groups of the
+// same level can share the latency-bound power iteration:
+//   sub_cov    : Gram of the group (float32 over at most SUB_BLOCKS tiles),
+//                column means (float64, into mus), covariance S in this
+//                thread's fragment entries (formed in float64, kept in float32)
+//   sub_power  : float32 power iteration of one or two groups' S, one barrier
+//                per step for both; v into vs (float64)
+//   sub_finish : float64 projections, orientation, the cut, the group's slice
+//                of the local order rewritten left child first
 template <int D>
-__device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* ids, uint16_t* loc,
-                              uint16_t* stok, double* zp, double* mus, double* vs, double* red_d, int* red_i,
-                              double* sh_sgn, int* hist, int* sh_sel, unsigned long long* sh_key,
-                              int* warp_tot, int* status, int s0, int nn, int iters) {
+__device__ void sub_cov(const uint16_t* rows, const uint16_t* loc, double* zp, double* mus, int s0, int nn,
+                        float (&S)[Gram<D>::ACC]) {
   using G = Gram<D>;
   using SM = SubSmem<D>;
   constexpr int RS = SM::RS;
@@ -984,31 +992,47 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
   // S = G / n - mu mu^T on this thread's fragment entries, formed in float64
   // and kept in float32: a subtree's groups are small and its Gram sums are
   // float32 already, and float32 steps halve the latency-bound iteration
-  // (the direction is scale-free, so rescaling v by an approximate norm every
-  // NORM_EVERY_F32 steps changes nothing; two unscaled float32 steps stay far
-  // from underflow for any nonzero covariance of distinct bf16 unit vectors).
-  constexpr int NORM_EVERY_F32 = 2;
   const double invn = 1.0 / (double)nn;
-  float S[G::ACC];
 #pragma unroll
   for (int j = 0; j < G::ACC; ++j) {
     int row, col;
     G::coord(j, warp, lane, row, col);
     S[j] = (float)((double)acc[j] * invn - mus[row] * mus[col]);
   }
-  // power iteration in the fragment layout: rows m0 + mt*16 + lane/4 + 8h,
-  // columns n0 + nt*8 + 2 (lane % 4) + e
-  float vl[G::NT * 2];
+}
+
+template <int D, bool PAIR>
+__device__ void sub_power(const float (&SA)[Gram<D>::ACC], const float (&SB)[Gram<D>::ACC], double* zp, double* vsA,
+                          double* vsB, int iters) {
+  // the direction is scale-free, so rescaling v by an approximate norm every
+  // NORM_EVERY_F32 steps changes nothing; two unscaled float32 steps stay far
+  // from underflow for any nonzero covariance of distinct bf16 unit vectors.
+  // A group whose S v vanishes keeps v = 0 (its norm step sets the scale to 0).
+  using G = Gram<D>;
+  constexpr int NORM_EVERY_F32 = 2;
+  constexpr int NG = PAIR ? 2 : 1;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wm = warp % 4, wn = warp / 4;
+  const int m0 = wm * G::WM, n0 = wn * G::WN;
+  (void)tid;
+  // rows m0 + mt*16 + lane/4 + 8h, columns n0 + nt*8 + 2 (lane % 4) + e
+  float vl[NG][G::NT * 2];
 #pragma unroll
-  for (int j = 0; j < G::NT * 2; ++j) vl[j] = 1.0f;
-  bool zero_dir = false;
+  for (int q = 0; q < NG; ++q)
+#pragma unroll
+    for (int j = 0; j < G::NT * 2; ++j) vl[q][j] = 1.0f;
+  bool zero_dir[NG];
+#pragma unroll
+  for (int q = 0; q < NG; ++q) zero_dir[q] = false;
   float* zpf = reinterpret_cast<float*>(zp);
   for (int iter = 0; iter < iters; ++iter) {
-    float* z = zpf + (iter & 1) * 2 * D;         // [wn][row]: the two column halves' partial sums
+    float* zb = zpf + (iter & 1) * 2 * NG * D;        // [group][wn][row]: the two column halves' partial sums
     const bool norm_step = (iter % NORM_EVERY_F32) == NORM_EVERY_F32 - 1 || iter == iters - 1;
-    float zr[G::MT][2];
+    float zr[NG][G::MT][2];
 #pragma unroll
-    for (int mt = 0; mt < G::MT; ++mt) { zr[mt][0] = 0.f; zr[mt][1] = 0.f; }
+    for (int q = 0; q < NG; ++q)
+#pragma unroll
+      for (int mt = 0; mt < G::MT; ++mt) { zr[q][mt][0] = 0.f; zr[q][mt][1] = 0.f; }
 #pragma unroll
     for (int nt = 0; nt < G::NT; ++nt)
 #pragma unroll
@@ -1016,49 +1040,75 @@ __device__ void subtree_split(const uint16_t* rows, double* pv, const int32_t* i
 #pragma unroll
         for (int mt = 0; mt < G::MT; ++mt)
 #pragma unroll
-          for (int h = 0; h < 2; ++h) zr[mt][h] = fmaf(S[(mt * G::NT + nt) * 4 + 2 * h + e], vl[nt * 2 + e], zr[mt][h]);
+          for (int h = 0; h < 2; ++h) {
+            zr[0][mt][h] = fmaf(SA[(mt * G::NT + nt) * 4 + 2 * h + e], vl[0][nt * 2 + e], zr[0][mt][h]);
+            if (PAIR) zr[NG - 1][mt][h] = fmaf(SB[(mt * G::NT + nt) * 4 + 2 * h + e], vl[NG - 1][nt * 2 + e], zr[NG - 1][mt][h]);
+          }
 #pragma unroll
     for (int o = 1; o <= 2; o <<= 1)
 #pragma unroll
-      for (int mt = 0; mt < G::MT; ++mt)
+      for (int q = 0; q < NG; ++q)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) zr[mt][h] += __shfl_xor_sync(0xffffffffu, zr[mt][h], o);
+        for (int mt = 0; mt < G::MT; ++mt)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) zr[q][mt][h] += __shfl_xor_sync(0xffffffffu, zr[q][mt][h], o);
     if ((lane & 3) == 0) {
 #pragma unroll
-      for (int mt = 0; mt < G::MT; ++mt)
+      for (int q = 0; q < NG; ++q)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) z[wn * D + m0 + mt * 16 + (lane >> 2) + 8 * h] = zr[mt][h];
+        for (int mt = 0; mt < G::MT; ++mt)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) zb[(q * 2 + wn) * D + m0 + mt * 16 + (lane >> 2) + 8 * h] = zr[q][mt][h];
     }
     __syncthreads();
-    float inv = 1.f;
-    if (norm_step) {
-      // every warp forms |z|^2 itself, in the same order: no second barrier
-      float sq = 0.f;
 #pragma unroll
-      for (int k = 0; k < D / 32; ++k) {
-        const float zz = z[lane + 32 * k] + z[D + lane + 32 * k];
-        sq = fmaf(zz, zz, sq);
+    for (int q = 0; q < NG; ++q) {
+      const float* z = zb + q * 2 * D;
+      float inv = 1.f;
+      if (norm_step) {
+        // every warp forms |z|^2 itself, in the same order: no second barrier
+        float sq = 0.f;
+#pragma unroll
+        for (int k = 0; k < D / 32; ++k) {
+          const float zz = z[lane + 32 * k] + z[D + lane + 32 * k];
+          sq = fmaf(zz, zz, sq);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        if (sq == 0.f) zero_dir[q] = true;
+        inv = zero_dir[q] ? 0.f : rsqrtf(sq);
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-      if (sq == 0.f) { zero_dir = true; break; }
-      inv = rsqrtf(sq);
-    }
-#pragma unroll
-    for (int nt = 0; nt < G::NT; ++nt) {
-      const float2 za = *reinterpret_cast<const float2*>(z + n0 + nt * 8 + 2 * (lane & 3));
-      const float2 zb = *reinterpret_cast<const float2*>(z + D + n0 + nt * 8 + 2 * (lane & 3));
-      vl[nt * 2] = (za.x + zb.x) * inv;
-      vl[nt * 2 + 1] = (za.y + zb.y) * inv;
+      for (int nt = 0; nt < G::NT; ++nt) {
+        const float2 za = *reinterpret_cast<const float2*>(z + n0 + nt * 8 + 2 * (lane & 3));
+        const float2 zc = *reinterpret_cast<const float2*>(z + D + n0 + nt * 8 + 2 * (lane & 3));
+        vl[q][nt * 2] = (za.x + zc.x) * inv;
+        vl[q][nt * 2 + 1] = (za.y + zc.y) * inv;
+      }
     }
   }
   if (wm == 0 && lane < 4) {
 #pragma unroll
-    for (int nt = 0; nt < G::NT; ++nt)
+    for (int q = 0; q < NG; ++q) {
+      double* vs = q == 0 ? vsA : vsB;
 #pragma unroll
-      for (int e = 0; e < 2; ++e) vs[n0 + nt * 8 + 2 * lane + e] = zero_dir ? 0.0 : (double)vl[nt * 2 + e];
+      for (int nt = 0; nt < G::NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) vs[n0 + nt * 8 + 2 * lane + e] = zero_dir[q] ? 0.0 : (double)vl[q][nt * 2 + e];
+    }
   }
   __syncthreads();
+}
+
+template <int D>
+__device__ void sub_finish(const uint16_t* rows, double* pv, const int32_t* ids, uint16_t* loc, uint16_t* stok,
+                           double* zp, const double* mus, const double* vs, double* red_d, int* red_i,
+                           double* sh_sgn, int* hist, int* sh_sel, unsigned long long* sh_key, int* warp_tot,
+                           int* status, int s0, int nn) {
+  using SM = SubSmem<D>;
+  constexpr int RS = SM::RS;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint16_t* lo = loc + s0;
   // projections p_t = v . (u_t - mu), float64; best |p| (lowest index on ties)
   double best_abs = -1.0, best_p = 0.0;
   int best_id = 0x7fffffff;
@@ -1183,7 +1233,7 @@ subtree_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restrict_
   uint16_t* loc = reinterpret_cast<uint16_t*>(smem_raw + SM::off_loc);
   uint16_t* stok = reinterpret_cast<uint16_t*>(smem_raw + SM::off_stok);
   double* zp = reinterpret_cast<double*>(smem_raw + SM::off_zp);
-  __shared__ double mus[D], vs[D], red_d[16];
+  __shared__ double mus[D], vs[D], mus2[D], vs2[D], red_d[16];
   __shared__ int red_i[8], hist[256], sh_sel[3], warp_tot[8];
   __shared__ unsigned long long sh_key;
   __shared__ double sh_sgn;
@@ -1217,11 +1267,24 @@ subtree_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restrict_
   int cur = 0;
   while (lvl_n[cur] > 0) {
     const int cnt = lvl_n[cur];
-    for (int i = 0; i < cnt; ++i) {
-      const int2 nd = lvl[cur][i];
-      if (nd.y >= 2)
-        subtree_split<D>(rows, pv, ids, loc, stok, zp, mus, vs, red_d, red_i, &sh_sgn, hist, sh_sel, &sh_key,
-                         warp_tot, status, nd.x * BLK, nd.y * BLK, iters);
+    // the level's groups two at a time (every listed group has at least 2 blocks)
+    for (int i = 0; i < cnt; i += SUB_PAIR ? 2 : 1) {
+      const int2 na = lvl[cur][i];
+      const bool two = SUB_PAIR && i + 1 < cnt;
+      const int2 nbn = two ? lvl[cur][i + 1] : na;
+      float SA[Gram<D>::ACC], SB[Gram<D>::ACC];
+      sub_cov<D>(rows, loc, zp, mus, na.x * BLK, na.y * BLK, SA);
+      if (two) {
+        sub_cov<D>(rows, loc, zp, mus2, nbn.x * BLK, nbn.y * BLK, SB);
+        sub_power<D, true>(SA, SB, zp, vs, vs2, iters);
+      } else {
+        sub_power<D, false>(SA, SA, zp, vs, vs, iters);
+      }
+      sub_finish<D>(rows, pv, ids, loc, stok, zp, mus, vs, red_d, red_i, &sh_sgn, hist, sh_sel, &sh_key, warp_tot,
+                    status, na.x * BLK, na.y * BLK);
+      if (two)
+        sub_finish<D>(rows, pv, ids, loc, stok, zp, mus2, vs2, red_d, red_i, &sh_sgn, hist, sh_sel, &sh_key,
+                      warp_tot, status, nbn.x * BLK, nbn.y * BLK);
     }
     if (tid == 0) {
       int m = 0;

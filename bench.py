@@ -200,7 +200,8 @@ def stage_rooflines(w, ksel, stage, peaks, clk):
       select    : q, k, v read once and their permuted copies written,
                   12 N d bytes, against HBM;
       attention : the main roofline entry.
-    The float64 peak is derived, not measured by the driver: 64 float64 FMA
+    traffic: the stage's DRAM bytes per layer from the committed capture (or
+    None). The float64 peak is derived, not measured by the driver: 64 float64 FMA
     per clock per SM x 148 SMs x 2 x the sampled maximum SM clock."""
     import math
     BH, N, d = w.B * w.H, w.N, w.d
@@ -223,6 +224,9 @@ def stage_rooflines(w, ksel, stage, peaks, clk):
     t = stage[2] * 1e-3
     out["select"] = {"bound": "hbm", "achieved": sbytes / t / 1e9, "peak": hbm, "unit": "GB/s",
                      "frac": sbytes / t / 1e9 / hbm, "algorithmic_bytes": sbytes}
+    traffic = stage_traffic(w)
+    for name in ("moments", "reblock", "select"):
+        out[name]["traffic"] = traffic.get(name)
     return out
 
 
@@ -245,6 +249,28 @@ def oracle_full_layers():
         _, _, dense = flops(w, so.num_selected(w.nb, w.ratio))
         out[name] = {"seconds_per_layer": round(t, 3), "eff_tflops": dense / t / 1e12,
                      "what": f"B={w.B} H={w.H} N={w.N} d={w.d} ratio={w.ratio}, every head and query block"}
+    return out
+
+
+def stage_traffic(w):
+    """DRAM bytes of each stage's kernels from the committed ncu capture
+    (profiles/stage_traffic.json: dram__bytes_read.sum + dram__bytes_write.sum
+    summed over the stage's launches on a few heads), scaled to this layer's
+    head count (every stage works head by head); a stage whose sources changed
+    since the capture gets None."""
+    import hashlib
+    out = {}
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "stage_traffic.json")))
+    except Exception:
+        return out
+    for name, st in rec.get("stages", {}).items():
+        try:
+            src = b"".join(open(os.path.join(ROOT, f), "rb").read() for f in st["sources"])
+            ok = hashlib.sha256(src).hexdigest() == st["sources_sha256"]
+            out[name] = st["dram_bytes"] / rec["heads_captured"] * w.H * w.B if ok else None
+        except Exception:
+            out[name] = None
     return out
 
 

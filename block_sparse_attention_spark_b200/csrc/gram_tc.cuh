@@ -128,14 +128,17 @@ __device__ void gram_tc_body(const uint16_t* __restrict__ X, RowF rowf, int ntil
       mma_commit(bar0 + 8u * (uint32_t)(g & 1));
     }
     if (g > 0) {
-      // the previous group's sums: wait for its MMAs, fold into float64
+      // the previous group's MMAs done: its ring half can be refilled at once,
+      // then its sums are folded into float64 while the loads are in flight
       ok = ok && __all_sync(0xffffffffu, mbar_wait(bar0 + 8u * (uint32_t)((g - 1) & 1), (uint32_t)(((g - 1) >> 1) & 1), status));
       fence_after();
-      if (ok) flush(g - 1);
-      fence_before();
     }
     if (g + 1 < ngroups) load_group(g + 1);
     cp_async_commit();
+    if (g > 0) {
+      if (ok) flush(g - 1);
+      fence_before();
+    }
     // column sums of this group (the MMAs read the same tiles)
     {
       const int a = col >> 6, c = (col & 63) >> 3, e = col & 7;

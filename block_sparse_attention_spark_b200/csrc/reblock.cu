@@ -43,6 +43,9 @@ constexpr int NORM_EVERY = 4;      // power-iteration steps between rescalings o
 template <int D>
 __global__ void __launch_bounds__(256)
 whiten_prep_kernel(const double* __restrict__ M, double* __restrict__ Lout, int* status) {
+  // A row-major with an odd row stride (D + 1 doubles): walking a column
+  // then touches a different bank pair on every row
+  constexpr int LDA = D + 1;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   double* A = reinterpret_cast<double*>(smem_raw);
   __shared__ double tr_sh;
@@ -50,11 +53,11 @@ whiten_prep_kernel(const double* __restrict__ M, double* __restrict__ Lout, int*
   const int tid = threadIdx.x, bh = blockIdx.x;
   const int warp = tid >> 5, lane = tid & 31, nwarps = blockDim.x >> 5;
   const double* Mb = M + (size_t)bh * D * D;
-  for (int e = tid; e < D * D; e += blockDim.x) A[e] = Mb[e];
+  for (int e = tid; e < D * D; e += blockDim.x) A[(e / D) * LDA + e % D] = Mb[e];
   __syncthreads();
   if (tid == 0) {
     double tr = 0.0;
-    for (int i = 0; i < D; ++i) tr += A[i * D + i];
+    for (int i = 0; i < D; ++i) tr += A[i * LDA + i];
     tr_sh = tr;
   }
   __syncthreads();
@@ -64,32 +67,32 @@ whiten_prep_kernel(const double* __restrict__ M, double* __restrict__ Lout, int*
     for (int e = tid; e < D * D; e += blockDim.x) L[e] = (e / D == e % D) ? 1.0 : 0.0;
     return;
   }
-  if (tid < D) A[tid * D + tid] += REG_EPS * (tr / D);
+  if (tid < D) A[tid * LDA + tid] += REG_EPS * (tr / D);
   __syncthreads();
   for (int j = 0; j < D; ++j) {
     if (tid == 0) {
-      const double piv = A[j * D + j];
+      const double piv = A[j * LDA + j];
       if (!(piv > 0.0)) set_status(status, STATUS_BAD_PIVOT);
-      A[j * D + j] = piv > 0.0 ? sqrt(piv) : 0.0;
+      A[j * LDA + j] = piv > 0.0 ? sqrt(piv) : 0.0;
     }
     __syncthreads();
-    const double dj = A[j * D + j];
+    const double dj = A[j * LDA + j];
     for (int i = j + 1 + tid; i < D; i += blockDim.x) {
-      const double l = dj > 0.0 ? A[i * D + j] / dj : 0.0;
-      A[i * D + j] = l;
+      const double l = dj > 0.0 ? A[i * LDA + j] / dj : 0.0;
+      A[i * LDA + j] = l;
       colj[i] = l;
     }
     __syncthreads();
     // trailing update of the lower triangle: warp per row, lanes along it
     for (int i = j + 1 + warp; i < D; i += nwarps) {
       const double li = colj[i];
-      for (int kk = j + 1 + lane; kk <= i; kk += 32) A[i * D + kk] -= li * colj[kk];
+      for (int kk = j + 1 + lane; kk <= i; kk += 32) A[i * LDA + kk] -= li * colj[kk];
     }
     __syncthreads();
   }
   for (int e = tid; e < D * D; e += blockDim.x) {
     const int i = e / D, j = e % D;
-    L[e] = (j <= i) ? A[e] : 0.0;
+    L[e] = (j <= i) ? A[i * LDA + j] : 0.0;
   }
 }
 
@@ -1349,7 +1352,7 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
   int2* nodes = ws_at<int2>(ws, pl.off_nodes);
   cudaError_t e;
 
-  const size_t smem_w = sizeof(double) * D * D;
+  const size_t smem_w = sizeof(double) * D * (D + 1);
   e = cudaFuncSetAttribute(whiten_prep_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_w);
   if (e != cudaSuccess) return e;
   whiten_prep_kernel<D><<<pl.BH, 256, smem_w, s>>>(M, L, status);

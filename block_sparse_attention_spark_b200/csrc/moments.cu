@@ -13,9 +13,10 @@
 // range of 64-token tiles of one head, widens each tile to float64 in shared
 // memory (double-buffered, the next tile's global loads in flight during the
 // current tile's MMAs) and accumulates the upper-triangle tiles of X^T X in
-// registers (72 of the 128 16x8 tiles for d = 128); with COLSUM also the
-// exact float64 column sums. Kernel 1b (moments_colsum): the column sums
-// alone, for the anchor when the query moment is not needed. Kernel 2
+// registers (72 of the 128 16x8 tiles for d = 128, five per warp of 16);
+// with COLSUM also the exact float64 column sums. Kernel 1b
+// (moments_colsum): the column sums alone, for the anchor when the query
+// moment is not needed. Kernel 2
 // (moments_reduce) adds a head's partials in a fixed order, mirrors the
 // triangle and divides by N. The number of token chunks depends on N only, so
 // a head's sums are the same whatever else shares the call.
@@ -24,22 +25,25 @@
 
 namespace spark {
 
+constexpr int MOM_THREADS = 512;                      // 16 warps: four per scheduler keep the MMA pipe fed
+
 template <int D>
 struct MomSmem {
   static constexpr int TT = BLK;                      // tokens per tile
   static constexpr int LD = D + 4;                    // float64 row stride (conflict-free fragments)
   static constexpr int TILE = TT * LD;                // doubles per tile buffer
   static constexpr size_t bytes = sizeof(double) * 2 * TILE;
-  static constexpr int CPT = TT * (D / 8) / 256;      // 16-byte chunks per thread and tile
+  static constexpr int CPT = TT * (D / 8) / MOM_THREADS;   // 16-byte chunks per thread and tile
 };
 
 template <int D, bool COLSUM>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(MOM_THREADS, 1)
 moments_gram64_kernel(const uint16_t* __restrict__ X, int N, int blocks_per_split, double* __restrict__ part) {
   using SM = MomSmem<D>;
   using TRI = TriTiles<D>;
   constexpr int LD = SM::LD;
-  constexpr int SLOTS = (TRI::PAIRS + 7) / 8;         // tiles per warp
+  constexpr int NW = MOM_THREADS / 32;
+  constexpr int SLOTS = (TRI::PAIRS + NW - 1) / NW;   // tiles per warp
   extern __shared__ __align__(16) double msm[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
   const int split = blockIdx.x, bh = blockIdx.y, splits = gridDim.x;
@@ -69,14 +73,14 @@ moments_gram64_kernel(const uint16_t* __restrict__ X, int N, int blocks_per_spli
   auto fetch = [&](int t) {
 #pragma unroll
     for (int i = 0; i < SM::CPT; ++i) {
-      const int c = tid + 256 * i, r = c / (D / 8), ch = c % (D / 8);
+      const int c = tid + MOM_THREADS * i, r = c / (D / 8), ch = c % (D / 8);
       pre[i] = __ldg(reinterpret_cast<const uint4*>(Xh + ((size_t)t * BLK + r) * D + ch * 8));
     }
   };
   auto stash = [&](int buf) {
 #pragma unroll
     for (int i = 0; i < SM::CPT; ++i) {
-      const int c = tid + 256 * i, r = c / (D / 8), ch = c % (D / 8);
+      const int c = tid + MOM_THREADS * i, r = c / (D / 8), ch = c % (D / 8);
       bf8_to_f64(pre[i], msm + buf * SM::TILE + r * LD + ch * 8, lane);
     }
   };
@@ -214,7 +218,7 @@ static cudaError_t run_moments(const Plan& pl, const uint16_t* q, const uint16_t
     e = cudaFuncSetAttribute(moments_gram64_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SM::bytes);
     if (e != cudaSuccess) return e;
-    moments_gram64_kernel<D, true><<<dim3(splits, pl.BH), 256, SM::bytes, s>>>(q, pl.N, bps, part);
+    moments_gram64_kernel<D, true><<<dim3(splits, pl.BH), MOM_THREADS, SM::bytes, s>>>(q, pl.N, bps, part);
   } else {
     moments_colsum_kernel<D><<<dim3(splits, pl.BH), 256, 0, s>>>(q, pl.N, bps, part);
   }
@@ -222,7 +226,7 @@ static cudaError_t run_moments(const Plan& pl, const uint16_t* q, const uint16_t
     e = cudaFuncSetAttribute(moments_gram64_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SM::bytes);
     if (e != cudaSuccess) return e;
-    moments_gram64_kernel<D, false><<<dim3(splits, pl.BH), 256, SM::bytes, s>>>(k, pl.N, bps, part + tstride);
+    moments_gram64_kernel<D, false><<<dim3(splits, pl.BH), MOM_THREADS, SM::bytes, s>>>(k, pl.N, bps, part + tstride);
   }
   moments_reduce_kernel<D><<<dim3(pl.BH, 2, D / 8), 256, 0, s>>>(part, splits, pl.N, MQ, MK, qmean,
                                                                  (gram_q ? 1 : 0) | (gram_k ? 2 : 0));

@@ -117,22 +117,29 @@ whiten_prep_kernel(const double* __restrict__ M, double* __restrict__ Lout, int*
 // Persistent CTAs, one per SM, each take a balanced contiguous range of the
 // layer's (head, 16-token tile) items, in segments of one head: per segment
 // the CTA loads that head's factor L into shared memory (float64), then its
-// eight warps each take their own tiles of the segment: rows staged as bf16
-// through a warp-private cp.async double buffer, widened to float64 as the A
-// fragments are read, 72 of the 128 16x8x16 products of the tile (the
-// k-chunks above the diagonal of L are skipped), the row norms by shuffles
-// inside the warp, and the bf16 rows written back through the staging
-// buffer just consumed. CTA-wide barriers only around the loads of L.
+// sixteen warps work in pairs, each pair on its own 16-token tiles: rows
+// staged as bf16 through a pair-private cp.async double buffer, widened to
+// float64 as the A fragments are read; each warp of the pair takes half of
+// the tile's 8-column output tiles ({0, 3, 4, 7, ...} and {1, 2, 5, 6, ...}:
+// 36 of the 72 16x8x16 products each, the k-chunks above the diagonal of L
+// being skipped); the two halves of each row norm meet in shared memory
+// behind a 64-thread named barrier, and the bf16 rows go back through the
+// staging buffer just consumed. Four warps per scheduler keep the float64
+// MMA pipe fed; CTA-wide barriers only around the loads of L.
 template <int D>
 struct NormSmem {
   static constexpr int LD = D + 4;                    // float64 row stride of L (conflict-free fragments)
   static constexpr int RS = D + 8;                    // bf16 row stride of a staged tile
-  static constexpr int TOK = 16;                      // tokens per warp tile
+  static constexpr int TOK = 16;                      // tokens per pair tile
+  static constexpr int THREADS = 512;
+  static constexpr int NP = THREADS / 64;             // warp pairs
   static constexpr int WTILE = TOK * RS;              // bf16 elements per staged tile
   static constexpr size_t off_x = sizeof(double) * D * LD;
-  static constexpr size_t bytes = off_x + sizeof(uint16_t) * 8 * 2 * WTILE;
+  static constexpr size_t off_n = off_x + sizeof(uint16_t) * NP * 2 * WTILE;
+  static constexpr size_t bytes = off_n + sizeof(double) * NP * 2 * TOK;   // row-norm halves [pair][half][token]
   static constexpr int CT = D / 8, KC = D / 16;
-  static constexpr int CH = TOK * (D / 8) / 32;       // 16-byte chunks per lane and tile
+  static constexpr int CPW = CT / 2;                  // 8-column output tiles per warp
+  static constexpr int CH = TOK * (D / 8) / 64;       // 16-byte chunks per thread of a pair and tile
 };
 
 // bf16 bits of u / r for a pair (u0, u1), low half u0; rinv = 1 / r.
@@ -148,15 +155,22 @@ __device__ __forceinline__ uint32_t bf16x2_of_quotients(double u0, double u1, do
 }
 
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(NormSmem<D>::THREADS, 1)
 normalize64_kernel(const uint16_t* __restrict__ X, const double* __restrict__ Lall, int N, int BH,
                    uint16_t* __restrict__ uhat) {
   using SM = NormSmem<D>;
-  constexpr int LD = SM::LD, RS = SM::RS, TOK = SM::TOK, CT = SM::CT, KC = SM::KC;
+  constexpr int LD = SM::LD, RS = SM::RS, TOK = SM::TOK, KC = SM::KC, CPW = SM::CPW, NP = SM::NP;
   extern __shared__ __align__(16) unsigned char nsm_raw[];
   double* Ls = reinterpret_cast<double*>(nsm_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
-  uint16_t* Xw = reinterpret_cast<uint16_t*>(nsm_raw + SM::off_x) + warp * 2 * SM::WTILE;
+  const int pw = warp >> 1, hh = warp & 1, ptid = tid & 63;
+  uint16_t* Xw = reinterpret_cast<uint16_t*>(nsm_raw + SM::off_x) + pw * 2 * SM::WTILE;
+  double* nsq = reinterpret_cast<double*>(nsm_raw + SM::off_n) + pw * 2 * TOK;
+  auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(1 + pw) : "memory"); };
+  // this warp's output tiles: (c % 4) in {0, 3} for the first warp of a pair, {1, 2} for the second
+  int cs[CPW];
+#pragma unroll
+  for (int j = 0; j < CPW; ++j) cs[j] = 4 * (j >> 1) + ((j & 1) ? (hh ? 2 : 3) : (hh ? 1 : 0));
   const int ntile = N / TOK;
   const long items = (long)BH * ntile;
   const long i0 = items * blockIdx.x / gridDim.x, i1 = items * (blockIdx.x + 1) / gridDim.x;
@@ -168,7 +182,7 @@ normalize64_kernel(const uint16_t* __restrict__ X, const double* __restrict__ La
     __syncthreads();                                   // every warp is done with the previous head's L
     {
       const double2* Lg = reinterpret_cast<const double2*>(Lall + (size_t)bh * D * D);
-      for (int e = tid; e < D * D / 2; e += 256) {
+      for (int e = tid; e < D * D / 2; e += SM::THREADS) {
         const int i = (2 * e) / D, j = (2 * e) % D;
         *reinterpret_cast<double2*>(Ls + i * LD + j) = Lg[e];
       }
@@ -179,24 +193,24 @@ normalize64_kernel(const uint16_t* __restrict__ X, const double* __restrict__ La
     auto load = [&](int t, int buf) {
 #pragma unroll
       for (int i = 0; i < SM::CH; ++i) {
-        const int c = lane + 32 * i, r = c / (D / 8), ch = c % (D / 8);
+        const int c = ptid + 64 * i, r = c / (D / 8), ch = c % (D / 8);
         cp_async16(Xw + buf * SM::WTILE + r * RS + ch * 8, Xh + ((size_t)t * TOK + r) * D + ch * 8);
       }
     };
-    int t = c0 + warp, buf = 0;
+    int t = c0 + pw, buf = 0;
     if (t < c1) load(t, 0);
     cp_async_commit();
-    for (; t < c1; t += 8, buf ^= 1) {
-      if (t + 8 < c1) load(t + 8, buf ^ 1);
+    for (; t < c1; t += NP, buf ^= 1) {
+      if (t + NP < c1) load(t + NP, buf ^ 1);
       cp_async_commit();
       cp_async_wait<1>();
-      __syncwarp();
-      const uint16_t* xs = Xw + buf * SM::WTILE;
-      double acc[CT][4];
+      pair_sync();                                     // both warps' copies of this tile have landed
+      uint16_t* xs = Xw + buf * SM::WTILE;
+      double acc[CPW][4];
 #pragma unroll
-      for (int c = 0; c < CT; ++c)
+      for (int j = 0; j < CPW; ++j)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[c][e] = 0.0;
+        for (int e = 0; e < 4; ++e) acc[j][e] = 0.0;
 #pragma unroll
       for (int kc = 0; kc < KC; ++kc) {
         // A = the tile's tokens x dims 16 kc..: a[i] = x[g + 8 (i % 2)][16 kc + t + 4 (i / 2)]
@@ -204,47 +218,52 @@ normalize64_kernel(const uint16_t* __restrict__ X, const double* __restrict__ La
 #pragma unroll
         for (int i = 0; i < 8; ++i) a[i] = (double)bf2f(xs[(g + 8 * (i % 2)) * RS + 16 * kc + t4 + 4 * (i / 2)]);
 #pragma unroll
-        for (int c = 0; c < CT; ++c) {
-          if (kc < (c >> 1)) continue;                   // L is zero above its diagonal
+        for (int j = 0; j < CPW; ++j) {
+          if (kc < (cs[j] >> 1)) continue;             // L is zero above its diagonal (warp-uniform)
           double b[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) b[i] = Ls[(16 * kc + t4 + 4 * i) * LD + 8 * c + g];
-          dmma16816(acc[c], a, b);
+          for (int i = 0; i < 4; ++i) b[i] = Ls[(16 * kc + t4 + 4 * i) * LD + 8 * cs[j] + g];
+          dmma16816(acc[j], a, b);
         }
       }
-      // |u|^2 of tokens g and g + 8: this lane's columns, then the 4 lanes of the row
+      // |u|^2 of tokens g and g + 8: this warp's columns, then the other half of the pair
       double s0 = 0.0, s1 = 0.0;
 #pragma unroll
-      for (int c = 0; c < CT; ++c) {
-        s0 = fma(acc[c][0], acc[c][0], s0);
-        s0 = fma(acc[c][1], acc[c][1], s0);
-        s1 = fma(acc[c][2], acc[c][2], s1);
-        s1 = fma(acc[c][3], acc[c][3], s1);
+      for (int j = 0; j < CPW; ++j) {
+        s0 = fma(acc[j][0], acc[j][0], s0);
+        s0 = fma(acc[j][1], acc[j][1], s0);
+        s1 = fma(acc[j][2], acc[j][2], s1);
+        s1 = fma(acc[j][3], acc[j][3], s1);
       }
       s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
       s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
       s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
       s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
-      const double r0 = sqrt(s0), r1 = sqrt(s1);
-      const double i0 = r0 > 0.0 ? 1.0 / r0 : 0.0, i1 = r1 > 0.0 ? 1.0 / r1 : 0.0;
-      __syncwarp();                                      // every lane is done reading the staged rows
-      uint16_t* os = Xw + buf * SM::WTILE;
+      if (t4 == 0) {
+        nsq[hh * TOK + g] = s0;
+        nsq[hh * TOK + g + 8] = s1;
+      }
+      pair_sync();                                     // both halves in place; both warps done with xs
+      const double n0 = nsq[g] + nsq[TOK + g], n1 = nsq[g + 8] + nsq[TOK + g + 8];
+      const double r0 = sqrt(n0), r1 = sqrt(n1);
+      const double inv0 = r0 > 0.0 ? 1.0 / r0 : 0.0, inv1 = r1 > 0.0 ? 1.0 / r1 : 0.0;
+      uint16_t* os = xs;
 #pragma unroll
-      for (int c = 0; c < CT; ++c) {
-        const int col = 8 * c + 2 * t4;
-        const uint32_t w0 = r0 > 0.0 ? bf16x2_of_quotients(acc[c][0], acc[c][1], r0, i0) : 0u;
-        const uint32_t w1 = r1 > 0.0 ? bf16x2_of_quotients(acc[c][2], acc[c][3], r1, i1) : 0u;
+      for (int j = 0; j < CPW; ++j) {
+        const int col = 8 * cs[j] + 2 * t4;
+        const uint32_t w0 = r0 > 0.0 ? bf16x2_of_quotients(acc[j][0], acc[j][1], r0, inv0) : 0u;
+        const uint32_t w1 = r1 > 0.0 ? bf16x2_of_quotients(acc[j][2], acc[j][3], r1, inv1) : 0u;
         *reinterpret_cast<uint32_t*>(os + g * RS + col) = w0;
         *reinterpret_cast<uint32_t*>(os + (g + 8) * RS + col) = w1;
       }
-      __syncwarp();
+      pair_sync();                                     // the staged bf16 rows are complete
 #pragma unroll
       for (int i = 0; i < SM::CH; ++i) {
-        const int c = lane + 32 * i, r = c / (D / 8), ch = c % (D / 8);
+        const int c = ptid + 64 * i, r = c / (D / 8), ch = c % (D / 8);
         *reinterpret_cast<uint4*>(Uh + ((size_t)t * TOK + r) * D + ch * 8) =
             *reinterpret_cast<const uint4*>(os + r * RS + ch * 8);
       }
-      __syncwarp();                                      // the buffer is refilled two tiles on
+      pair_sync();                                     // staging read and norms used: both may be reused
     }
     cp_async_wait<0>();
   }
@@ -1365,7 +1384,8 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
     e = cudaFuncSetAttribute(normalize64_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)NormSmem<D>::bytes);
     if (e != cudaSuccess) return e;
-    normalize64_kernel<D><<<(int)std::min<long>(items, sms), 256, NormSmem<D>::bytes, s>>>(x, L, pl.N, pl.BH, uhat);
+    normalize64_kernel<D><<<(int)std::min<long>(items, sms), NormSmem<D>::THREADS, NormSmem<D>::bytes, s>>>(
+        x, L, pl.N, pl.BH, uhat);
   }
 
   tree_build_kernel<<<1, 32, 0, s>>>(pl.nb, nodes);

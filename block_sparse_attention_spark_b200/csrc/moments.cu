@@ -13,7 +13,8 @@
 // range of 64-token tiles of one head, widens each tile to float64 in shared
 // memory (double-buffered, the next tile's global loads in flight during the
 // current tile's MMAs) and accumulates the upper-triangle tiles of X^T X in
-// registers (72 of the 128 16x8 tiles for d = 128, five per warp of 16);
+// registers (72 of the 128 16x8 tiles for d = 128: five for warps 0-7 and
+// four for warps 8-15, 18 per scheduler);
 // with COLSUM also the exact float64 column sums. Kernel 1b
 // (moments_colsum): the column sums alone, for the anchor when the query
 // moment is not needed. Kernel 2
@@ -42,8 +43,13 @@ moments_gram64_kernel(const uint16_t* __restrict__ X, int N, int blocks_per_spli
   using SM = MomSmem<D>;
   using TRI = TriTiles<D>;
   constexpr int LD = SM::LD;
+  // PAIRS = NW * base + extra tiles: warps below `extra` take base + 1, the
+  // rest base, so that every scheduler (warps w, w + 4, ...) gets the same
+  // share (extra is a multiple of 4 for d = 64 and d = 128)
   constexpr int NW = MOM_THREADS / 32;
-  constexpr int SLOTS = (TRI::PAIRS + NW - 1) / NW;   // tiles per warp
+  constexpr int BASE = TRI::PAIRS / NW, EXTRA = TRI::PAIRS - BASE * NW;
+  constexpr int SLOTS = BASE + (EXTRA > 0 ? 1 : 0);  // tiles per warp, at most
+  static_assert(EXTRA % 4 == 0, "equal shares per scheduler");
   extern __shared__ __align__(16) double msm[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
   const int split = blockIdx.x, bh = blockIdx.y, splits = gridDim.x;
@@ -54,10 +60,11 @@ moments_gram64_kernel(const uint16_t* __restrict__ X, int N, int blocks_per_spli
 
   int pr[SLOTS], pc[SLOTS];
   bool pv[SLOTS];
+  const int first = warp * BASE + min(warp, EXTRA), count = BASE + (warp < EXTRA ? 1 : 0);
 #pragma unroll
   for (int s = 0; s < SLOTS; ++s) {
-    const int p = warp * SLOTS + s;
-    pv[s] = p < TRI::PAIRS;
+    const int p = first + s;
+    pv[s] = s < count;
     pr[s] = 0;
     pc[s] = 0;
     if (pv[s]) TRI::decode(p, pr[s], pc[s]);

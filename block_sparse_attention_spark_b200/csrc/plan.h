@@ -50,6 +50,7 @@ struct Plan {
   size_t total = 0;
   // extra device room used by spark_forward_host
   size_t off_hq = 0, off_hk = 0, off_hv = 0, off_hout = 0, off_hlse = 0;
+  size_t host_slice = 0;   // spark_forward_host: workspace bytes of one compute lane
   size_t host_total = 0;
 };
 

@@ -48,7 +48,27 @@ static spark_status validate(const spark_params* p) {
 
 static size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
 
-bool make_plan(const spark_params* p, Plan* pl) {
+// spark_forward_host runs the flattened B*H heads as HOST_CHUNKS chunks of
+// consecutive heads (fewer when there are fewer heads), each a problem of its
+// own (B = 1, H = its heads), computed on HOST_LANES lanes: chunk c on lane
+// c % lanes, in that lane's slice of the workspace.
+constexpr int HOST_CHUNKS = 8;
+constexpr int HOST_LANES = 2;
+static int host_chunks(int BH) { return std::min(BH, HOST_CHUNKS); }
+static int host_lanes(int BH) { return std::min(host_chunks(BH), HOST_LANES); }
+static int host_head0(int BH, int c) { return (int)(((long)BH * c) / host_chunks(BH)); }
+static spark_params host_chunk_params(const spark_params* p, int BH, int c) {
+  spark_params pc = *p;
+  pc.B = 1;
+  pc.H = host_head0(BH, c + 1) - host_head0(BH, c);
+  return pc;
+}
+
+static bool make_plan_impl(const spark_params* p, Plan* pl, bool host);
+
+bool make_plan(const spark_params* p, Plan* pl) { return make_plan_impl(p, pl, true); }
+
+static bool make_plan_impl(const spark_params* p, Plan* pl, bool host) {
   if (validate(p) != SPARK_OK) return false;
   Plan& P = *pl;
   P = Plan();
@@ -151,6 +171,17 @@ bool make_plan(const spark_params* p, Plan* pl) {
     P.off_scores = take((size_t)P.score_heads * per_head);
   }
   P.total = o;
+  if (!host) return true;
+  // host-buffer pass: one workspace slice per lane, large enough for the
+  // largest chunk's plan, then device copies of q, k, v, out and lse
+  P.host_slice = 0;
+  for (int c = 0; c < host_chunks(P.BH); ++c) {
+    const spark_params pc = host_chunk_params(p, P.BH, c);
+    Plan plc;
+    if (!make_plan_impl(&pc, &plc, false)) return false;
+    P.host_slice = std::max(P.host_slice, align_up(plc.total));
+  }
+  o = (size_t)host_lanes(P.BH) * P.host_slice;
   P.off_hq = take(BH * N * d * 2);
   P.off_hk = take(BH * N * d * 2);
   P.off_hv = take(BH * N * d * 2);
@@ -380,10 +411,9 @@ spark_status spark_forward(const spark_params* p, const void* q, const void* k, 
 // Copy streams and events of the host-buffer entry point, one set per device,
 // created on first use and kept for the life of the process.
 namespace {
-constexpr int HOST_CHUNKS = 4;             // head chunks pipelined through copy-in, compute, copy-out
 constexpr int HOST_MAX_DEVICES = 64;
 struct HostPipe {
-  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaStream_t h2d = nullptr, d2h = nullptr, lane[HOST_LANES] = {};
   cudaEvent_t entry = nullptr, done = nullptr, in[HOST_CHUNKS] = {}, comp[HOST_CHUNKS] = {};
   bool ready = false;
 };
@@ -402,6 +432,8 @@ HostPipe* host_pipe() {                     // call with g_host_mu held
     for (int c = 0; ok && c < HOST_CHUNKS; ++c)
       ok = cudaEventCreateWithFlags(&hp.in[c], cudaEventDisableTiming) == cudaSuccess &&
            cudaEventCreateWithFlags(&hp.comp[c], cudaEventDisableTiming) == cudaSuccess;
+    for (int l = 0; ok && l < HOST_LANES; ++l)
+      ok = cudaStreamCreateWithFlags(&hp.lane[l], cudaStreamNonBlocking) == cudaSuccess;
     if (!ok) return nullptr;
     hp.ready = true;
   }
@@ -409,18 +441,21 @@ HostPipe* host_pipe() {                     // call with g_host_mu held
 }
 }  // namespace
 
-// Heads are independent, so the pass runs in up to HOST_CHUNKS chunks of
-// consecutive heads: chunk c + 1 is copied in (one copy stream) while chunk c
-// is computed on the caller's stream and chunk c - 1 is copied out (a second
-// copy stream). The copies start after the work already queued on the
-// caller's stream, and the caller's stream waits for the last copy out.
+// Heads are independent, so the pass runs as up to HOST_CHUNKS chunks of
+// consecutive heads: the chunks are copied in one after another (one copy
+// stream), each is computed as soon as it has arrived on one of HOST_LANES
+// compute streams (chunk c on lane c % lanes, in the lane's workspace slice,
+// so two chunks' kernels can share the GPU: one chunk's latency-bound
+// partition fills the SMs another chunk's attention leaves idle), and copied
+// out when done (a second copy stream). Everything starts after the work
+// already queued on the caller's stream, which waits for the last copy out.
 spark_status spark_forward_host(const spark_params* p, const void* q_host, const void* k_host,
                                 const void* v_host, void* out_host, float* lse_host, void* ws,
                                 size_t ws_bytes, cudaStream_t stream) {
   const spark_status vs = validate(p);
   if (vs != SPARK_OK) return vs;
   Plan pl;
-  make_plan(p, &pl);
+  if (!make_plan(p, &pl)) return SPARK_ERR_INVALID_ARG;
   if (!q_host || !k_host || !v_host || !out_host) return SPARK_ERR_INVALID_ARG;
   if (ws == nullptr || !aligned16(ws)) return SPARK_ERR_INVALID_ARG;
   if (ws_bytes < pl.host_total) return SPARK_ERR_WORKSPACE;
@@ -430,18 +465,14 @@ spark_status spark_forward_host(const spark_params* p, const void* q_host, const
   char* dout = ws_at<char>(ws, pl.off_hout);
   float* dlse = lse_host ? ws_at<float>(ws, pl.off_hlse) : nullptr;
   const size_t head_bytes = (size_t)pl.N * pl.d * 2;   // one head of q, k, v or out
-  const int nch = std::min(pl.BH, HOST_CHUNKS);
+  const int nch = host_chunks(pl.BH), lanes = host_lanes(pl.BH);
 
-  // every chunk is a problem of its own (B = 1, H = its heads) run in this
-  // workspace: check them all before anything is queued
-  auto head0 = [&](int c) { return (int)(((long)pl.BH * c) / nch); };
+  // every chunk must fit its lane's slice: check them all before anything is queued
   for (int c = 0; c < nch; ++c) {
-    spark_params pc = *p;
-    pc.B = 1;
-    pc.H = head0(c + 1) - head0(c);
+    const spark_params pc = host_chunk_params(p, pl.BH, c);
     Plan plc;
     if (validate(&pc) != SPARK_OK || !make_plan(&pc, &plc)) return SPARK_ERR_INVALID_ARG;
-    if (plc.total > pl.total) return SPARK_ERR_WORKSPACE;
+    if (plc.total > pl.host_slice) return SPARK_ERR_WORKSPACE;
   }
   std::lock_guard<std::mutex> guard(g_host_mu);
   HostPipe* hp = host_pipe();
@@ -449,8 +480,11 @@ spark_status spark_forward_host(const spark_params* p, const void* q_host, const
   if (cudaEventRecord(hp->entry, stream) != cudaSuccess) return SPARK_ERR_CUDA;
   if (cudaStreamWaitEvent(hp->h2d, hp->entry, 0) != cudaSuccess) return SPARK_ERR_CUDA;
   if (cudaStreamWaitEvent(hp->d2h, hp->entry, 0) != cudaSuccess) return SPARK_ERR_CUDA;
+  for (int l = 0; l < lanes; ++l)
+    if (cudaStreamWaitEvent(hp->lane[l], hp->entry, 0) != cudaSuccess) return SPARK_ERR_CUDA;
   for (int c = 0; c < nch; ++c) {
-    const size_t off = (size_t)head0(c) * head_bytes, len = (size_t)(head0(c + 1) - head0(c)) * head_bytes;
+    const int h0 = host_head0(pl.BH, c), h1 = host_head0(pl.BH, c + 1);
+    const size_t off = (size_t)h0 * head_bytes, len = (size_t)(h1 - h0) * head_bytes;
     if (cudaMemcpyAsync(dq + off, (const char*)q_host + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
         cudaMemcpyAsync(dk + off, (const char*)k_host + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
         cudaMemcpyAsync(dv + off, (const char*)v_host + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
@@ -458,19 +492,17 @@ spark_status spark_forward_host(const spark_params* p, const void* q_host, const
       return SPARK_ERR_CUDA;
   }
   for (int c = 0; c < nch; ++c) {
-    const int h0 = head0(c), hc = head0(c + 1) - h0;
+    const int h0 = host_head0(pl.BH, c), hc = host_head0(pl.BH, c + 1) - h0;
     const size_t off = (size_t)h0 * head_bytes, len = (size_t)hc * head_bytes;
-    // the chunk as a problem of its own: hc independent heads (the workspace,
-    // sized for all heads, is reused chunk after chunk on this stream)
-    spark_params pc = *p;
-    pc.B = 1;
-    pc.H = hc;
-    if (cudaStreamWaitEvent(stream, hp->in[c], 0) != cudaSuccess) return SPARK_ERR_CUDA;
+    cudaStream_t ls = hp->lane[c % lanes];
+    void* lws = ws_at<char>(ws, (size_t)(c % lanes) * pl.host_slice);
+    const spark_params pc = host_chunk_params(p, pl.BH, c);
+    if (cudaStreamWaitEvent(ls, hp->in[c], 0) != cudaSuccess) return SPARK_ERR_CUDA;
     const spark_status r = spark_forward(&pc, dq + off, dk + off, dv + off, dout + off,
-                                         dlse ? dlse + (size_t)h0 * pl.N : nullptr, nullptr, nullptr, ws, pl.total,
-                                         stream);
+                                         dlse ? dlse + (size_t)h0 * pl.N : nullptr, nullptr, nullptr, lws,
+                                         pl.host_slice, ls);
     if (r != SPARK_OK) return r;
-    if (cudaEventRecord(hp->comp[c], stream) != cudaSuccess) return SPARK_ERR_CUDA;
+    if (cudaEventRecord(hp->comp[c], ls) != cudaSuccess) return SPARK_ERR_CUDA;
     if (cudaStreamWaitEvent(hp->d2h, hp->comp[c], 0) != cudaSuccess) return SPARK_ERR_CUDA;
     if (cudaMemcpyAsync((char*)out_host + off, dout + off, len, cudaMemcpyDeviceToHost, hp->d2h) != cudaSuccess)
       return SPARK_ERR_CUDA;
@@ -478,6 +510,7 @@ spark_status spark_forward_host(const spark_params* p, const void* q_host, const
                                     cudaMemcpyDeviceToHost, hp->d2h) != cudaSuccess)
       return SPARK_ERR_CUDA;
   }
+  // the copy-out stream has waited for every chunk's compute
   if (cudaEventRecord(hp->done, hp->d2h) != cudaSuccess) return SPARK_ERR_CUDA;
   if (cudaStreamWaitEvent(stream, hp->done, 0) != cudaSuccess) return SPARK_ERR_CUDA;
   return SPARK_OK;

@@ -261,18 +261,26 @@ spark_status spark_forward(const spark_params* p, const void* q, const void* k, 
  * invalid. */
 int32_t spark_forward_launches(const spark_params* p);
 
-/* Device bytes spark_forward_host needs: spark_workspace_size() plus room
- * for device copies of q, k, v, out and lse. */
+/* Device bytes spark_forward_host needs: one workspace per compute lane
+ * (below), each spark_workspace_size() of the largest head chunk run as a
+ * problem of its own, plus room for device copies of q, k, v, out and lse of
+ * all heads. At large head counts this is less than spark_workspace_size()
+ * of the whole problem. */
 size_t spark_host_workspace_size(const spark_params* p);
 
 /* The whole pass for HOST tensors (pinned memory recommended): copies q, k,
  * v to the device, runs spark_forward, copies out (and lse if not NULL)
- * back. Heads are independent, so the pass runs in up to four chunks of
- * consecutive heads, pipelined: the next chunk is copied in and the previous
- * one copied out while one is computed. The kernels run on `stream`; the
- * copies run on two copy streams of the library (created on first use per
- * device, kept for the life of the process), which start after the work
- * already queued on `stream`, and `stream` waits for the last copy out.
+ * back. Heads are independent, so the pass runs as up to eight chunks of
+ * consecutive heads (B*H flattened), each a problem of its own (B = 1,
+ * H = its heads; results equal spark_forward's on the whole problem bit for
+ * bit), pipelined: chunks are copied in one after another on a copy stream,
+ * each is computed once it has arrived on one of two compute streams (chunk
+ * c on stream c % 2, in that stream's own part of ws, so two chunks' kernels
+ * may run at the same time) and copied out when done on a second copy
+ * stream. These four streams belong to the library (created on first use
+ * per device, kept for the life of the process); all of them start after
+ * the work already queued on `stream`, and `stream` waits for the last copy
+ * out.
  * Asynchronous like every call: the host buffers must stay valid until the
  * stream reaches the end of the call. ws is DEVICE memory of
  * spark_host_workspace_size() bytes. Calls from several host threads are

@@ -61,7 +61,20 @@ def test_validate_accepts_workloads():
             assert spark.validate(p) == 0
             assert spark.num_selected(p) == so.num_selected(w.nb, r)
             assert spark.workspace_size(p) > 0
-            assert spark.host_workspace_size(p) > spark.workspace_size(p)
+            assert spark.host_workspace_size(p) >= _host_bytes_at_least(w.B, w.H, w.N, w.d, r)
+
+
+def _host_bytes_at_least(B, H, N, d, r):
+    """The host-buffer pass keeps device copies of q, k, v, out and lse of
+    every head, and one workspace per compute lane (two lanes when there are
+    two or more heads), each for the largest of up to eight head chunks run
+    as problems of their own."""
+    BH = B * H
+    chunks = min(BH, 8)
+    largest = -(-BH // chunks)
+    lanes = min(chunks, 2)
+    staging = 4 * BH * N * d * 2 + BH * N * 4
+    return lanes * spark.workspace_size(spark.params(1, largest, N, d, r)) + staging
 
 
 @pytest.mark.parametrize("kw,code", [

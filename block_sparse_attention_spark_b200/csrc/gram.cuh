@@ -24,14 +24,18 @@ struct Gram {
 
   // Stage 64 rows of D bf16 into smem. rows[r] (if non-null) gives the source
   // row of tile row r, else row0 + r. base points at row 0 of the matrix.
+  // Thread tid copies chunk tid % (D / 8) of rows tid / (D / 8) + RSTEP k;
+  // all of its row indices are read before the first copy is issued.
+  static constexpr int RSTEP = THREADS / (D / 8), LROWS = BLK / RSTEP;
+  static_assert(CHUNKS % THREADS == 0, "whole chunks per thread");
   __device__ static void load_tile(uint16_t* sm, const uint16_t* base, const int32_t* rows,
                                    long row0, int tid) {
+    const int ch = tid % (D / 8), r0 = tid / (D / 8);
+    long src[LROWS];
 #pragma unroll
-    for (int c = tid; c < CHUNKS; c += THREADS) {
-      const int r = c / (D / 8), ch = c % (D / 8);
-      const long src = rows ? (long)rows[r] : row0 + r;
-      cp_async16(sm + r * RS + ch * 8, base + src * D + ch * 8);
-    }
+    for (int k = 0; k < LROWS; ++k) src[k] = rows ? (long)rows[r0 + RSTEP * k] : row0 + r0 + RSTEP * k;
+#pragma unroll
+    for (int k = 0; k < LROWS; ++k) cp_async16(sm + (r0 + RSTEP * k) * RS + ch * 8, base + src[k] * D + ch * 8);
   }
 
   __device__ static void tile_mma(const uint16_t* sm, float (&acc)[ACC], int warp, int lane) {

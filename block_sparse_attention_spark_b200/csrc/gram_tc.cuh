@@ -70,18 +70,31 @@ __device__ void gram_tc_body(const uint16_t* __restrict__ X, RowF rowf, int ntil
   const int ngroups = (ntiles + GT_GROUP - 1) / GT_GROUP;
 
   // cp.async of one group's tiles into ring half g & 1 (128-byte swizzle:
-  // 16-byte chunk c of row r lands at chunk c ^ (r % 8) of the 128-byte row)
+  // 16-byte chunk c of row r lands at chunk c ^ (r % 8) of the 128-byte row).
+  // Thread tid copies chunk tid % 16 of rows tid / 16 + 16 k of each tile;
+  // it reads all of its row indices first, so their latencies overlap and
+  // the copies follow in one burst.
+  constexpr int RSTEP = GT_THREADS / (D / 8), RPT = GT_TOK / RSTEP;
   auto load_group = [&](int g) {
     const uint32_t gb = base + (uint32_t)((g & 1) * L::GROUP);
     const int t0 = g * GT_GROUP;
-    for (int i = tid; i < GT_GROUP * GT_TOK * (D / 8); i += GT_THREADS) {
-      const int tt = i / (GT_TOK * (D / 8)), rem = i % (GT_TOK * (D / 8));
-      const int r = rem / (D / 8), ch = rem % (D / 8);
-      if (t0 + tt >= ntiles) continue;
-      const int a = ch >> 3, c = ch & 7;
-      const uint32_t dst = gb + (uint32_t)(tt * L::TILE + a * L::ATOM + r * 128 + ((c ^ (r & 7)) << 4));
-      const uint16_t* src = X + (size_t)rowf(t0 + tt, r) * D + ch * 8;
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
+    const int ch = tid % (D / 8), r0 = tid / (D / 8);
+    const int a = ch >> 3, c = ch & 7;
+    int src[GT_GROUP][RPT];
+#pragma unroll
+    for (int tt = 0; tt < GT_GROUP; ++tt)
+#pragma unroll
+      for (int k = 0; k < RPT; ++k) src[tt][k] = t0 + tt < ntiles ? (int)rowf(t0 + tt, r0 + RSTEP * k) : 0;
+#pragma unroll
+    for (int tt = 0; tt < GT_GROUP; ++tt) {
+      if (t0 + tt >= ntiles) break;
+#pragma unroll
+      for (int k = 0; k < RPT; ++k) {
+        const int r = r0 + RSTEP * k;
+        const uint32_t dst = gb + (uint32_t)(tt * L::TILE + a * L::ATOM + r * 128 + ((c ^ (r & 7)) << 4));
+        const uint16_t* srcp = X + (size_t)src[tt][k] * D + ch * 8;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(srcp));
+      }
     }
   };
   double acc[64];

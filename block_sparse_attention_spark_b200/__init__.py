@@ -24,7 +24,7 @@ LAYOUTS = {"q_reuse_k": 0, "k_reuse_q": 1, "separate": 2}
 SUMMARIES = {"reweight": 0, "meanpool": 1}
 TAILS = {"query": 0, "block": 1}
 WS = {"MQ": 0, "MK": 1, "QMEAN": 2, "PERM": 3, "SEL": 4, "QM": 5, "KM": 6, "KT": 7, "VT": 8,
-      "BETA": 9, "UHAT": 10}
+      "BETA": 9, "UHAT": 10, "PAIRS": 11}
 STATUS = {0: "SPARK_OK", 1: "SPARK_ERR_INVALID_ARG", 2: "SPARK_ERR_UNSUPPORTED",
           3: "SPARK_ERR_WORKSPACE", 4: "SPARK_ERR_CUDA", 5: "SPARK_ERR_TIMEOUT"}
 

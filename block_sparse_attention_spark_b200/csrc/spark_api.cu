@@ -533,6 +533,7 @@ size_t spark_workspace_region(const spark_params* p, int32_t region, size_t* byt
     case SPARK_WS_VT: off = pl.off_vt; sz = BH * nbp * d * 2; break;
     case SPARK_WS_BETA: off = pl.off_beta; sz = BH * nbp * 4; break;
     case SPARK_WS_UHAT: off = pl.off_uhat; sz = BH * N * d * 2; break;
+    case SPARK_WS_PAIRS: off = pl.off_pairs; sz = BH * ((nb + 1) / 2) * 8; break;
     default: return (size_t)-1;
   }
   if (bytes) *bytes = sz;

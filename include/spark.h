@@ -298,11 +298,13 @@ spark_status spark_forward_host(const spark_params* p, const void* q_host, const
  * [B,H,nb,d] f64 block means, SPARK_WS_KT/VT [B,H,nbp,d] bf16 summaries and
  * SPARK_WS_BETA [B,H,nbp] f32 biases with nbp = nb rounded up to 128 (rows
  * past nb are zero), SPARK_WS_UHAT [B,H,N,d] bf16 normalised whitened
- * tokens of the partitioned side (original token order). */
+ * tokens of the partitioned side (original token order), SPARK_WS_PAIRS
+ * [B,H,(nb+1)/2] pairs of int32 (the query blocks each attention unit runs
+ * together, written by spark_attn_fwd; partner -1 for a lone block). */
 enum {
   SPARK_WS_MQ = 0, SPARK_WS_MK = 1, SPARK_WS_QMEAN = 2, SPARK_WS_PERM = 3, SPARK_WS_SEL = 4,
   SPARK_WS_QM = 5, SPARK_WS_KM = 6, SPARK_WS_KT = 7, SPARK_WS_VT = 8, SPARK_WS_BETA = 9,
-  SPARK_WS_UHAT = 10
+  SPARK_WS_UHAT = 10, SPARK_WS_PAIRS = 11
 };
 size_t spark_workspace_region(const spark_params* p, int32_t region, size_t* bytes);
 

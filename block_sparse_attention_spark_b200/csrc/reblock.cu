@@ -308,8 +308,9 @@ __global__ void init_idx_kernel(int32_t* idx, int N, long total) {
 }
 
 // ------------------------------------------------------------------ block-wide helpers
-// Exclusive prefix count of 0/1 flags over a 256-thread block (and the total).
-__device__ __forceinline__ int block_excl_scan_256(int flag, int* warp_tot, int& total) {
+// Exclusive prefix count of 0/1 flags over a block of NW warps (and the total).
+template <int NW>
+__device__ __forceinline__ int block_excl_scan(int flag, int* warp_tot, int& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const unsigned m = __ballot_sync(0xffffffffu, flag);
   const int within = __popc(m & ((1u << lane) - 1u));
@@ -317,7 +318,7 @@ __device__ __forceinline__ int block_excl_scan_256(int flag, int* warp_tot, int&
   __syncthreads();
   int before = 0, tot = 0;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) {
+  for (int w = 0; w < NW; ++w) {
     const int c = warp_tot[w];
     before += (w < warp) ? c : 0;
     tot += c;
@@ -327,8 +328,9 @@ __device__ __forceinline__ int block_excl_scan_256(int flag, int* warp_tot, int&
   return before + within;
 }
 
-// Exclusive prefix sum of per-thread counts over a 256-thread block (and the total).
-__device__ __forceinline__ int block_excl_sum_256(int v, int* warp_tot, int& total) {
+// Exclusive prefix sum of per-thread counts over a block of NW warps (and the total).
+template <int NW>
+__device__ __forceinline__ int block_excl_sum(int v, int* warp_tot, int& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = v;
 #pragma unroll
@@ -340,7 +342,7 @@ __device__ __forceinline__ int block_excl_sum_256(int v, int* warp_tot, int& tot
   __syncthreads();
   int before = 0, tot = 0;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) {
+  for (int w = 0; w < NW; ++w) {
     const int c = warp_tot[w];
     before += (w < warp) ? c : 0;
     tot += c;
@@ -524,7 +526,7 @@ __device__ void power_iterate_regs(const double (&Sr)[D / 32][D / 8], double* zb
 // rest after them. pkey(i) / pid(i): ordered key and token index of member
 // i; put(dst, i) moves member i to position dst. UNR: members per thread and
 // pass (8 for keys in global memory, 1 for keys in shared memory).
-template <int UNR, class KeyF, class IdF, class PutF>
+template <int UNR, int NW, class KeyF, class IdF, class PutF>
 __device__ void cut_partition(int n, int nL, KeyF pkey, IdF pid, PutF put, int* hist, int* sh_sel,
                               unsigned long long* sh_key, int* warp_tot, int* red_i, int* status) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -544,7 +546,7 @@ __device__ void cut_partition(int n, int nL, KeyF pkey, IdF pid, PutF put, int* 
   __syncthreads();
   if (tid == 0) {
     int a = 0, b = 0;
-    for (int w = 0; w < 8; ++w) { a += red_i[w]; b += warp_tot[w]; }
+    for (int w = 0; w < NW; ++w) { a += red_i[w]; b += warp_tot[w]; }
     sh_sel[0] = a;
     sh_sel[1] = b;
   }
@@ -577,7 +579,7 @@ __device__ void cut_partition(int n, int nL, KeyF pkey, IdF pid, PutF put, int* 
       cnt += gl[u];
     }
     int tot;
-    int l = UNR == 1 ? block_excl_scan_256(cnt, warp_tot, tot) : block_excl_sum_256(cnt, warp_tot, tot);
+    int l = UNR == 1 ? block_excl_scan<NW>(cnt, warp_tot, tot) : block_excl_sum<NW>(cnt, warp_tot, tot);
     int r = max(0, min(tid * UNR, n - base)) - l;              // members before this thread going right
 #pragma unroll
     for (int u = 0; u < UNR; ++u) {
@@ -595,11 +597,12 @@ __device__ void cut_partition(int n, int nL, KeyF pkey, IdF pid, PutF put, int* 
 }
 
 // The cut over a group's projections in global scratch (pv, pi), written
-// over the group's index slice ids.
+// over the group's index slice ids, by a block of NW warps.
+template <int NW>
 __device__ void cut_and_partition(int n, int nL, double sgn, const double* pv, const int32_t* pi,
                                   int32_t* ids, int* hist, int* sh_sel, unsigned long long* sh_key,
                                   int* warp_tot, int* red_i, int* status) {
-  cut_partition<8>(
+  cut_partition<8, NW>(
       n, nL, [&](int i) -> uint64_t { return ordered_key(sgn * pv[i]); }, [&](int i) { return pi[i]; },
       [&](int dst, int i) { ids[dst] = pi[i]; }, hist, sh_sel, sh_key, warp_tot, red_i, status);
 }
@@ -624,6 +627,7 @@ struct SplitSmem {
 // get chunk Gram partials: a right half's Gram sum is its parent's (kept
 // from the level above) minus its sibling's.
 constexpr int BIG_CHUNK_TILES = 32;
+constexpr int BIG_SELECT_WIDE_TOKENS = 8192;   // groups this large: 1024-thread select blocks
 
 template <int D>
 __global__ void __launch_bounds__(256, 1)
@@ -875,15 +879,20 @@ big_project_kernel(const uint16_t* __restrict__ uhat, int N, const int2* __restr
   }
 }
 
-__global__ void __launch_bounds__(256)
+// THREADS = 1024 for the levels with large groups (the select and partition
+// passes are latency-bound loops over the group's keys), 256 below; the cut
+// and the stable order do not depend on it.
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS)
 big_select_kernel(int N, const int2* __restrict__ nodes, int nnodes, int chunks, const double* __restrict__ cand,
                   int32_t* __restrict__ idx, const double* __restrict__ pval, const int32_t* __restrict__ pidx,
                   int* status) {
+  constexpr int NW = THREADS / 32;
   __shared__ int hist[256];
   __shared__ int sh_sel[3];
   __shared__ unsigned long long sh_key;
-  __shared__ int warp_tot[8];
-  __shared__ int red_i[8];
+  __shared__ int warp_tot[NW];
+  __shared__ int red_i[NW];
   __shared__ double sh_sgn;
   const int tid = threadIdx.x, k = blockIdx.x, bh = blockIdx.y;
   const int2 node = nodes[k];
@@ -901,8 +910,8 @@ big_select_kernel(int N, const int2* __restrict__ nodes, int nnodes, int chunks,
   }
   __syncthreads();
   const size_t gpos = (size_t)bh * N + (size_t)node.x * BLK;
-  cut_and_partition(n, nL, sh_sgn, pval + gpos, pidx + gpos, idx + gpos, hist, sh_sel, &sh_key, warp_tot,
-                    red_i, status);
+  cut_and_partition<NW>(n, nL, sh_sgn, pval + gpos, pidx + gpos, idx + gpos, hist, sh_sel, &sh_key, warp_tot,
+                        red_i, status);
 }
 
 // ------------------------------------------------------------------ whole small subtrees
@@ -1234,7 +1243,7 @@ __device__ void sub_finish(const uint16_t* rows, double* pv, const int32_t* ids,
       stok[rank] = lo[tid];
     }
   } else {
-    cut_partition<1>(
+    cut_partition<1, 8>(
         nn, nL, [&](int t) -> uint64_t { return ordered_key(sgn * pv[t]); }, [&](int t) { return ids[lo[t]]; },
         [&](int dst, int t) { stok[dst] = lo[t]; }, hist, sh_sel, sh_key, warp_tot, red_i, status);
   }
@@ -1436,7 +1445,10 @@ static cudaError_t run_reblock(const Plan& pl, const uint16_t* x, const double* 
                                                                    pl.power_iters);
     big_project_kernel<D><<<dim3(ch, cnt, pl.BH), 256, smem_proj, s>>>(uhat, pl.N, nd, cnt, ch, idx, binfo, pval,
                                                                       pidx, bcand);
-    big_select_kernel<<<dim3(cnt, pl.BH), 256, 0, s>>>(pl.N, nd, cnt, ch, bcand, idx, pval, pidx, status);
+    if (pl.level_maxg[lv] * BLK >= BIG_SELECT_WIDE_TOKENS)
+      big_select_kernel<1024><<<dim3(cnt, pl.BH), 1024, 0, s>>>(pl.N, nd, cnt, ch, bcand, idx, pval, pidx, status);
+    else
+      big_select_kernel<256><<<dim3(cnt, pl.BH), 256, 0, s>>>(pl.N, nd, cnt, ch, bcand, idx, pval, pidx, status);
   }
   const long nbt = (long)pl.BH * pl.nb;
   leaf_sort_kernel<<<(int)((nbt + 7) / 8), 256, 0, s>>>(idx, perm, nbt);

@@ -478,10 +478,19 @@ spark_status spark_forward_host(const spark_params* p, const void* q_host, const
   HostPipe* hp = host_pipe();
   if (hp == nullptr) return SPARK_ERR_CUDA;
   if (cudaEventRecord(hp->entry, stream) != cudaSuccess) return SPARK_ERR_CUDA;
-  if (cudaStreamWaitEvent(hp->h2d, hp->entry, 0) != cudaSuccess) return SPARK_ERR_CUDA;
-  if (cudaStreamWaitEvent(hp->d2h, hp->entry, 0) != cudaSuccess) return SPARK_ERR_CUDA;
+  // once anything is queued, a failure still orders the caller's stream after
+  // all of it (the workspace and the host buffers stay in use until then)
+  auto fail = [&](spark_status st) {
+    for (int l = 0; l < lanes; ++l)
+      if (cudaEventRecord(hp->comp[l], hp->lane[l]) == cudaSuccess) cudaStreamWaitEvent(hp->d2h, hp->comp[l], 0);
+    if (cudaEventRecord(hp->in[0], hp->h2d) == cudaSuccess) cudaStreamWaitEvent(hp->d2h, hp->in[0], 0);
+    if (cudaEventRecord(hp->done, hp->d2h) == cudaSuccess) cudaStreamWaitEvent(stream, hp->done, 0);
+    return st;
+  };
+  if (cudaStreamWaitEvent(hp->h2d, hp->entry, 0) != cudaSuccess) return fail(SPARK_ERR_CUDA);
+  if (cudaStreamWaitEvent(hp->d2h, hp->entry, 0) != cudaSuccess) return fail(SPARK_ERR_CUDA);
   for (int l = 0; l < lanes; ++l)
-    if (cudaStreamWaitEvent(hp->lane[l], hp->entry, 0) != cudaSuccess) return SPARK_ERR_CUDA;
+    if (cudaStreamWaitEvent(hp->lane[l], hp->entry, 0) != cudaSuccess) return fail(SPARK_ERR_CUDA);
   for (int c = 0; c < nch; ++c) {
     const int h0 = host_head0(pl.BH, c), h1 = host_head0(pl.BH, c + 1);
     const size_t off = (size_t)h0 * head_bytes, len = (size_t)(h1 - h0) * head_bytes;
@@ -489,7 +498,7 @@ spark_status spark_forward_host(const spark_params* p, const void* q_host, const
         cudaMemcpyAsync(dk + off, (const char*)k_host + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
         cudaMemcpyAsync(dv + off, (const char*)v_host + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
         cudaEventRecord(hp->in[c], hp->h2d) != cudaSuccess)
-      return SPARK_ERR_CUDA;
+      return fail(SPARK_ERR_CUDA);
   }
   for (int c = 0; c < nch; ++c) {
     const int h0 = host_head0(pl.BH, c), hc = host_head0(pl.BH, c + 1) - h0;
@@ -497,22 +506,22 @@ spark_status spark_forward_host(const spark_params* p, const void* q_host, const
     cudaStream_t ls = hp->lane[c % lanes];
     void* lws = ws_at<char>(ws, (size_t)(c % lanes) * pl.host_slice);
     const spark_params pc = host_chunk_params(p, pl.BH, c);
-    if (cudaStreamWaitEvent(ls, hp->in[c], 0) != cudaSuccess) return SPARK_ERR_CUDA;
+    if (cudaStreamWaitEvent(ls, hp->in[c], 0) != cudaSuccess) return fail(SPARK_ERR_CUDA);
     const spark_status r = spark_forward(&pc, dq + off, dk + off, dv + off, dout + off,
                                          dlse ? dlse + (size_t)h0 * pl.N : nullptr, nullptr, nullptr, lws,
                                          pl.host_slice, ls);
-    if (r != SPARK_OK) return r;
-    if (cudaEventRecord(hp->comp[c], ls) != cudaSuccess) return SPARK_ERR_CUDA;
-    if (cudaStreamWaitEvent(hp->d2h, hp->comp[c], 0) != cudaSuccess) return SPARK_ERR_CUDA;
+    if (r != SPARK_OK) return fail(r);
+    if (cudaEventRecord(hp->comp[c], ls) != cudaSuccess) return fail(SPARK_ERR_CUDA);
+    if (cudaStreamWaitEvent(hp->d2h, hp->comp[c], 0) != cudaSuccess) return fail(SPARK_ERR_CUDA);
     if (cudaMemcpyAsync((char*)out_host + off, dout + off, len, cudaMemcpyDeviceToHost, hp->d2h) != cudaSuccess)
-      return SPARK_ERR_CUDA;
+      return fail(SPARK_ERR_CUDA);
     if (lse_host && cudaMemcpyAsync(lse_host + (size_t)h0 * pl.N, dlse + (size_t)h0 * pl.N, (size_t)hc * pl.N * 4,
                                     cudaMemcpyDeviceToHost, hp->d2h) != cudaSuccess)
-      return SPARK_ERR_CUDA;
+      return fail(SPARK_ERR_CUDA);
   }
   // the copy-out stream has waited for every chunk's compute
-  if (cudaEventRecord(hp->done, hp->d2h) != cudaSuccess) return SPARK_ERR_CUDA;
-  if (cudaStreamWaitEvent(stream, hp->done, 0) != cudaSuccess) return SPARK_ERR_CUDA;
+  if (cudaEventRecord(hp->done, hp->d2h) != cudaSuccess) return fail(SPARK_ERR_CUDA);
+  if (cudaStreamWaitEvent(stream, hp->done, 0) != cudaSuccess) return fail(SPARK_ERR_CUDA);
   return SPARK_OK;
 }
 

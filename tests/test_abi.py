@@ -64,6 +64,20 @@ def test_validate_accepts_workloads():
             assert spark.host_workspace_size(p) >= _host_bytes_at_least(w.B, w.H, w.N, w.d, r)
 
 
+@pytest.mark.parametrize("B,H", [(1, 1), (1, 2), (1, 3), (2, 5), (1, 9), (1, 16), (2, 20), (1, 40), (3, 37)])
+def test_host_workspace_holds_two_lanes_and_the_copies(B, H):
+    """The host-buffer pass: room for the device copies of every head plus one
+    workspace per compute lane for the largest head chunk; from 16 heads on
+    (chunks of at most a quarter of the heads, two lanes) that is less than
+    the whole problem's workspace plus the copies."""
+    N, d, r = 64 * 40, 128, 0.2
+    p = spark.params(B, H, N, d, r)
+    staging = 4 * B * H * N * d * 2 + B * H * N * 4
+    assert spark.host_workspace_size(p) >= _host_bytes_at_least(B, H, N, d, r)
+    if B * H >= 16:
+        assert spark.host_workspace_size(p) < spark.workspace_size(p) + staging
+
+
 def _host_bytes_at_least(B, H, N, d, r):
     """The host-buffer pass keeps device copies of q, k, v, out and lse of
     every head, and one workspace per compute lane (two lanes when there are

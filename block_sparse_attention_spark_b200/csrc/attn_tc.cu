@@ -17,21 +17,24 @@
 // tile, each row masking the blocks it selected. One running softmax over
 // both term sets = the log-sum-exp merge of the two branches.
 //
-// A CTA runs two such units side by side in two independent slots (pairs
-// 2c and 2c+1), each with its own Q, K and V buffers and TMEM columns. Each
+// A CTA runs one such unit (SLOTS = 1; the code also runs two units side by
+// side, SLOTS = 2) with its own Q, K and V buffers and 256 TMEM columns, and
+// two CTAs share an SM: one CTA's prologue (selection masks, Q and first K/V
+// loads) and epilogue (O readout, scatter) overlap the other's tiles. The
 // slot double-buffers S in TMEM, so the tensor cores compute S_{j+1} (and
 // P_{j-1} V_{j-1}) while the slot's softmax works on S_j.
 //
-// Roles (384 threads):
-//   warps 0-3  softmax of slot 0, warps 4-7 softmax of slot 1: one thread
-//              per query row (TMEM lane = row), the 64 columns of a tile.
-//              Lazy-rescaled online softmax (the reference max moves only
-//              when the row max grows by more than 2^8); P (bf16 pairs) is
-//              written over the first 32 columns of the tile's S buffer.
-//   warp 8 / 9 TMA producer of slot 0 / 1: Q once, then K_j and V_j of
-//              every tile into two-stage K and V rings.
-//   warp 10/11 MMA-issuing thread of slot 0 / 1 (warp 10 also allocates
-//              TMEM): S_j = Q K_j^T (M128 N64 K=d, K-major smem operands),
+// Roles (192 threads; with SLOTS = 2 the softmax warps are 0-7, the
+// producers 8-9 and the MMA threads 10-11, 384 threads):
+//   warps 0-3  softmax: one thread per query row (TMEM lane = row), the 64
+//              columns of a tile. Lazy-rescaled online softmax (the
+//              reference max moves only when the row max grows by more
+//              than 2^8); P (bf16 pairs) is written over the first 32
+//              columns of the tile's S buffer.
+//   warp 4     TMA producer: Q once, then K_j and V_j of every tile into
+//              two-stage K and V rings.
+//   warp 5     MMA-issuing thread (this warp also allocates TMEM):
+//              S_j = Q K_j^T (M128 N64 K=d, K-major smem operands),
 //              O += P_j V_j (M128 N=d K=64, P read from TMEM, V an MN-major
 //              smem operand). S_{j+2} goes into S_j's buffer after P_j V_j;
 //              the MMAs of one thread complete in issue order, so that
@@ -123,11 +126,15 @@ namespace tc {
 
 constexpr int ROWS = 128;
 constexpr int KEYS = 64;                 // keys (or summaries) per tile = one block
-constexpr int SLOTS = 2;
+constexpr int SLOTS = 1;                 // units per CTA (two CTAs share an SM)
+constexpr int CTAS_PER_SM = 2;
 constexpr int STAGES = 2;                // K and V ring depth per slot
-constexpr int THREADS = 384;
-constexpr uint32_t TMEM_COLS = 512;
+constexpr int SM_WARPS = 4 * SLOTS;      // softmax warps: 4 per slot
+constexpr int PROD_WARP0 = SM_WARPS;     // TMA producer of slot s: warp PROD_WARP0 + s
+constexpr int MMA_WARP0 = SM_WARPS + SLOTS;   // MMA issuer of slot s: warp MMA_WARP0 + s
+constexpr int THREADS = 32 * (SM_WARPS + 2 * SLOTS);
 constexpr uint32_t SLOT_COLS = 256;      // TMEM columns per slot
+constexpr uint32_t TMEM_COLS = SLOT_COLS * SLOTS;
 constexpr uint32_t O_OFF = 128;          // O within a slot's columns
 constexpr float LAZY_RESCALE = 8.0f;     // log2 units
 constexpr int MASK_WORDS = SPARK_MAX_BLOCKS / 32;
@@ -209,7 +216,7 @@ struct Maps {
 // EXT: the block tail granularity or a context segment may be present (an
 // instance without them carries none of their per-tile branches).
 template <int D, bool EXT>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
 attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta, const float* __restrict__ ttab,
                const int32_t* __restrict__ perm, const int32_t* __restrict__ sel, const int2* __restrict__ pairs,
                int N, int nb, int nb_pad, int ksel, uint16_t* __restrict__ out, float* __restrict__ lse, int C,
@@ -262,19 +269,19 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 10) {
+  if (warp == MMA_WARP0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_sh)),
                  "r"(TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   __syncthreads();
   // the unit's two query blocks (video CTAs; context CTAs have no pairs)
-  static_assert(SLOTS == 2, "two units per CTA");
+  static_assert(SLOTS == 1 || SLOTS == 2, "one or two units per CTA");
   auto load_unit = [&](int s) -> int2 {
     const int u = SLOTS * blockIdx.x + s;
     return ((int)blockIdx.x < nvid && u < npairs) ? pairs[(size_t)bh * npairs + u] : make_int2(-1, -1);
   };
-  const int2 unit0 = load_unit(0), unit1 = load_unit(1);
+  const int2 unit0 = load_unit(0), unit1 = SLOTS > 1 ? load_unit(1) : make_int2(-1, -1);
   auto unit_of = [&](int s) -> int2 { return s == 0 ? unit0 : unit1; };
   for (int qb = 0; qb < 2 * SLOTS; ++qb) {
     const int2 un = unit_of(qb >> 1);
@@ -292,22 +299,21 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
   __syncthreads();
   fence_after();
   {
-    int c0 = 0, c1 = 0;
+    int cs[SLOTS];
+#pragma unroll
+    for (int s = 0; s < SLOTS; ++s) cs[s] = 0;
     for (int w = tid; w < nwords; w += THREADS) {
-      const uint32_t u0 = selm[0][0][w] | selm[0][1][w];
-      const uint32_t u1 = selm[1][0][w] | selm[1][1][w];
-      unionm[0][w] = u0;
-      unionm[1][w] = u1;
-      c0 += __popc(u0);
-      c1 += __popc(u1);
+#pragma unroll
+      for (int s = 0; s < SLOTS; ++s) {
+        const uint32_t u = selm[s][0][w] | selm[s][1][w];
+        unionm[s][w] = u;
+        cs[s] += __popc(u);
+      }
     }
-    for (int o = 16; o > 0; o >>= 1) {
-      c0 += __shfl_xor_sync(0xffffffffu, c0, o);
-      c1 += __shfl_xor_sync(0xffffffffu, c1, o);
-    }
-    if (lane == 0) {
-      count_sh[warp][0] = c0;
-      count_sh[warp][1] = c1;
+#pragma unroll
+    for (int s = 0; s < SLOTS; ++s) {
+      for (int o = 16; o > 0; o >>= 1) cs[s] += __shfl_xor_sync(0xffffffffu, cs[s], o);
+      if (lane == 0) count_sh[warp][s] = cs[s];
     }
   }
   __syncthreads();
@@ -335,7 +341,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
   }
   const uint32_t tmem = tmem_base_sh;
 
-  if (warp < 8) {
+  if (warp < SM_WARPS) {
     // ------------------------------------------------ softmax of slot warp / 4, one thread per row
     const int s = warp >> 2;
     const int Ts = T[s], TEs = TE[s], TXs = TX[s];
@@ -532,9 +538,9 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
         if (lse_out != nullptr && dst_ok) lse_out[orow] = (m_ref + log2f(l)) * 0.6931471805599453f;
       }
     }
-  } else if (warp == 8 || warp == 9) {
-    // ------------------------------------------------ TMA producer of slot warp - 8
-    const int s = warp - 8;
+  } else if (warp < MMA_WARP0) {
+    // ------------------------------------------------ TMA producer of slot warp - PROD_WARP0
+    const int s = warp - PROD_WARP0;
     if (lane == 0 && T[s] > 0) {
       const int crow0 = (SLOTS * ((int)blockIdx.x - nvid) + s) * ROWS;   // context CTAs
       mbar_arrive_tx(q_full(s), L::Q_BYTES);
@@ -599,8 +605,8 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
       issued_sh[s][1] = iv;
     }
   } else {
-    // ------------------------------------------------ MMA issuer of slot warp - 10
-    const int s = warp - 10;
+    // ------------------------------------------------ MMA issuer of slot warp - MMA_WARP0
+    const int s = warp - MMA_WARP0;
     if (lane == 0 && T[s] > 0) {
       const int Ts = T[s];
       bool ok = true;
@@ -667,25 +673,25 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ beta
   __syncthreads();
   fence_after();
   if (abort_sh) {
-    if ((warp == 8 || warp == 9) && lane == 0) {
+    if (warp >= PROD_WARP0 && warp < MMA_WARP0 && lane == 0) {
       // copies issued but never observed by the MMA thread
-      const int s = warp - 8;
+      const int s = warp - PROD_WARP0;
       if (T[s] > 0 && !q_seen_sh[s]) mbar_wait(q_full(s), 0, status);
       for (int j = consumed_sh[s][0]; j < issued_sh[s][0]; ++j)
         mbar_wait(k_full(s, j % STAGES), (uint32_t)(j / STAGES) & 1u, status);
       for (int j = consumed_sh[s][1]; j < issued_sh[s][1]; ++j)
         mbar_wait(v_full(s, j % STAGES), (uint32_t)(j / STAGES) & 1u, status);
     }
-    if ((warp == 10 || warp == 11) && lane == 0 && mma_used_sh[warp - 10]) {
+    if (warp >= MMA_WARP0 && lane == 0 && mma_used_sh[warp - MMA_WARP0]) {
       // one more commit: its arrival means every MMA of this thread has completed
-      mma_commit(drain(warp - 10));
-      mbar_wait(drain(warp - 10), 0, status);
+      mma_commit(drain(warp - MMA_WARP0));
+      mbar_wait(drain(warp - MMA_WARP0), 0, status);
     }
     fence_before();
     __syncthreads();
     fence_after();
   }
-  if (warp == 10) {
+  if (warp == MMA_WARP0) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
   }
 }

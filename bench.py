@@ -290,6 +290,21 @@ def attn_traffic(w):
         return None
 
 
+def max_over_ranks(ms, dist, dev):
+    """The slowest rank's time, on every rank (ms itself with one rank)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, flop_per_replica, ms):
+    """Whole-job TFLOP/s: every rank runs one replica in the max-over-ranks time."""
+    return world * flop_per_replica / (ms * 1e-3) / 1e12
+
+
 def cpu_cores():
     return len(os.sched_getaffinity(0))
 
@@ -420,15 +435,10 @@ def run_spark(a):
         raise RuntimeError("device status not OK after the timed steps")
     stage = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(4)]
 
-    t_max = total_ms
-    if dist is not None:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt.item())
-
+    t_max = max_over_ranks(total_ms, dist, dev)
     exact, comp, dense = flops(w, ksel)
     ms_per_layer = t_max / a.steps
-    value = world * dense / (ms_per_layer * 1e-3) / 1e12
+    value = job_throughput(world, dense, ms_per_layer)
 
     # dominant kernel: the attention (exact + compressed branches, one launch)
     attn_ms = stage[3]
@@ -462,11 +472,7 @@ def run_spark(a):
                 fwd()
             e1.record(stream)
             barrier()
-            ms = e0.elapsed_time(e1) / 3
-            if dist is not None:
-                tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-                dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-                ms = float(tt.item())
+            ms = max_over_ranks(e0.elapsed_time(e1) / 3, dist, dev)
             ex, cp, dn = flops(w, ks)
             sweep[str(r)] = {"ksel": ks, "ms_per_layer": round(ms, 3),
                              "eff_tflops": round(dn / (ms * 1e-3) / 1e12, 2),
@@ -490,12 +496,8 @@ def run_spark(a):
             spark.forward_host(p, qp, kp, vp, op, hws)
         e1.record(stream)
         barrier()
-        ms = e0.elapsed_time(e1) / ne
-        if dist is not None:
-            tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ms = float(tt.item())
-        e2e = {"value": world * dense / (ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms,
+        ms = max_over_ranks(e0.elapsed_time(e1) / ne, dist, dev)
+        e2e = {"value": job_throughput(world, dense, ms), "unit": UNIT, "ms_per_step": ms,
                "h2d_bytes_per_step": 3 * qh.nbytes, "d2h_bytes_per_step": qh.nbytes,
                "api": "spark_forward_host (pinned host buffers)"}
         del hws
